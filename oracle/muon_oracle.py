@@ -1,0 +1,158 @@
+"""fp64 CPU oracle for the batched Muon update (test infrastructure only).
+
+This module is the reference that the CUDA path is checked against.  Only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import it; the product path never does.  It shares no code with the CUDA
+library: it is a plain, slow restatement of the method in numpy, with one
+library primitive (the fp64 matrix product ``@``) as a step.
+
+Sources (page title, section):
+
+* DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销"
+  (hankli.space), section "Muon 核心：Newton-Schulz 迭代": normalise
+  G0 = G / ||G||_F, then G_{t+1} = 1.5 G_t - 0.5 G_t G_t^T G_t; the code
+  listing there transposes when rows > cols, adds 1e-7 to the norm and
+  transposes back at the end.
+* Same post, section "代码实现 / Vanilla Muon（Baseline，单 GPU）": momentum
+  buffer ``buf = momentum * buf + grad`` (multiply, then add), then
+  ``p -= lr * update``.
+* DMuon training guide "训练指南", section "超参数指南": Nesterov look-ahead
+  input is ``grad + momentum * buf``; ``weight_decay`` is a Muon parameter
+  (section "第 4 步：创建优化器") without a stated formula.
+
+Readings where the pages are silent (each listed in the design doc):
+
+* Nesterov uses the buffer *after* its update (the update is the first
+  statement of the step on the blog's Vanilla Muon).
+* Weight decay is decoupled and uses the pre-update weight:
+  W' = W (1 - lr wd) - lr X.
+* The per-parameter lr scale "0.2 sqrt(max(m, n))" mentioned in the guide's
+  hyper-parameter table is not applied (the blog's step uses plain ``-lr``).
+* The transpose test is strict (rows > cols), as in the blog listing.
+
+All pins that tie these functions to the pages and to mathematics live in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+#: Added to the Frobenius norm before dividing (blog, "Muon 核心" code listing).
+NORM_EPS = 1e-7
+#: Cubic Newton-Schulz coefficients (blog, "Muon 核心", G_{t+1} equation).
+NS_A = 1.5
+NS_B = -0.5
+
+
+def momentum_update(buf32: np.ndarray, g32: np.ndarray, mu: float) -> np.ndarray:
+    """Momentum buffer ``buf <- mu * buf + g`` in float32.
+
+    Blog, "代码实现 / Vanilla Muon": ``state['buf'].mul_(momentum).add_(grad)``.
+    Two separately rounded float32 operations (a product, then a sum), so the
+    result is fl32(fl32(mu * buf) + g), with no fused multiply-add.
+    """
+    buf32 = np.asarray(buf32, dtype=np.float32)
+    g32 = np.asarray(g32, dtype=np.float32)
+    mu32 = np.float32(mu)
+    prod = np.multiply(buf32, mu32, dtype=np.float32)
+    return np.add(prod, g32, dtype=np.float32)
+
+
+def nesterov_input(g32: np.ndarray, buf_new32: np.ndarray, mu: float,
+                   nesterov: bool) -> np.ndarray:
+    """Input of the orthogonalisation, in fp64.
+
+    Guide, "超参数指南" (nesterov row): ``ns_input = grad + mu * buf`` with the
+    already-updated buffer; without Nesterov the input is the buffer itself.
+    """
+    buf64 = np.asarray(buf_new32, dtype=np.float64)
+    if not nesterov:
+        return buf64
+    return np.asarray(g32, dtype=np.float64) + np.float64(np.float32(mu)) * buf64
+
+
+def frobenius_normalize(G: np.ndarray) -> np.ndarray:
+    """X0 = G / (||G||_F + 1e-7)  (blog, "Muon 核心", G_0 and the listing)."""
+    G = np.asarray(G, dtype=np.float64)
+    norm = np.sqrt(np.sum(G * G))
+    return G / (norm + NORM_EPS)
+
+
+def ns_iteration(X: np.ndarray) -> np.ndarray:
+    """One cubic step X <- 1.5 X - 0.5 (X X^T) X  (blog, "Muon 核心")."""
+    A = X @ X.T
+    return NS_A * X + NS_B * (A @ X)
+
+
+def newton_schulz(G: np.ndarray, steps: int) -> np.ndarray:
+    """Orthogonalise one 2-D matrix with ``steps`` cubic Newton-Schulz steps.
+
+    Blog, "Muon 核心" listing: transpose when rows > cols, normalise, iterate,
+    transpose back.  Returns fp64 with the input's shape.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    if G.ndim != 2:
+        raise ValueError("newton_schulz needs a 2-D matrix")
+    if steps < 0:
+        raise ValueError("steps must be >= 0")
+    transposed = G.shape[0] > G.shape[1]
+    X = G.T.copy() if transposed else G.copy()
+    X = frobenius_normalize(X)
+    for _ in range(steps):
+        X = ns_iteration(X)
+    return X.T.copy() if transposed else X
+
+
+def muon_weight_update(W: np.ndarray, X: np.ndarray, lr: float, wd: float) -> np.ndarray:
+    """W' = W (1 - lr wd) - lr X in fp64 (blog ``p.add_(update, alpha=-lr)``,
+    with decoupled weight decay as read above).  lr and wd are taken as the
+    float32 values a caller passes through the C ABI."""
+    lr64 = np.float64(np.float32(lr))
+    wd64 = np.float64(np.float32(wd))
+    return np.asarray(W, dtype=np.float64) * (1.0 - lr64 * wd64) - lr64 * X
+
+
+def muon_step(W, g, buf, *, lr: float, momentum: float, nesterov: bool,
+              weight_decay: float, ns_steps: int):
+    """One Muon update of one matrix.
+
+    Inputs are numpy arrays: ``W`` and ``g`` as float32 (bf16 values widen
+    exactly), ``buf`` float32.  Returns ``(buf_new float32, X fp64, W_new fp64)``.
+    """
+    buf_new = momentum_update(buf, g, momentum)
+    M = nesterov_input(g, buf_new, momentum, nesterov)
+    X = newton_schulz(M, ns_steps)
+    W_new = muon_weight_update(W, X, lr, weight_decay)
+    return buf_new, X, W_new
+
+
+def orthogonality_error(X: np.ndarray) -> float:
+    """||X X^T - I||_F measured on the short side of X.
+
+    Blog, "调试技巧" (check_orthogonality) uses the row Gram; for a tall
+    output that Gram is rank-deficient, so the short side is used instead.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if X.shape[0] > X.shape[1]:
+        X = X.T
+    R = X @ X.T
+    R[np.diag_indices_from(R)] -= 1.0
+    return float(np.sqrt(np.sum(R * R)))
+
+
+def relative_frobenius(a: np.ndarray, b: np.ndarray) -> float:
+    """||a - b||_F / ||b||_F (0 when both are zero)."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    den = np.sqrt(np.sum(b * b))
+    num = np.sqrt(np.sum((a - b) ** 2))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else float("inf")
+    return float(num / den)
+
+
+def ns_flops(rows: int, cols: int, steps: int) -> float:
+    """Useful Newton-Schulz FLOPs of one matrix: per step m^2 n for the
+    symmetric product X X^T and 2 m^2 n for (X X^T) X, m = min, n = max."""
+    m, n = min(rows, cols), max(rows, cols)
+    return float(steps) * 3.0 * m * m * n

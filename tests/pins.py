@@ -1,0 +1,263 @@
+"""Pins: facts fixed by the pages or by mathematics, used to check the oracle.
+
+Each ``pin_*`` function takes the oracle module (or a deliberately broken
+copy of it) and raises ``AssertionError`` when the implementation disagrees
+with the fact.  ``tests/test_oracle_pins.py`` runs them on the real oracle and
+shows that plausible mistakes planted in a copy of the oracle fail at least
+one of them.
+
+None of the expected values below is obtained by calling the function under
+test: they come from a scalar recurrence, an independent Jacobi SVD, exact
+rational arithmetic, or an algebraic identity.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+EPS = 1e-7   # blog "Muon 核心" listing: G / (G.norm() + 1e-7)
+
+
+# ----------------------------------------------------------------- helpers
+def cubic_map(s: float, k: int) -> float:
+    """f^k(s) for f(s) = 1.5 s - 0.5 s^3: the action of one cubic step on a
+    single singular value (blog, "Muon 核心" G_{t+1} equation applied to
+    G = U diag(s) V^T)."""
+    for _ in range(k):
+        s = 1.5 * s - 0.5 * s * s * s
+    return s
+
+
+def jacobi_svd(G: np.ndarray, tol: float = 1e-15, max_sweeps: int = 60):
+    """One-sided (Hestenes) Jacobi SVD written out by hand.
+
+    Returns U (p x r), sigma (r), V (q x r) with G = U diag(sigma) V^T, where
+    r = min(p, q).  Rotations orthogonalise the columns of the tall
+    orientation until every pair is orthogonal to ``tol``.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    flip = G.shape[0] < G.shape[1]
+    A = (G.T if flip else G).copy()
+    q = A.shape[1]
+    V = np.eye(q)
+    for _ in range(max_sweeps):
+        rotated = False
+        for i in range(q - 1):
+            for j in range(i + 1, q):
+                a = float(A[:, i] @ A[:, i])
+                b = float(A[:, j] @ A[:, j])
+                c = float(A[:, i] @ A[:, j])
+                if abs(c) <= tol * math.sqrt(a * b) or c == 0.0:
+                    continue
+                rotated = True
+                zeta = (b - a) / (2.0 * c)
+                t = math.copysign(1.0, zeta) / (abs(zeta) + math.sqrt(1.0 + zeta * zeta))
+                cs = 1.0 / math.sqrt(1.0 + t * t)
+                sn = cs * t
+                ai, aj = A[:, i].copy(), A[:, j].copy()
+                A[:, i] = cs * ai - sn * aj
+                A[:, j] = sn * ai + cs * aj
+                vi, vj = V[:, i].copy(), V[:, j].copy()
+                V[:, i] = cs * vi - sn * vj
+                V[:, j] = sn * vi + cs * vj
+        if not rotated:
+            break
+    sigma = np.sqrt(np.sum(A * A, axis=0))
+    U = np.zeros_like(A)
+    nz = sigma > 0
+    U[:, nz] = A[:, nz] / sigma[nz]
+    if flip:
+        return V, sigma, U
+    return U, sigma, V
+
+
+def _rel(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    d = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (d if d > 0 else 1.0))
+
+
+def _semi_orthogonal(rng, m: int, n: int) -> np.ndarray:
+    """An m x n matrix with orthonormal rows (m <= n)."""
+    Q, _ = np.linalg.qr(rng.standard_normal((n, m)))
+    return Q.T.copy()
+
+
+def exact_f32_round(x: Fraction) -> np.float32:
+    """Round an exact rational to the nearest float32, ties to even."""
+    guess = np.float32(float(x))
+    cands = {float(guess), float(np.nextafter(guess, np.float32(np.inf))),
+             float(np.nextafter(guess, np.float32(-np.inf)))}
+    best = None
+    for c in sorted(cands):
+        err = abs(Fraction(c) - x)
+        if best is None or err < best[0]:
+            best = (err, c)
+        elif err == best[0]:
+            # tie: keep the one with an even last mantissa bit
+            bits = np.array([c], dtype=np.float32).view(np.uint32)[0]
+            if bits & 1 == 0:
+                best = (err, c)
+    return np.float32(best[1])
+
+
+# -------------------------------------------------------------------- pins
+def pin_scalar_closed_form(o) -> None:
+    """A 1x1 input reduces to s0 = x / (|x| + 1e-7), s <- 1.5 s - 0.5 s^3."""
+    for x in (3.0, -2.5, 1e-6, -1e-7, 0.37, 0.0):
+        for k in (0, 1, 2, 5, 9):
+            got = o.newton_schulz(np.array([[x]]), k)[0, 0]
+            want = cubic_map(x / (abs(x) + EPS), k)
+            assert abs(got - want) <= 1e-15 * max(1.0, abs(want)), (x, k, got, want)
+
+
+def pin_spectral_map(o, seed: int = 11) -> None:
+    """For small random matrices (both orientations) the output equals
+    U diag(f^k(sigma / (||G||_F + 1e-7))) V^T, with U, sigma, V from a
+    hand-written Jacobi SVD: cubic NS is an odd matrix polynomial and acts on
+    each singular value independently."""
+    rng = np.random.default_rng(seed)
+    for (p, q) in ((1, 7), (5, 5), (7, 3), (12, 30), (30, 12), (48, 96), (17, 17)):
+        G = rng.standard_normal((p, q))
+        if p == q == 17:
+            G = np.triu(G) + 0.3 * np.eye(p)   # non-normal square input
+        U, sig, V = jacobi_svd(G)
+        nrm = math.sqrt(float(np.sum(G * G)))
+        for k in (1, 3, 5):
+            fs = np.array([cubic_map(s / (nrm + EPS), k) for s in sig])
+            want = (U * fs) @ V.T
+            got = o.newton_schulz(G, k)
+            assert got.shape == G.shape
+            assert _rel(got, want) <= 1e-12, (p, q, k, _rel(got, want))
+
+
+def pin_orthogonal_input(o, seed: int = 12) -> None:
+    """Orthogonal rows are a fixed point of the inner cubic step (f(1) = 1);
+    the full function maps c*Q to f^k(c / (c sqrt(m) + 1e-7)) * Q."""
+    rng = np.random.default_rng(seed)
+    for (m, n) in ((8, 8), (16, 40), (33, 64)):
+        Q = _semi_orthogonal(rng, m, n)
+        assert _rel(o.ns_iteration(Q), Q) <= 1e-14
+        for c in (1.0, 0.01, 50.0):
+            for k in (0, 1, 5):
+                s0 = c / (c * math.sqrt(m) + EPS)
+                want = cubic_map(s0, k) * Q
+                assert _rel(o.newton_schulz(c * Q, k), want) <= 1e-13
+                assert _rel(o.newton_schulz((c * Q).T, k), want.T) <= 1e-13
+
+
+def pin_monotone_error(o, seed: int = 13) -> None:
+    """||X X^T - I||_F does not increase with the step count: after
+    normalisation every singular value lies in [0, 1], where f is increasing
+    and f(s) >= s, so each value moves monotonically toward 1."""
+    rng = np.random.default_rng(seed)
+    cases = [rng.standard_normal((64, 128)),
+             _semi_orthogonal(rng, 32, 48) * rng.uniform(0.5, 1.0, size=(32, 1)),
+             rng.standard_normal((96, 40))]
+    for G in cases:
+        errs = []
+        for k in range(0, 12):
+            X = o.newton_schulz(G, k)
+            errs.append(o.orthogonality_error(X))
+        for a, b in zip(errs, errs[1:]):
+            assert b <= a + 1e-12, errs
+
+
+def pin_symmetries(o, seed: int = 14) -> None:
+    """NS(G^T) = NS(G)^T; NS(cG) = NS(G) for c > 0 far above the epsilon;
+    zero maps to zero; a rank-8 input with equal singular values follows the
+    scalar map from 1/sqrt(8)."""
+    rng = np.random.default_rng(seed)
+    G = rng.standard_normal((24, 56))
+    G *= 1e3 / np.linalg.norm(G)          # eps / ||G|| = 1e-10: far below the bound
+    assert _rel(o.newton_schulz(G.T, 5), o.newton_schulz(G, 5).T) <= 1e-13
+    assert _rel(o.newton_schulz(1000.0 * G, 5), o.newton_schulz(G, 5)) <= 1e-9
+    Z = o.newton_schulz(np.zeros((6, 9)), 5)
+    assert np.all(Z == 0.0)
+    U = _semi_orthogonal(rng, 8, 64).T           # 64 x 8, orthonormal columns
+    V = _semi_orthogonal(rng, 8, 96).T           # 96 x 8
+    R = U @ V.T                                   # rank 8, singular values 1
+    X = o.newton_schulz(R, 5)
+    want = cubic_map(1.0 / (math.sqrt(8.0) + EPS), 5) * R   # ||R||_F = sqrt(8)
+    assert _rel(X, want) <= 1e-13
+
+
+def pin_momentum_bitwise(o, seed: int = 15) -> None:
+    """buf' = fl32(fl32(mu * buf) + g): each value checked against exact
+    rational arithmetic rounded once per operation (blog, Vanilla Muon:
+    ``mul_(momentum)`` then ``add_(grad)``)."""
+    rng = np.random.default_rng(seed)
+    buf = (rng.standard_normal(300) * 10.0 ** rng.integers(-8, 4, 300)).astype(np.float32)
+    g = (rng.standard_normal(300) * 10.0 ** rng.integers(-8, 4, 300)).astype(np.float32)
+    buf[:3] = [0.0, -0.0, 1.0]
+    g[:3] = [0.0, 0.0, -0.95]
+    for mu in (0.95, 0.9, 0.5):
+        got = o.momentum_update(buf, g, mu)
+        assert got.dtype == np.float32
+        mu32 = Fraction(float(np.float32(mu)))
+        for i in range(buf.size):
+            p = exact_f32_round(mu32 * Fraction(float(buf[i])))
+            want = exact_f32_round(Fraction(float(p)) + Fraction(float(g[i])))
+            assert got[i].tobytes() == want.tobytes() or (got[i] == 0 and want == 0), (i, got[i], want)
+
+
+def pin_nesterov_post_update(o) -> None:
+    """Nesterov input uses the updated buffer: with mu = 0.5 and buf = -2 g
+    the updated buffer is exactly 0, so the input is g itself (it would be 0
+    with the pre-update buffer, and 2g - ... with no Nesterov)."""
+    rng = np.random.default_rng(16)
+    g = (rng.standard_normal((8, 12))).astype(np.float32)
+    buf = (-2.0 * g).astype(np.float32)
+    buf_new, X, _ = o.muon_step(np.zeros((8, 12), np.float32), g, buf, lr=0.1,
+                                momentum=0.5, nesterov=True, weight_decay=0.0, ns_steps=3)
+    assert np.all(buf_new == 0.0)
+    U, sig, V = jacobi_svd(g.astype(np.float64))
+    nrm = math.sqrt(float(np.sum(g.astype(np.float64) ** 2)))
+    want = (U * np.array([cubic_map(s / (nrm + EPS), 3) for s in sig])) @ V.T
+    assert _rel(X, want) <= 1e-12
+
+
+def _hadamard(n: int) -> np.ndarray:
+    """Sylvester Hadamard matrix of order n (a power of two)."""
+    H = np.array([[1.0]])
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def pin_update_closed_form(o, seed: int = 17) -> None:
+    """With g = c Q where Q has orthonormal rows made of +-1/4 entries (rows of
+    a 16x16 Hadamard matrix over 4, exact in float32), a zero buffer and
+    Nesterov, the input is (1 + mu) g, so X = f^k(sigma0) Q with
+    sigma0 = ||M|| / sqrt(m) / (||M|| + 1e-7), and W' = W (1 - lr wd) - lr X,
+    for wide, square and tall (transposed) matrices."""
+    rng = np.random.default_rng(seed)
+    H = _hadamard(16) / 4.0
+    for (m, tall) in ((8, False), (8, True), (16, False)):
+        Q = H[:m].copy()
+        c = 2.0 ** -9
+        g = (c * Q).astype(np.float32)
+        if tall:
+            g, Q = g.T.copy(), Q.T.copy()
+        W = (rng.standard_normal(g.shape) * 0.02).astype(np.float32)
+        lr, mu, wd, k = 0.02, 0.95, 0.01, 5
+        buf_new, X, Wn = o.muon_step(W, g, np.zeros_like(g), lr=lr, momentum=mu,
+                                     nesterov=True, weight_decay=wd, ns_steps=k)
+        assert np.array_equal(buf_new, g)
+        mu64 = float(np.float32(mu))
+        alpha = c + mu64 * c                  # every |M_ij| / |Q_ij| (one fp64 rounding)
+        nrm = alpha * math.sqrt(m)            # ||M||_F: m orthonormal rows scaled by alpha
+        sig0 = alpha / (nrm + EPS)
+        Xw = cubic_map(sig0, k) * Q
+        assert _rel(X, Xw) <= 1e-13, _rel(X, Xw)
+        lr64, wd64 = float(np.float32(lr)), float(np.float32(wd))
+        Ww = W.astype(np.float64) * (1.0 - lr64 * wd64) - lr64 * Xw
+        assert np.max(np.abs(Wn - Ww)) <= 1e-15
+
+
+ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
+            pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
+            pin_nesterov_post_update, pin_update_closed_form)

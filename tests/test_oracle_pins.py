@@ -1,0 +1,114 @@
+"""The oracle against facts the pages and mathematics fix (CPU only).
+
+Each pin in ``tests/pins.py`` runs on the oracle and must hold.  The
+mutation tests then plant one plausible mistake at a time in a copy of the
+oracle (on the CPU) and check that at least one pin catches it, which is what
+makes the pins worth trusting.
+"""
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import muon_oracle
+from tests import pins
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pin_holds(pin):
+    pin(oracle)
+
+
+def test_jacobi_svd_matches_lapack():
+    rng = np.random.default_rng(3)
+    for shape in ((5, 9), (9, 5), (16, 16)):
+        G = rng.standard_normal(shape)
+        U, s, V = pins.jacobi_svd(G)
+        assert np.allclose((U * s) @ V.T, G, atol=1e-13)
+        assert np.allclose(np.sort(s)[::-1], np.linalg.svd(G, compute_uv=False), atol=1e-13)
+
+
+def test_exact_rounding_helper():
+    from fractions import Fraction
+    assert pins.exact_f32_round(Fraction(1, 3)) == np.float32(1.0 / 3.0)
+    # 1 + 2^-24 is a tie between 1 and 1 + 2^-23: ties to even gives 1
+    assert pins.exact_f32_round(Fraction(1) + Fraction(1, 2 ** 24)) == np.float32(1.0)
+
+
+def _mutant(**overrides):
+    """A copy of the oracle module with some functions or constants replaced."""
+    m = types.ModuleType("mutant_oracle")
+    for k in dir(muon_oracle):
+        if not k.startswith("__"):
+            setattr(m, k, getattr(muon_oracle, k))
+    for k, v in overrides.items():
+        setattr(m, k, v)
+    # rebind the module-level helpers so that replaced pieces are used
+    def newton_schulz(G, steps):
+        G = np.asarray(G, dtype=np.float64)
+        transposed = G.shape[0] > G.shape[1]
+        X = G.T.copy() if transposed else G.copy()
+        X = m.frobenius_normalize(X)
+        for _ in range(steps):
+            X = m.ns_iteration(X)
+        return X.T.copy() if transposed else X
+
+    def muon_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps):
+        buf_new = m.momentum_update(buf, g, momentum)
+        M = m.nesterov_input(g, buf_new, momentum, nesterov)
+        X = m.newton_schulz(M, ns_steps)
+        return buf_new, X, m.muon_weight_update(W, X, lr, weight_decay)
+
+    if "newton_schulz" not in overrides:
+        m.newton_schulz = newton_schulz
+    if "muon_step" not in overrides:
+        m.muon_step = muon_step
+    return m
+
+
+def _no_eps(G):
+    G = np.asarray(G, dtype=np.float64)
+    n = np.sqrt(np.sum(G * G))
+    return G / n if n > 0 else G
+
+
+MUTANTS = {
+    "sign_of_cubic_term": dict(ns_iteration=lambda X: 1.5 * X + 0.5 * (X @ X.T) @ X),
+    "coefficient_3_not_1.5": dict(ns_iteration=lambda X: 3.0 * X - 0.5 * (X @ X.T) @ X),
+    # X^T X in place of X X^T: only expressible for square X (otherwise the
+    # shapes do not conform), where it differs unless X is normal.
+    "gram_of_columns": dict(ns_iteration=lambda X: 1.5 * X - 0.5 * ((X.T @ X) @ X if X.shape[0] == X.shape[1] else (X @ X.T) @ X)),
+    "one_step_short": dict(ns_iteration=lambda X: X),
+    "dropped_norm_eps": dict(frobenius_normalize=_no_eps),
+    "eps_on_squared_norm": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64) / np.sqrt(np.sum(np.asarray(G, np.float64) ** 2) + 1e-7)),
+    "no_normalisation": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64)),
+    "fma_momentum": dict(momentum_update=lambda b, g, mu: (np.float64(np.float32(mu)) * np.asarray(b, np.float64) + np.asarray(g, np.float64)).astype(np.float32)),
+    "lerp_momentum": dict(momentum_update=lambda b, g, mu: (np.float32(mu) * np.asarray(b, np.float32) + np.float32(1 - mu) * np.asarray(g, np.float32)).astype(np.float32)),
+    "nesterov_pre_update": dict(),   # filled below
+    "weight_decay_sign": dict(muon_weight_update=lambda W, X, lr, wd: np.asarray(W, np.float64) * (1.0 + float(np.float32(lr)) * float(np.float32(wd))) - float(np.float32(lr)) * X),
+    "update_sign": dict(muon_weight_update=lambda W, X, lr, wd: np.asarray(W, np.float64) * (1.0 - float(np.float32(lr)) * float(np.float32(wd))) + float(np.float32(lr)) * X),
+}
+
+
+def _pre_update_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps):
+    M = muon_oracle.nesterov_input(g, buf, momentum, nesterov)       # old buffer
+    buf_new = muon_oracle.momentum_update(buf, g, momentum)
+    X = muon_oracle.newton_schulz(M, ns_steps)
+    return buf_new, X, muon_oracle.muon_weight_update(W, X, lr, weight_decay)
+
+
+MUTANTS["nesterov_pre_update"] = dict(muon_step=_pre_update_step)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    m = _mutant(**MUTANTS[name])
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(m)
+        except (AssertionError, FloatingPointError, ValueError, ZeroDivisionError):
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passes every pin"
