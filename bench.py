@@ -1,0 +1,368 @@
+"""Benchmark of the batched Muon update (cubic Newton-Schulz) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+                    [--impl ours|reference]
+
+One step = one dmuon_muon_step_batched call over the whole workload (momentum,
+Nesterov, normalisation, k Newton-Schulz steps, weight update) with its
+inputs resident in HBM.  The metric is useful Newton-Schulz throughput: per
+matrix and NS step, m^2 n FLOPs for X X^T plus 2 m^2 n for (X X^T) X, with
+m = min(rows, cols), n = max(rows, cols).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of the
+workload (weak scaling, no collective on the data path); the step time is the
+maximum over ranks and `value` adds up all ranks' FLOPs.
+
+--impl reference times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload and in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "Muon-step ms & NS TFLOP/s (Llama-8B shapes), % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- dist
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_sample_specs(wl):
+    """A bounded sample of the workload for the fp64 oracle: the first layer's
+    attention projections for the Llama stack, else the first matrices, up to
+    about 2e12 useful FLOPs (10-30 s on a many-core host)."""
+    from newton_schulz_09_b200 import synthetic
+    budget = 2.2e12
+    chosen, fl = [], 0.0
+    order = range(len(wl.specs))
+    if wl.name == "llama8b":
+        order = [0, 1, 2, 3]          # layer 0: q, k, v, o
+    for i in order:
+        s = wl.specs[i]
+        f = 3.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) * wl.ns_steps
+        if chosen and fl + f > budget:
+            break
+        chosen.append(i)
+        fl += f
+    return chosen, fl
+
+
+def time_oracle(wl, subset):
+    """Runs the oracle's Muon step on host copies of the subset; returns
+    (seconds, threads)."""
+    import numpy as np
+    import oracle
+    from newton_schulz_09_b200 import synthetic
+    t = synthetic.make_tensors(wl, device="cpu", subset=subset)
+    host = [(p.float().numpy(), g.float().numpy(), b.numpy())
+            for p, g, b in zip(t.params, t.grads, t.bufs)]
+    threads = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info
+        info = [d for d in threadpool_info() if d.get("internal_api") == "openblas"]
+        if info:
+            threads = int(info[0]["num_threads"])
+    except Exception:
+        pass
+    t0 = time.perf_counter()
+    for W, g, b in host:
+        oracle.muon_step(W, g, b, lr=wl.lr, momentum=wl.momentum, nesterov=wl.nesterov,
+                         weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+    dt = time.perf_counter() - t0
+    del np
+    return dt, threads
+
+
+def cpu_baseline(wl):
+    subset, fl = cpu_sample_specs(wl)
+    secs, threads = time_oracle(wl, subset)
+    names = ",".join(f"{wl.specs[i].name}({wl.specs[i].rows}x{wl.specs[i].cols})" for i in subset)
+    return {"value": fl / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one Muon step (k={wl.ns_steps}) of {names}: {fl:.3e} useful NS FLOPs "
+                      f"in {secs:.2f} s, fp64 numpy/OpenBLAS"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from newton_schulz_09_b200 import synthetic
+    wl = synthetic.workload(args.workload)
+    subset, fl = cpu_sample_specs(wl)
+    for _ in range(max(0, args.warmup)):
+        pass   # the oracle has no warm-up state; each step is timed as it stands
+    secs = []
+    threads = 1
+    for _ in range(args.steps):
+        s, threads = time_oracle(wl, subset)
+        secs.append(s)
+    tot = sum(secs)
+    value = fl * len(secs) / tot / 1e12
+    names = ",".join(wl.specs[i].name for i in subset)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / len(secs) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "sample": names, "ns_steps": wl.ns_steps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"each step: one Muon step of {names} ({fl:.3e} FLOPs)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import newton_schulz_09_b200 as dm
+    from newton_schulz_09_b200 import synthetic
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    dm.load_library()
+    peaks, peak_src = load_peaks()
+
+    wl = synthetic.workload(args.workload)
+    t = synthetic.make_tensors(wl, device=dev, flat=True, seed_offset=rank)
+    stream = torch.cuda.current_stream(dev)
+    fl = synthetic.ns_flops(wl)
+
+    def step():
+        dm.dmuon_muon_step_batched(t.params, t.grads, t.bufs, lr=wl.lr, momentum=wl.momentum,
+                                   nesterov=wl.nesterov, weight_decay=wl.weight_decay,
+                                   ns_steps=wl.ns_steps)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    status = dm.dmuon_device_status()
+    if status != 0:
+        raise RuntimeError(f"device error word {status} after warm-up")
+
+    # ---- device-timed region (inputs resident in HBM, larger than L2)
+    sampler = ClockSampler(dev.index)
+    dm.dmuon_stage_times(reset=True)
+    dm.dmuon_stage_timing(True)
+    launches0 = dm.dmuon_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    launches = dm.dmuon_launch_count() - launches0
+    dm.dmuon_stage_timing(False)
+    stages = dm.dmuon_stage_times(reset=True)
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world, dev)
+    value = fl * world / (ms * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel (the GEMM stage: 2 m^2 n per step)
+    gemm_ms, gemm_n = stages["gemm"]
+    syrk_ms, syrk_n = stages["syrk"]
+    gemm_fl_per_launch = sum(2.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
+    syrk_fl_per_launch = sum(1.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
+    peak = peaks["bf16_tflops_sustained"]
+    gemm_tf = gemm_fl_per_launch / (gemm_ms / gemm_n * 1e-3) / 1e12 if gemm_n else None
+    syrk_tf = syrk_fl_per_launch / (syrk_ms / syrk_n * 1e-3) / 1e12 if syrk_n else None
+    roofline = {
+        "kernel": "ns_stage_kernel<GEMM, bf16>", "bound": "tensor",
+        "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
+        "frac": (gemm_tf / peak) if gemm_tf else None, "traffic": None,
+        "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+        "syrk": {"achieved": syrk_tf, "frac": (syrk_tf / peak) if syrk_tf else None},
+        "stage_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
+    }
+
+    # ---- end to end through the public API: pinned host grads in, weights out
+    e2e = None
+    if not args.no_e2e:
+        pflat, gflat, _ = t.flat
+        h_g = torch.empty(gflat.shape, dtype=gflat.dtype, pin_memory=True)
+        h_g.copy_(gflat)
+        h_w = torch.empty(pflat.shape, dtype=pflat.dtype, pin_memory=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            gflat.copy_(h_g, non_blocking=True)
+            step()
+            h_w.copy_(pflat, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps, world, dev)
+        e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": gflat.numel() * gflat.element_size(),
+               "d2h_bytes_per_step": pflat.numel() * pflat.element_size()}
+        del h_g, h_w
+
+    status = dm.dmuon_device_status()
+    if status != 0:
+        raise RuntimeError(f"device error word {status}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "pct_of_bf16_peak": {
+                "measured_sustained": value / world / peaks["bf16_tflops_sustained"],
+                "measured_burst": value / world / peaks["bf16_tflops"],
+                "nominal_2250": value / world / NOMINAL_BF16_TFLOPS,
+                "peak_source": peak_src},
+            "config": {"workload": wl.name, "matrices": len(wl.specs), "ns_steps": wl.ns_steps,
+                       "useful_ns_flops_per_step_per_gpu": fl,
+                       "l2": f"inputs larger than L2 ({wl.numel * 8 / 1e9:.0f} GB per GPU)",
+                       "parallelism": f"replicas x{world}"},
+            "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roofline, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

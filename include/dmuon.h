@@ -1,0 +1,182 @@
+/*
+ * dmuon.h -- C ABI of the B200 (sm_100a) batched Muon update.
+ *
+ * The method: for every 2-D weight matrix W with gradient g and fp32
+ * momentum buffer buf,
+ *   buf  <- momentum * buf + g                    (two fp32 roundings, no FMA)
+ *   M    <- g + momentum * buf   (Nesterov)   or   M <- buf
+ *   X0   <- M / (||M||_F + 1e-7), taken as its transpose when rows > cols
+ *   X    <- 1.5 X - 0.5 (X X^T) X                 (k times)
+ *   W    <- W (1 - lr * weight_decay) - lr * X    (X transposed back)
+ *
+ * Sources (page title, section):
+ *   DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销"
+ *     - "Muon 核心：Newton-Schulz 迭代": normalisation, the cubic step, and the
+ *       newton_schulz() listing (transpose when rows > cols, +1e-7 on the norm);
+ *     - "代码实现 / Vanilla Muon": momentum mul_/add_, the update p -= lr * X,
+ *       and skipping parameters without a gradient.
+ *   DMuon training guide "训练指南"
+ *     - "第 4 步：创建优化器" (lr, momentum, ns_steps, nesterov, weight_decay);
+ *     - "超参数指南" (Nesterov input grad + mu * buf).
+ * Weight decay is read as decoupled, on the pre-update weight (the guide
+ * names the parameter without a formula).
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are dense and row-major: element (r, c) at base[r * cols + c].
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *     the arrays of pointers / shapes themselves, which are HOST arrays read
+ *     during the call only.  Updated tensors are written in place.
+ *   - Calls are asynchronous: they only enqueue work on `stream` (a
+ *     cudaStream_t; NULL is the legacy default stream).  Device pointers must
+ *     stay valid until the stream reaches that work.
+ *   - Errors are returned before anything is enqueued; the message is in
+ *     dmuon_last_error() (per host thread).  NaN/Inf in the data propagate and
+ *     are not reported.
+ *   - The first call with a new set of shapes / pointers builds a launch plan
+ *     (host work plus one small synchronous upload); later identical calls
+ *     reuse it.  Make that first call before capturing a CUDA graph.
+ */
+#ifndef DMUON_H_
+#define DMUON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dmuon_stream_t; /* same type as cudaStream_t */
+
+/* Element types. */
+enum { DMUON_F32 = 0, DMUON_BF16 = 1 };
+
+/* Return codes (0 = success, negative = error, nothing was enqueued). */
+enum {
+  DMUON_OK = 0,
+  DMUON_ERR_INVALID_ARG = -1,  /* NULL pointer, size < 1, steps < 0, count < 0, misaligned element pointer */
+  DMUON_ERR_UNSUPPORTED = -2,  /* dtype, or a size beyond the limits below */
+  DMUON_ERR_NO_WORKSPACE = -3, /* workspace too small, or allocation failed */
+  DMUON_ERR_CUDA = -4,         /* a CUDA runtime call failed (see dmuon_last_error) */
+  DMUON_ERR_TIMEOUT = -5       /* a bounded device-side wait gave up (see dmuon_device_status) */
+};
+
+/* Size limits: min(rows, cols) <= DMUON_MAX_M, max(rows, cols) <= DMUON_MAX_N. */
+#define DMUON_MAX_M 32768
+#define DMUON_MAX_N (1 << 24)
+#define DMUON_MAX_STEPS 1000
+
+/* Shape and storage types of one matrix.  The momentum buffer is always fp32.
+ * param_dtype selects the arithmetic: bf16 parameters run the iteration with
+ * bf16 operands (fp32 accumulation); fp32 parameters use tf32 operands with
+ * fp32 storage. */
+typedef struct {
+  int64_t rows, cols;
+  int32_t param_dtype, grad_dtype;
+} dmuon_shape;
+
+/*
+ * dmuon_ns_orthogonalize -- Newton-Schulz orthogonalisation of one bf16
+ * matrix, in place: X <- NS_steps(X) with the normalisation and implicit
+ * transpose of the blog's newton_schulz() listing ("Muon 核心" section).
+ *   X       device pointer, rows x cols (m x n here) bf16, row-major; read and
+ *           overwritten with the result (same layout, bf16, round-to-nearest).
+ *   m, n    rows and cols, >= 1.
+ *   steps   number of cubic steps, >= 0 (0 returns the normalised input).
+ * Scratch memory comes from a library-owned per-stream arena (grown on
+ * demand with cudaMalloc, kept until dmuon_release_cache()).
+ */
+int dmuon_ns_orthogonalize(void* X, int64_t m, int64_t n, int steps, dmuon_stream_t stream);
+
+/* Same, with element type `dtype` (DMUON_BF16 or DMUON_F32) and
+ * caller-provided scratch of ws_bytes >= dmuon_ns_workspace_bytes(m, n, dtype)
+ * (device memory, any contents; it must not be used by anything else until
+ * the stream has finished the call). */
+int dmuon_ns_orthogonalize_ex(void* X, int64_t m, int64_t n, int steps, int dtype,
+                              void* workspace, size_t ws_bytes, dmuon_stream_t stream);
+size_t dmuon_ns_workspace_bytes(int64_t m, int64_t n, int dtype);
+
+/*
+ * dmuon_muon_step_batched -- one Muon update of `count` matrices, with one
+ * launch per stage for all of them (the per-parameter loop of the blog's
+ * Vanilla Muon, "代码实现" section, done as grouped kernels).
+ *   params[i]  device pointer to W_i (rows x cols, param_dtype), updated in place.
+ *   grads[i]   device pointer to g_i (rows x cols, grad_dtype), read only; NULL
+ *              skips matrix i entirely (no momentum, no update), as the blog
+ *              skips parameters whose grad is None.
+ *   bufs[i]    device pointer to the fp32 momentum buffer (rows x cols),
+ *              updated in place.
+ *   shapes[i]  host array, see dmuon_shape.
+ *   lr, momentum, weight_decay   scalars (fp32); nesterov != 0 enables the
+ *              Nesterov input; ns_steps >= 0.
+ * No two matrices may overlap in memory.  count == 0 is a no-op.
+ * Scratch as for dmuon_ns_orthogonalize.
+ */
+int dmuon_muon_step_batched(void* const params[], const void* const grads[], float* const bufs[],
+                            const dmuon_shape shapes[], int count, float lr, float momentum,
+                            int nesterov, float weight_decay, int ns_steps, dmuon_stream_t stream);
+
+/* Same with caller-provided scratch of ws_bytes >= dmuon_workspace_bytes(). */
+int dmuon_muon_step_batched_ex(void* const params[], const void* const grads[], float* const bufs[],
+                               const dmuon_shape shapes[], int count, float lr, float momentum,
+                               int nesterov, float weight_decay, int ns_steps, void* workspace,
+                               size_t ws_bytes, dmuon_stream_t stream);
+
+/* Scratch bytes needed by dmuon_muon_step_batched_ex for these shapes
+ * (matrices with a NULL gradient may be left out or counted; counting them
+ * over-estimates).  Returns 0 for invalid shapes. */
+size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps);
+
+/* Last error message of the calling host thread ("" if none). */
+const char* dmuon_last_error(void);
+
+/* Static description of the compiled backend, e.g.
+ * "cubic NS · tcgen05 SYRK+GEMM · sm_100a" (cf. the training guide's
+ * get_ns_backend() self-check in "日志与调试"). */
+const char* dmuon_backend_string(void);
+
+/* Device error word of the current device: 0 if no kernel reported a
+ * problem, else a DMUON_ERR_* code.  Synchronises the device first.
+ * clear != 0 resets the word to 0. */
+int dmuon_device_status(int clear);
+
+/* Frees the library's cached plans and scratch arenas (synchronises the
+ * device).  Safe to call at any time from the host. */
+void dmuon_release_cache(void);
+
+/* Kernel kinds reported by the timing and launch counters below. */
+enum {
+  DMUON_KERNEL_PROLOGUE = 0, /* momentum, Nesterov input, norm partials, copy into X */
+  DMUON_KERNEL_FINALIZE = 1, /* per-matrix norm and scale */
+  DMUON_KERNEL_SYRK = 2,     /* A = X X^T (upper tiles) */
+  DMUON_KERNEL_GEMM = 3,     /* X <- 1.5 X - 0.5 A X, last step fused with the update */
+  DMUON_KERNEL_APPLY = 4,    /* update for ns_steps == 0 */
+  DMUON_KERNEL_KINDS = 5
+};
+
+/* Per-kernel timing: while enabled, every launch is bracketed by CUDA events
+ * recorded on the caller's stream (so the numbers are device time of that
+ * stream).  dmuon_stage_times() synchronises the device, adds up the elapsed
+ * time of every bracketed launch since the last reset, and fills ms[k] and
+ * launches[k] for k < n (n <= DMUON_KERNEL_KINDS); reset != 0 clears them. */
+int dmuon_stage_timing(int enable);
+int dmuon_stage_times(double* ms, int64_t* launches, int n, int reset);
+
+/* Number of kernels this library has launched in this process. */
+int64_t dmuon_launch_count(void);
+
+/* Test hook: the next `n` library allocations fail as if the device were out
+ * of memory (host-side fault injection; 0 disables). */
+void dmuon_debug_fail_allocations(int n);
+
+/* Test hook: launches one CTA that waits on a barrier nothing arrives at,
+ * with a wait limit of `limit_us` microseconds, then records
+ * DMUON_ERR_TIMEOUT in the device error word and returns.  Exercises the
+ * bounded-wait path of the kernels without hanging the GPU. */
+int dmuon_debug_wait_timeout(int limit_us, dmuon_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMUON_H_ */

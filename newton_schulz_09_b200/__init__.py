@@ -1,0 +1,279 @@
+"""B200-native (sm_100a) batched Muon update: momentum, Nesterov, Frobenius
+normalisation, cubic Newton-Schulz and the decoupled weight update, done by
+hand-written tcgen05/TMA kernels behind the C ABI of ``include/dmuon.h``.
+
+This module is argument marshalling only: it passes tensor addresses, shapes
+and the current CUDA stream to ``libdmuon.so``.  Every step of the update
+runs in that library; there is no Python or CPU fallback, and the functions
+raise if the library or a CUDA device is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "DMUON_F32", "DMUON_BF16", "DmuonError", "load_library", "library_path",
+    "dmuon_ns_orthogonalize", "dmuon_ns_orthogonalize_ex", "dmuon_ns_workspace_bytes",
+    "dmuon_muon_step_batched", "dmuon_muon_step_batched_ex", "dmuon_workspace_bytes",
+    "dmuon_last_error", "dmuon_backend_string", "dmuon_device_status", "dmuon_release_cache",
+    "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
+    "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS",
+]
+
+#: Kernel kinds of dmuon_stage_times(), in order.
+KERNEL_KINDS = ("prologue", "finalize", "syrk", "gemm", "apply")
+
+DMUON_F32 = 0
+DMUON_BF16 = 1
+ERRORS = {0: "DMUON_OK", -1: "DMUON_ERR_INVALID_ARG", -2: "DMUON_ERR_UNSUPPORTED",
+          -3: "DMUON_ERR_NO_WORKSPACE", -4: "DMUON_ERR_CUDA", -5: "DMUON_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libdmuon.so")
+_lib = None
+
+
+class DmuonError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class DmuonShape(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("param_dtype", ctypes.c_int32), ("grad_dtype", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads libdmuon.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m newton_schulz_09_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, f32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                             ctypes.c_float, ctypes.c_size_t)
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    sp = ctypes.POINTER(DmuonShape)
+    sig = {
+        "dmuon_ns_orthogonalize": (i32, [vp, i64, i64, i32, vp]),
+        "dmuon_ns_orthogonalize_ex": (i32, [vp, i64, i64, i32, i32, vp, sz, vp]),
+        "dmuon_ns_workspace_bytes": (sz, [i64, i64, i32]),
+        "dmuon_muon_step_batched": (i32, [pp, pp, pp, sp, i32, f32, f32, i32, f32, i32, vp]),
+        "dmuon_muon_step_batched_ex": (i32, [pp, pp, pp, sp, i32, f32, f32, i32, f32, i32, vp, sz, vp]),
+        "dmuon_workspace_bytes": (sz, [sp, i32, i32]),
+        "dmuon_last_error": (ctypes.c_char_p, []),
+        "dmuon_backend_string": (ctypes.c_char_p, []),
+        "dmuon_device_status": (i32, [i32]),
+        "dmuon_release_cache": (None, []),
+        "dmuon_debug_fail_allocations": (None, [i32]),
+        "dmuon_debug_wait_timeout": (i32, [i32, vp]),
+        "dmuon_stage_timing": (i32, [i32]),
+        "dmuon_stage_times": (i32, [ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_int64), i32, i32]),
+        "dmuon_launch_count": (ctypes.c_int64, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(code: int) -> None:
+    if code != 0:
+        raise DmuonError(code, load_library().dmuon_last_error().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return DMUON_BF16
+    if t == torch.float32:
+        return DMUON_F32
+    raise TypeError(f"unsupported dtype {t}; use torch.bfloat16 or torch.float32")
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _cuda_matrix(t: torch.Tensor, what: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if t.dim() != 2:
+        raise ValueError(f"{what} must be 2-D (the Muon path is for matrices)")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous (row-major)")
+
+
+# ---------------------------------------------------------------- orthogonalise
+def dmuon_ns_workspace_bytes(m: int, n: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(load_library().dmuon_ns_workspace_bytes(m, n, _dtype_code(dtype)))
+
+
+def dmuon_ns_orthogonalize(X: torch.Tensor, steps: int = 5) -> torch.Tensor:
+    """In-place cubic Newton-Schulz of one bf16 matrix with library-owned scratch."""
+    lib = load_library()
+    _cuda_matrix(X, "X")
+    if X.dtype != torch.bfloat16:
+        raise TypeError("dmuon_ns_orthogonalize takes bf16; use dmuon_ns_orthogonalize_ex for fp32")
+    with torch.cuda.device(X.device):
+        _check(lib.dmuon_ns_orthogonalize(X.data_ptr(), X.shape[0], X.shape[1], steps,
+                                          _stream(X.device)))
+    return X
+
+
+def dmuon_ns_orthogonalize_ex(X: torch.Tensor, steps: int = 5,
+                              workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """In-place cubic Newton-Schulz of one bf16 or fp32 matrix; scratch comes
+    from ``workspace`` or from PyTorch's allocator."""
+    lib = load_library()
+    _cuda_matrix(X, "X")
+    dt = _dtype_code(X.dtype)
+    need = int(lib.dmuon_ns_workspace_bytes(X.shape[0], X.shape[1], dt))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib.dmuon_ns_orthogonalize_ex(X.data_ptr(), X.shape[0], X.shape[1], steps, dt,
+                                             workspace.data_ptr(), workspace.numel(),
+                                             _stream(X.device)))
+    return X
+
+
+# ---------------------------------------------------------------- Muon step
+class _Batch:
+    """ctypes arrays describing a list of matrices."""
+
+    def __init__(self, params, grads, bufs):
+        n = len(params)
+        if len(grads) != n or len(bufs) != n:
+            raise ValueError("params, grads and bufs must have the same length")
+        self.n = n
+        self.P = (ctypes.c_void_p * max(n, 1))()
+        self.G = (ctypes.c_void_p * max(n, 1))()
+        self.B = (ctypes.c_void_p * max(n, 1))()
+        self.S = (DmuonShape * max(n, 1))()
+        dev = None
+        for i, (p, g, b) in enumerate(zip(params, grads, bufs)):
+            _cuda_matrix(p, f"params[{i}]")
+            _cuda_matrix(b, f"bufs[{i}]")
+            if b.dtype != torch.float32 or b.shape != p.shape:
+                raise ValueError(f"bufs[{i}] must be fp32 with the parameter's shape")
+            if g is not None:
+                _cuda_matrix(g, f"grads[{i}]")
+                if g.shape != p.shape:
+                    raise ValueError(f"grads[{i}] must have the parameter's shape")
+            dev = dev or p.device
+            for t in (p, b) + ((g,) if g is not None else ()):
+                if t.device != dev:
+                    raise ValueError("all tensors must be on one device")
+            self.P[i] = p.data_ptr()
+            self.G[i] = g.data_ptr() if g is not None else None
+            self.B[i] = b.data_ptr()
+            gd = _dtype_code(g.dtype) if g is not None else _dtype_code(p.dtype)
+            self.S[i] = DmuonShape(p.shape[0], p.shape[1], _dtype_code(p.dtype), gd)
+        self.device = dev
+
+    def args(self):
+        pp = ctypes.POINTER(ctypes.c_void_p)
+        return (ctypes.cast(self.P, pp), ctypes.cast(self.G, pp), ctypes.cast(self.B, pp),
+                ctypes.cast(self.S, ctypes.POINTER(DmuonShape)), self.n)
+
+
+def dmuon_workspace_bytes(params: Sequence[torch.Tensor], ns_steps: int = 5,
+                          grads: Optional[Sequence[Optional[torch.Tensor]]] = None) -> int:
+    lib = load_library()
+    n = len(params)
+    S = (DmuonShape * max(n, 1))()
+    for i, p in enumerate(params):
+        g = grads[i] if grads is not None else None
+        gd = _dtype_code(g.dtype) if g is not None else _dtype_code(p.dtype)
+        S[i] = DmuonShape(p.shape[0], p.shape[1], _dtype_code(p.dtype), gd)
+    return int(lib.dmuon_workspace_bytes(S, n, ns_steps))
+
+
+def dmuon_muon_step_batched(params, grads, bufs, lr: float = 0.02, momentum: float = 0.95,
+                            nesterov: bool = True, weight_decay: float = 0.0,
+                            ns_steps: int = 5) -> None:
+    """One Muon update of all matrices, scratch from the library's arena."""
+    lib = load_library()
+    b = _Batch(params, grads, bufs)
+    if b.n == 0:
+        return
+    with torch.cuda.device(b.device):
+        _check(lib.dmuon_muon_step_batched(*b.args(), lr, momentum, 1 if nesterov else 0,
+                                           weight_decay, ns_steps, _stream(b.device)))
+
+
+def dmuon_muon_step_batched_ex(params, grads, bufs, lr: float = 0.02, momentum: float = 0.95,
+                               nesterov: bool = True, weight_decay: float = 0.0,
+                               ns_steps: int = 5,
+                               workspace: Optional[torch.Tensor] = None) -> None:
+    """One Muon update of all matrices; scratch from ``workspace`` (a uint8
+    CUDA tensor) or from PyTorch's allocator."""
+    lib = load_library()
+    b = _Batch(params, grads, bufs)
+    if b.n == 0:
+        return
+    need = dmuon_workspace_bytes(params, ns_steps, grads)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=b.device)
+    with torch.cuda.device(b.device):
+        _check(lib.dmuon_muon_step_batched_ex(*b.args(), lr, momentum, 1 if nesterov else 0,
+                                              weight_decay, ns_steps, workspace.data_ptr(),
+                                              workspace.numel(), _stream(b.device)))
+
+
+# ---------------------------------------------------------------- misc
+def dmuon_last_error() -> str:
+    return load_library().dmuon_last_error().decode()
+
+
+def dmuon_backend_string() -> str:
+    return load_library().dmuon_backend_string().decode()
+
+
+def dmuon_device_status(clear: bool = False) -> int:
+    return int(load_library().dmuon_device_status(1 if clear else 0))
+
+
+def dmuon_release_cache() -> None:
+    load_library().dmuon_release_cache()
+
+
+def dmuon_debug_fail_allocations(n: int) -> None:
+    load_library().dmuon_debug_fail_allocations(n)
+
+
+def dmuon_debug_wait_timeout(limit_us: int, device: Optional[torch.device] = None) -> None:
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(load_library().dmuon_debug_wait_timeout(limit_us, _stream(dev)))
+
+
+def dmuon_stage_timing(enable: bool) -> None:
+    _check(load_library().dmuon_stage_timing(1 if enable else 0))
+
+
+def dmuon_stage_times(reset: bool = False) -> dict:
+    """{kind: (milliseconds, launches)} accumulated while timing was enabled."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(load_library().dmuon_stage_times(ms, cnt, n, 1 if reset else 0))
+    return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def dmuon_launch_count() -> int:
+    return int(load_library().dmuon_launch_count())

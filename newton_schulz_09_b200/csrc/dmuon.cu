@@ -1,0 +1,841 @@
+// Host side of the batched Muon update: argument checks, launch plans,
+// scratch layout, TMA descriptors and the C ABI declared in include/dmuon.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "dmuon.h"
+#include "kernels.cuh"
+
+namespace dmuon {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+// ------------------------------------------------------------------ errors
+thread_local std::string t_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DMUON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+std::mutex g_mu;
+int g_fail_allocs = 0;
+
+cudaError_t lib_malloc(void** p, size_t bytes) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_fail_allocs > 0) {
+      --g_fail_allocs;
+      *p = nullptr;
+      return cudaErrorMemoryAllocation;
+    }
+  }
+  return cudaMalloc(p, bytes);
+}
+
+// ------------------------------------------------------------------ driver
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor: `inner` elements per row (contiguous), `outer` rows,
+// row pitch `pitch_elems`; box `box_inner` x `box_outer`, 128-byte swizzle,
+// zero fill out of bounds.
+bool encode_2d(CUtensorMap* map, int dtype, void* base, uint64_t inner, uint64_t outer,
+               uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int eb = dtype == DMUON_BF16 ? 2 : 4;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * eb};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype == DMUON_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ inputs
+struct MatIn {
+  void* W;
+  const void* G;
+  float* buf;
+  int64_t rows, cols;
+  int pdt, gdt;
+  int mode;
+};
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+int elem_bytes(int dt) { return dt == DMUON_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_matrix(const MatIn& x, int i) {
+  if (x.rows < 1 || x.cols < 1)
+    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: rows and cols must be >= 1 (got %lld x %lld)", i,
+                (long long)x.rows, (long long)x.cols);
+  if ((x.pdt != DMUON_BF16 && x.pdt != DMUON_F32) || (x.gdt != DMUON_BF16 && x.gdt != DMUON_F32))
+    return fail(DMUON_ERR_UNSUPPORTED, "matrix %d: dtype must be DMUON_BF16 or DMUON_F32", i);
+  const int64_t m = std::min(x.rows, x.cols), n = std::max(x.rows, x.cols);
+  if (m > DMUON_MAX_M || n > DMUON_MAX_N)
+    return fail(DMUON_ERR_UNSUPPORTED, "matrix %d: %lld x %lld exceeds the size limits", i,
+                (long long)x.rows, (long long)x.cols);
+  if (!x.W || !x.G)
+    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: NULL pointer", i);
+  if (x.mode == kModeMuon && !x.buf)
+    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: NULL momentum buffer", i);
+  if (!aligned(x.W, elem_bytes(x.pdt)) || !aligned(x.G, elem_bytes(x.gdt)) ||
+      (x.buf && !aligned(x.buf, 4)))
+    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: pointer not aligned to its element size", i);
+  return DMUON_OK;
+}
+
+// ------------------------------------------------------------------ layout
+// Scratch per matrix: X0 [, X1] [, A], then per group the tile partials and
+// the per-matrix scales.  Every region starts on a 1024-byte boundary.
+struct MatLayout {
+  int64_t m, n, ldx, lda;
+  size_t x0, x1, a;        // byte offsets in the workspace (x1/a = SIZE_MAX if unused)
+  size_t o0, o1;           // tf32 operand copies of X0/X1 (fp32 only; else == x0/x1)
+  int64_t ptiles, ptiles_c;
+};
+struct GroupLayout {
+  int dtype;
+  std::vector<int> idx;    // indices into the input matrix array
+  size_t partials, scales; // byte offsets
+  int64_t ptiles;
+};
+struct Layout {
+  std::vector<MatLayout> mats;   // parallel to the input matrices
+  std::vector<GroupLayout> groups;
+  size_t bytes = 0;
+};
+
+Layout make_layout(const std::vector<MatIn>& in, int steps) {
+  Layout L;
+  L.mats.resize(in.size());
+  size_t off = 0;
+  for (int dt : {DMUON_BF16, DMUON_F32}) {
+    GroupLayout g;
+    g.dtype = dt;
+    g.ptiles = 0;
+    for (size_t i = 0; i < in.size(); ++i)
+      if (in[i].pdt == dt) g.idx.push_back(static_cast<int>(i));
+    if (g.idx.empty()) continue;
+    const int eb = elem_bytes(dt);
+    const int64_t q = 16 / eb;   // 16-byte row pitch granularity
+    for (int i : g.idx) {
+      MatLayout& ml = L.mats[i];
+      ml.m = std::min(in[i].rows, in[i].cols);
+      ml.n = std::max(in[i].rows, in[i].cols);
+      ml.ldx = round_up(ml.n, q);
+      ml.lda = round_up(ml.m, q);
+      const size_t xb = static_cast<size_t>(ml.m) * ml.ldx * eb;
+      const size_t ab = static_cast<size_t>(ml.m) * ml.lda * eb;
+      ml.x0 = off; off = align_up(off + xb, 1024);
+      ml.x1 = SIZE_MAX; ml.a = SIZE_MAX;
+      if (steps >= 2) { ml.x1 = off; off = align_up(off + xb, 1024); }
+      ml.o0 = ml.x0; ml.o1 = ml.x1;
+      if (dt == DMUON_F32 && steps >= 1) {
+        ml.o0 = off; off = align_up(off + xb, 1024);
+        if (steps >= 2) { ml.o1 = off; off = align_up(off + xb, 1024); }
+      }
+      if (steps >= 1) { ml.a = off; off = align_up(off + ab, 1024); }
+      ml.ptiles_c = cdiv(in[i].cols, kPT);
+      ml.ptiles = cdiv(in[i].rows, kPT) * ml.ptiles_c;
+      g.ptiles += ml.ptiles;
+    }
+    g.partials = off; off = align_up(off + sizeof(float) * g.ptiles, 1024);
+    g.scales = off; off = align_up(off + sizeof(float) * g.idx.size(), 1024);
+    L.groups.push_back(std::move(g));
+  }
+  L.bytes = off;
+  return L;
+}
+
+// ------------------------------------------------------------------ plans
+struct GroupPlan {
+  int dtype;
+  int nmat;
+  int first;              // first MatDesc index of the group
+  int64_t ptiles;
+  int syrk_tiles, gemm_tiles;
+  const int* syrk_order; const int* syrk_prefix;
+  const int* gemm_order; const int* gemm_prefix;
+  const int64_t* pprefix;
+  float* partials;
+};
+
+struct Plan {
+  std::vector<uint8_t> key;
+  uint64_t hash = 0;
+  int device = 0;
+  void* dmem = nullptr;
+  const MatDesc* d_mats = nullptr;
+  const MatMaps* d_maps = nullptr;
+  std::vector<GroupPlan> groups;
+  ~Plan() {
+    if (dmem) cudaFree(dmem);
+  }
+};
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;
+};
+DeviceInfo g_dev[64];
+std::list<std::unique_ptr<Plan>> g_plans;   // most recently used first
+constexpr size_t kMaxPlans = 16;
+
+struct Arena {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Arena> g_arenas;
+
+uint64_t fnv1a(const uint8_t* p, size_t n) {
+  uint64_t h = 1469598103934665603ull;
+  for (size_t i = 0; i < n; ++i) { h ^= p[i]; h *= 1099511628211ull; }
+  return h;
+}
+
+template <typename T>
+void put(std::vector<uint8_t>& v, const T& x) {
+  const uint8_t* p = reinterpret_cast<const uint8_t*>(&x);
+  v.insert(v.end(), p, p + sizeof(T));
+}
+
+int device_setup(int dev) {
+  if (dev < 0 || dev >= 64) return fail(DMUON_ERR_CUDA, "device index %d out of range", dev);
+  DeviceInfo& d = g_dev[dev];
+  if (d.ready) return DMUON_OK;
+  cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(DMUON_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                major, minor);
+  e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+  const void* ks[] = {
+      reinterpret_cast<const void*>(&ns_stage_kernel<kSyrk, __nv_bfloat16>),
+      reinterpret_cast<const void*>(&ns_stage_kernel<kGemm, __nv_bfloat16>),
+      reinterpret_cast<const void*>(&ns_stage_kernel<kSyrk, float>),
+      reinterpret_cast<const void*>(&ns_stage_kernel<kGemm, float>)};
+  for (const void* k : ks) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+  }
+  if (!encode_fn()) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  d.ready = true;
+  return DMUON_OK;
+}
+
+// SYRK tiles of an m x m Gram: column bands of 256 with row bands 0..2J+1.
+int64_t syrk_tiles_of(int64_t m) {
+  const int64_t nJ = cdiv(m, kBN), nI = cdiv(m, kBM);
+  return (nJ - 1) * nJ + nI;
+}
+int64_t gemm_tiles_of(int64_t m, int64_t n) { return cdiv(m, kBM) * cdiv(n, kBN); }
+
+// Builds (or finds) the plan for these matrices and this workspace.
+int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** out) {
+  std::vector<uint8_t> key;
+  key.reserve(64 + in.size() * 56);
+  put(key, dev);
+  put(key, steps > 1 ? 2 : steps);
+  put(key, ws);
+  put(key, static_cast<int64_t>(in.size()));
+  for (const MatIn& x : in) {
+    put(key, x.W); put(key, x.G); put(key, x.buf);
+    put(key, x.rows); put(key, x.cols);
+    put(key, x.pdt); put(key, x.gdt); put(key, x.mode);
+  }
+  const uint64_t h = fnv1a(key.data(), key.size());
+  for (auto it = g_plans.begin(); it != g_plans.end(); ++it) {
+    if ((*it)->hash == h && (*it)->key == key) {
+      g_plans.splice(g_plans.begin(), g_plans, it);
+      *out = g_plans.front().get();
+      return DMUON_OK;
+    }
+  }
+
+  const Layout L = make_layout(in, steps);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const int nmat = static_cast<int>(in.size());
+
+  // Host image of the plan's device memory.
+  std::vector<MatDesc> descs(nmat);
+  std::vector<MatMaps> maps(nmat);
+  struct GroupArrays {
+    std::vector<int> so, sp, go, gp;
+    std::vector<int64_t> pp;
+  };
+  std::vector<GroupArrays> ga(L.groups.size());
+  std::unique_ptr<Plan> P(new Plan());
+  P->key = std::move(key);
+  P->hash = h;
+  P->device = dev;
+
+  int first = 0;
+  std::vector<int> desc_of(nmat, -1);
+  for (size_t gi = 0; gi < L.groups.size(); ++gi) {
+    const GroupLayout& g = L.groups[gi];
+    const int dt = g.dtype;
+    const int eb = elem_bytes(dt);
+    const int BK = 128 / eb;
+    GroupPlan gp{};
+    gp.dtype = dt;
+    gp.nmat = static_cast<int>(g.idx.size());
+    gp.first = first;
+    gp.ptiles = g.ptiles;
+    GroupArrays& A = ga[gi];
+    A.pp.push_back(0);
+    for (int k = 0; k < gp.nmat; ++k) {
+      const int i = g.idx[k];
+      const MatIn& x = in[i];
+      const MatLayout& ml = L.mats[i];
+      MatDesc& d = descs[first + k];
+      desc_of[i] = first + k;
+      std::memset(&d, 0, sizeof(d));
+      d.W = x.W; d.G = x.G; d.buf = x.buf;
+      d.rows = x.rows; d.cols = x.cols;
+      d.ldx = ml.ldx; d.lda = ml.lda;
+      d.X[0] = wsb + ml.x0;
+      d.X[1] = (ml.x1 != SIZE_MAX) ? wsb + ml.x1 : nullptr;
+      d.Xop[0] = wsb + ml.o0;
+      d.Xop[1] = (ml.o1 != SIZE_MAX) ? wsb + ml.o1 : nullptr;
+      d.A = (ml.a != SIZE_MAX) ? wsb + ml.a : nullptr;
+      d.scale = reinterpret_cast<float*>(wsb + g.scales) + k;
+      d.lr_mult = 1.0f;
+      d.m = static_cast<int>(ml.m); d.n = static_cast<int>(ml.n);
+      d.T = x.rows > x.cols ? 1 : 0;
+      d.mode = x.mode;
+      d.g_bf16 = x.gdt == DMUON_BF16 ? 1 : 0;
+      d.vec4 = (x.cols % 4 == 0) && aligned(x.W, 16) && aligned(x.G, 16) &&
+               (x.buf == nullptr || aligned(x.buf, 16));
+      d.ptiles_c = static_cast<int>(ml.ptiles_c);
+      A.pp.push_back(A.pp.back() + ml.ptiles);
+      if (ws) {
+        MatMaps& mm = maps[first + k];
+        std::memset(&mm, 0, sizeof(mm));
+        bool okm = true;
+        for (int b = 0; b < 2; ++b) {
+          void* xb = d.Xop[b];
+          if (!xb) { mm.xk[b] = mm.xk[0]; mm.xmn[b] = mm.xmn[0]; continue; }
+          okm &= encode_2d(&mm.xk[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBM);
+          // MN-major 32-bit operands need 32-byte swizzle units.
+          okm &= encode_2d(&mm.xmn[b], dt, xb, ml.n, ml.m, ml.ldx, BK, BK,
+                           dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                           : CU_TENSOR_MAP_SWIZZLE_128B);
+        }
+        if (d.A) okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+        if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed for matrix %d", i);
+      }
+    }
+    // Longest K first: SYRK contracts over n, the GEMM over m.
+    std::vector<int> ord(gp.nmat);
+    for (int k = 0; k < gp.nmat; ++k) ord[k] = k;
+    std::vector<int> so = ord, go = ord;
+    std::stable_sort(so.begin(), so.end(), [&](int a, int b) {
+      const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
+      return x.n != y.n ? x.n > y.n : x.m > y.m;
+    });
+    std::stable_sort(go.begin(), go.end(), [&](int a, int b) {
+      const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
+      return x.m != y.m ? x.m > y.m : x.n > y.n;
+    });
+    int64_t st = 0, gt = 0;
+    A.sp.push_back(0);
+    A.gp.push_back(0);
+    for (int k = 0; k < gp.nmat; ++k) {
+      st += syrk_tiles_of(descs[first + so[k]].m);
+      gt += gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
+      A.sp.push_back(static_cast<int>(st));
+      A.gp.push_back(static_cast<int>(gt));
+    }
+    if (st > INT32_MAX || gt > INT32_MAX)
+      return fail(DMUON_ERR_UNSUPPORTED, "too many tiles in one launch");
+    A.so = so; A.go = go;
+    gp.syrk_tiles = static_cast<int>(st);
+    gp.gemm_tiles = static_cast<int>(gt);
+    gp.partials = reinterpret_cast<float*>(wsb + g.partials);
+    P->groups.push_back(gp);
+    first += gp.nmat;
+  }
+
+  // Pack: descs | maps | per group (pprefix, syrk order/prefix, gemm order/prefix).
+  size_t off = 0;
+  const size_t o_desc = off; off = align_up(off + sizeof(MatDesc) * nmat, 128);
+  const size_t o_maps = off; off = align_up(off + sizeof(MatMaps) * nmat, 128);
+  std::vector<size_t> o_g(ga.size() * 5);
+  for (size_t gi = 0; gi < ga.size(); ++gi) {
+    o_g[gi * 5 + 0] = off; off = align_up(off + sizeof(int64_t) * ga[gi].pp.size(), 128);
+    o_g[gi * 5 + 1] = off; off = align_up(off + sizeof(int) * ga[gi].so.size(), 128);
+    o_g[gi * 5 + 2] = off; off = align_up(off + sizeof(int) * ga[gi].sp.size(), 128);
+    o_g[gi * 5 + 3] = off; off = align_up(off + sizeof(int) * ga[gi].go.size(), 128);
+    o_g[gi * 5 + 4] = off; off = align_up(off + sizeof(int) * ga[gi].gp.size(), 128);
+  }
+  std::vector<uint8_t> img(off, 0);
+  std::memcpy(img.data() + o_desc, descs.data(), sizeof(MatDesc) * nmat);
+  std::memcpy(img.data() + o_maps, maps.data(), sizeof(MatMaps) * nmat);
+  for (size_t gi = 0; gi < ga.size(); ++gi) {
+    std::memcpy(img.data() + o_g[gi * 5 + 0], ga[gi].pp.data(), sizeof(int64_t) * ga[gi].pp.size());
+    std::memcpy(img.data() + o_g[gi * 5 + 1], ga[gi].so.data(), sizeof(int) * ga[gi].so.size());
+    std::memcpy(img.data() + o_g[gi * 5 + 2], ga[gi].sp.data(), sizeof(int) * ga[gi].sp.size());
+    std::memcpy(img.data() + o_g[gi * 5 + 3], ga[gi].go.data(), sizeof(int) * ga[gi].go.size());
+    std::memcpy(img.data() + o_g[gi * 5 + 4], ga[gi].gp.data(), sizeof(int) * ga[gi].gp.size());
+  }
+  cudaError_t e = lib_malloc(&P->dmem, img.size());
+  if (e != cudaSuccess) {
+    P->dmem = nullptr;
+    return fail(DMUON_ERR_NO_WORKSPACE, "plan allocation of %zu bytes failed", img.size());
+  }
+  e = cudaMemcpy(P->dmem, img.data(), img.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "plan upload");
+  uint8_t* base = static_cast<uint8_t*>(P->dmem);
+  for (size_t gi = 0; gi < P->groups.size(); ++gi) {
+    GroupPlan& gp = P->groups[gi];
+    gp.pprefix = reinterpret_cast<const int64_t*>(base + o_g[gi * 5 + 0]);
+    gp.syrk_order = reinterpret_cast<const int*>(base + o_g[gi * 5 + 1]);
+    gp.syrk_prefix = reinterpret_cast<const int*>(base + o_g[gi * 5 + 2]);
+    gp.gemm_order = reinterpret_cast<const int*>(base + o_g[gi * 5 + 3]);
+    gp.gemm_prefix = reinterpret_cast<const int*>(base + o_g[gi * 5 + 4]);
+  }
+  P->d_mats = reinterpret_cast<const MatDesc*>(base + o_desc);
+  P->d_maps = reinterpret_cast<const MatMaps*>(base + o_maps);
+  g_plans.emplace_front(std::move(P));
+  Plan* plan = g_plans.front().get();
+  while (g_plans.size() > kMaxPlans) {
+    cudaDeviceSynchronize();   // an evicted plan may still be read by queued kernels
+    g_plans.pop_back();
+  }
+  *out = plan;
+  return DMUON_OK;
+}
+
+// ------------------------------------------------------------------ launch
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per bounded device wait
+
+// Launch bookkeeping: a process-wide launch counter and, when enabled,
+// CUDA-event brackets around each launch for per-kernel device time.
+int64_t g_launches = 0;
+bool g_timing = false;
+struct Bracket {
+  cudaEvent_t a, b;
+  int kind;
+};
+std::vector<Bracket> g_brackets;       // recorded, not yet harvested
+std::vector<cudaEvent_t> g_event_pool;
+double g_kind_ms[DMUON_KERNEL_KINDS] = {0};
+int64_t g_kind_n[DMUON_KERNEL_KINDS] = {0};
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct LaunchScope {
+  cudaStream_t st;
+  int kind;
+  cudaEvent_t a = nullptr;
+  LaunchScope(cudaStream_t s, int k) : st(s), kind(k) {
+    ++g_launches;
+    if (g_timing) {
+      a = pool_event();
+      cudaEventRecord(a, st);
+    }
+  }
+  ~LaunchScope() {
+    if (a) {
+      cudaEvent_t b = pool_event();
+      cudaEventRecord(b, st);
+      g_brackets.push_back(Bracket{a, b, kind});
+    }
+  }
+};
+
+template <typename E>
+void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float lr, float mu,
+                  int nesterov, float wd, int steps, cudaStream_t st) {
+  ElemParams ep;
+  ep.mats = P.d_mats + g.first;
+  ep.ptile_prefix = g.pprefix;
+  ep.partials = g.partials;
+  ep.nmat = g.nmat;
+  ep.ntiles = g.ptiles;
+  ep.mu = mu;
+  ep.nesterov = nesterov;
+  ep.lr = lr;
+  ep.wd = wd;
+  const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
+  {
+    LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
+    prologue_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+  }
+  {
+    LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
+    finalize_kernel<<<g.nmat, 32, 0, st>>>(ep);
+  }
+  if (steps == 0) {
+    LaunchScope ls(st, DMUON_KERNEL_APPLY);
+    apply_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+    return;
+  }
+  NsParams np;
+  np.mats = P.d_mats + g.first;
+  np.maps = P.d_maps + g.first;
+  np.nmat = g.nmat;
+  np.lr = lr;
+  np.wd = wd;
+  np.err = d.err;
+  np.wait_limit_ns = kWaitLimitNs;
+  for (int s = 0; s < steps; ++s) {
+    np.cur = s & 1;
+    np.first = s == 0;
+    np.last = s == steps - 1;
+    np.order = g.syrk_order;
+    np.tile_prefix = g.syrk_prefix;
+    np.ntiles = g.syrk_tiles;
+    {
+      LaunchScope ls(st, DMUON_KERNEL_SYRK);
+      ns_stage_kernel<kSyrk, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+    }
+    np.order = g.gemm_order;
+    np.tile_prefix = g.gemm_prefix;
+    np.ntiles = g.gemm_tiles;
+    {
+      LaunchScope ls(st, DMUON_KERNEL_GEMM);
+      ns_stage_kernel<kGemm, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+    }
+  }
+}
+
+int launch_plan(const Plan& P, float lr, float mu, int nesterov, float wd, int steps,
+                cudaStream_t st) {
+  const DeviceInfo& d = g_dev[P.device];
+  for (const GroupPlan& g : P.groups) {
+    if (g.dtype == DMUON_BF16) launch_group<__nv_bfloat16>(P, g, d, lr, mu, nesterov, wd, steps, st);
+    else launch_group<float>(P, g, d, lr, mu, nesterov, wd, steps, st);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return DMUON_OK;
+}
+
+std::mutex g_api_mu;
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  return device_setup(*dev);
+}
+
+int arena_get(int dev, cudaStream_t st, size_t bytes, void** out) {
+  Arena& a = g_arenas[std::make_pair(dev, st)];
+  if (a.bytes < bytes) {
+    if (a.ptr) {
+      cudaStreamSynchronize(st);
+      cudaFree(a.ptr);
+      a.ptr = nullptr;
+      a.bytes = 0;
+    }
+    cudaError_t e = lib_malloc(&a.ptr, bytes);
+    if (e != cudaSuccess) {
+      a.ptr = nullptr;
+      cudaGetLastError();
+      return fail(DMUON_ERR_NO_WORKSPACE, "scratch allocation of %zu bytes failed", bytes);
+    }
+    a.bytes = bytes;
+  }
+  *out = a.ptr;
+  return DMUON_OK;
+}
+
+int gather(void* const params[], const void* const grads[], float* const bufs[],
+           const dmuon_shape shapes[], int count, int ns_steps, std::vector<MatIn>* in) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count must be >= 0");
+  if (ns_steps < 0 || ns_steps > DMUON_MAX_STEPS)
+    return fail(DMUON_ERR_INVALID_ARG, "ns_steps must be in [0, %d]", DMUON_MAX_STEPS);
+  if (count == 0) return DMUON_OK;
+  if (!params || !grads || !bufs || !shapes)
+    return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  in->reserve(count);
+  for (int i = 0; i < count; ++i) {
+    if (grads[i] == nullptr) continue;   // no gradient: skipped
+    MatIn x;
+    x.W = params[i];
+    x.G = grads[i];
+    x.buf = bufs[i];
+    x.rows = shapes[i].rows;
+    x.cols = shapes[i].cols;
+    x.pdt = shapes[i].param_dtype;
+    x.gdt = shapes[i].grad_dtype;
+    x.mode = kModeMuon;
+    const int r = check_matrix(x, i);
+    if (r != DMUON_OK) return r;
+    in->push_back(x);
+  }
+  return DMUON_OK;
+}
+
+int run(const std::vector<MatIn>& in, int steps, void* ws, size_t ws_bytes, bool own_ws,
+        float lr, float mu, int nesterov, float wd, cudaStream_t st) {
+  if (in.empty()) return DMUON_OK;
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  int r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  const size_t need = make_layout(in, steps).bytes;
+  if (own_ws) {
+    r = arena_get(dev, st, need, &ws);
+    if (r != DMUON_OK) return r;
+  } else {
+    if (!ws) return fail(DMUON_ERR_INVALID_ARG, "NULL workspace");
+    if (ws_bytes < need)
+      return fail(DMUON_ERR_NO_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed",
+                  ws_bytes, need);
+    if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  Plan* plan = nullptr;
+  r = get_plan(in, steps, ws, dev, &plan);
+  if (r != DMUON_OK) return r;
+  return launch_plan(*plan, lr, mu, nesterov, wd, steps, st);
+}
+
+}  // namespace
+}  // namespace dmuon
+
+using namespace dmuon;
+
+extern "C" {
+
+int dmuon_muon_step_batched_ex(void* const params[], const void* const grads[], float* const bufs[],
+                               const dmuon_shape shapes[], int count, float lr, float momentum,
+                               int nesterov, float weight_decay, int ns_steps, void* workspace,
+                               size_t ws_bytes, dmuon_stream_t stream) {
+  t_last_error.clear();
+  std::vector<MatIn> in;
+  int r = gather(params, grads, bufs, shapes, count, ns_steps, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, ns_steps, workspace, ws_bytes, false, lr, momentum, nesterov ? 1 : 0, weight_decay,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dmuon_muon_step_batched(void* const params[], const void* const grads[], float* const bufs[],
+                            const dmuon_shape shapes[], int count, float lr, float momentum,
+                            int nesterov, float weight_decay, int ns_steps, dmuon_stream_t stream) {
+  t_last_error.clear();
+  std::vector<MatIn> in;
+  int r = gather(params, grads, bufs, shapes, count, ns_steps, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, ns_steps, nullptr, 0, true, lr, momentum, nesterov ? 1 : 0, weight_decay,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps) {
+  if (count <= 0 || !shapes || ns_steps < 0 || ns_steps > DMUON_MAX_STEPS) return 0;
+  std::vector<MatIn> in(count);
+  for (int i = 0; i < count; ++i) {
+    MatIn& x = in[i];
+    x.W = x.buf = nullptr;
+    x.G = nullptr;
+    x.rows = shapes[i].rows;
+    x.cols = shapes[i].cols;
+    x.pdt = shapes[i].param_dtype;
+    x.gdt = shapes[i].grad_dtype;
+    x.mode = kModeMuon;
+    if (x.rows < 1 || x.cols < 1 || (x.pdt != DMUON_BF16 && x.pdt != DMUON_F32)) return 0;
+  }
+  return make_layout(in, ns_steps).bytes;
+}
+
+static int ortho_input(void* X, int64_t m, int64_t n, int steps, int dtype, std::vector<MatIn>* in) {
+  if (steps < 0 || steps > DMUON_MAX_STEPS)
+    return fail(DMUON_ERR_INVALID_ARG, "steps must be in [0, %d]", DMUON_MAX_STEPS);
+  MatIn x;
+  x.W = X;
+  x.G = X;
+  x.buf = nullptr;
+  x.rows = m;
+  x.cols = n;
+  x.pdt = dtype;
+  x.gdt = dtype;
+  x.mode = kModeOrtho;
+  const int r = check_matrix(x, 0);
+  if (r != DMUON_OK) return r;
+  in->push_back(x);
+  return DMUON_OK;
+}
+
+int dmuon_ns_orthogonalize_ex(void* X, int64_t m, int64_t n, int steps, int dtype, void* workspace,
+                              size_t ws_bytes, dmuon_stream_t stream) {
+  t_last_error.clear();
+  std::vector<MatIn> in;
+  int r = ortho_input(X, m, n, steps, dtype, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, steps, workspace, ws_bytes, false, 0.0f, 0.0f, 0, 0.0f,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dmuon_ns_orthogonalize(void* X, int64_t m, int64_t n, int steps, dmuon_stream_t stream) {
+  t_last_error.clear();
+  std::vector<MatIn> in;
+  int r = ortho_input(X, m, n, steps, DMUON_BF16, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, steps, nullptr, 0, true, 0.0f, 0.0f, 0, 0.0f,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dmuon_ns_workspace_bytes(int64_t m, int64_t n, int dtype) {
+  if (m < 1 || n < 1 || (dtype != DMUON_BF16 && dtype != DMUON_F32)) return 0;
+  std::vector<MatIn> in(1);
+  in[0].rows = m;
+  in[0].cols = n;
+  in[0].pdt = in[0].gdt = dtype;
+  in[0].mode = kModeOrtho;
+  return make_layout(in, 2).bytes;
+}
+
+const char* dmuon_last_error(void) { return t_last_error.c_str(); }
+
+const char* dmuon_backend_string(void) {
+  return "cubic Newton-Schulz · tcgen05 UMMA 128x256 SYRK (upper tiles) + GEMM (fused combine/update) "
+         "· TMA 128B-swizzle · TMEM double buffer · sm_100a";
+}
+
+int dmuon_device_status(int clear) {
+  t_last_error.clear();
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  return v;
+}
+
+void dmuon_release_cache(void) {
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  cudaDeviceSynchronize();
+  g_plans.clear();
+  for (auto& kv : g_arenas)
+    if (kv.second.ptr) cudaFree(kv.second.ptr);
+  g_arenas.clear();
+}
+
+int dmuon_stage_timing(int enable) {
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  g_timing = enable != 0;
+  return DMUON_OK;
+}
+
+int dmuon_stage_times(double* ms, int64_t* launches, int n, int reset) {
+  t_last_error.clear();
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  for (const Bracket& br : g_brackets) {
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, br.a, br.b) == cudaSuccess) {
+      g_kind_ms[br.kind] += t;
+      g_kind_n[br.kind] += 1;
+    }
+    g_event_pool.push_back(br.a);
+    g_event_pool.push_back(br.b);
+  }
+  g_brackets.clear();
+  for (int k = 0; k < n && k < DMUON_KERNEL_KINDS; ++k) {
+    if (ms) ms[k] = g_kind_ms[k];
+    if (launches) launches[k] = g_kind_n[k];
+  }
+  if (reset)
+    for (int k = 0; k < DMUON_KERNEL_KINDS; ++k) { g_kind_ms[k] = 0.0; g_kind_n[k] = 0; }
+  return DMUON_OK;
+}
+
+int64_t dmuon_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  return g_launches;
+}
+
+void dmuon_debug_fail_allocations(int n) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_fail_allocs = n > 0 ? n : 0;
+}
+
+int dmuon_debug_wait_timeout(int limit_us, dmuon_stream_t stream) {
+  t_last_error.clear();
+  if (limit_us < 1 || limit_us > 10000000)
+    return fail(DMUON_ERR_INVALID_ARG, "limit_us must be in [1, 1e7]");
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  int r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  ++g_launches;
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      g_dev[dev].err, static_cast<uint64_t>(limit_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return DMUON_OK;
+}
+
+}  // extern "C"

@@ -158,33 +158,60 @@ class Tensors:
     grads: List[torch.Tensor]
     bufs: List[torch.Tensor]
     prior_grads: List[List[torch.Tensor]]   # [step][matrix], empty unless prior_steps > 0
+    flat: Optional[tuple] = None             # (params, grads, bufs) flat storage when drawn flat
 
 
 def make_tensors(wl: Workload, device="cpu", subset: Optional[Sequence[int]] = None,
-                 draw_grads: bool = True) -> Tensors:
+                 draw_grads: bool = True, flat: bool = False, seed_offset: int = 0) -> Tensors:
     """Draw the workload's tensors on ``device``.
 
     Every matrix gets its own generator seeded from (workload seed, index), so
     a subset draws exactly the tensors the full workload would.  Momentum
     buffers start at zero; workloads with a momentum history carry
-    ``prior_steps`` extra gradient sets to be applied first.
+    ``prior_steps`` extra gradient sets to be applied first.  ``flat`` places
+    each kind (weights, gradients, buffers) in one contiguous allocation, the
+    matrices being views into it; ``seed_offset`` draws an independent copy.
     """
     idx = list(range(len(wl.specs))) if subset is None else list(subset)
     params, grads, bufs = [], [], []
     prior = [[] for _ in range(wl.prior_steps)]
+    if flat:
+        tot = sum(wl.specs[i].numel for i in idx)
+        pflat = torch.empty(tot, dtype=wl.dtype, device=device)
+        gflat = torch.empty(tot, dtype=wl.dtype, device=device) if draw_grads else None
+        bflat = torch.zeros(tot, dtype=torch.float32, device=device)
+    off = 0
     for i in idx:
         spec = wl.specs[i]
-        gen = _gen(wl.seed * 1_000_003 + i, device)
-        w = torch.empty((spec.rows, spec.cols), dtype=torch.float32, device=device)
+        shape = (spec.rows, spec.cols)
+        gen = _gen(wl.seed * 1_000_003 + i + 7_919 * seed_offset, device)
+        w = torch.empty(shape, dtype=torch.float32, device=device)
         w.normal_(0.0, wl.w_std, generator=gen)
-        params.append(w.to(wl.dtype))
+        if flat:
+            params.append(pflat[off:off + spec.numel].view(shape))
+            params[-1].copy_(w)
+        else:
+            params.append(w.to(wl.dtype))
         del w
         for s in range(wl.prior_steps):
             prior[s].append(_draw_grad(spec, wl.grad_std, wl.dtype, device, gen))
         if draw_grads:
-            grads.append(_draw_grad(spec, wl.grad_std, wl.dtype, device, gen))
-        bufs.append(torch.zeros((spec.rows, spec.cols), dtype=torch.float32, device=device))
-    return Tensors(params, grads, bufs, prior)
+            g = _draw_grad(spec, wl.grad_std, wl.dtype, device, gen)
+            if flat:
+                grads.append(gflat[off:off + spec.numel].view(shape))
+                grads[-1].copy_(g)
+                del g
+            else:
+                grads.append(g)
+        if flat:
+            bufs.append(bflat[off:off + spec.numel].view(shape))
+        else:
+            bufs.append(torch.zeros(shape, dtype=torch.float32, device=device))
+        off += spec.numel
+    t = Tensors(params, grads, bufs, prior)
+    if flat:
+        t.flat = (pflat, gflat, bflat)
+    return t
 
 
 def ns_flops(wl: Workload, steps: Optional[int] = None) -> float:

@@ -1,0 +1,111 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol declared in
+include/dmuon.h, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import newton_schulz_09_b200 as dm
+from newton_schulz_09_b200 import build as dmbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dmuon.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dmbuild.build()
+    return dm.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dmuon_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("dmuon_ns_orthogonalize", "dmuon_muon_step_batched",
+                 "dmuon_muon_step_batched_ex", "dmuon_workspace_bytes", "dmuon_last_error",
+                 "dmuon_backend_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_built_for_sm100a_only():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(dmbuild.NVCC_FLAGS)
+
+
+def _shapes(*dims, pdt=dm.DMUON_BF16, gdt=dm.DMUON_BF16):
+    S = (dm.DmuonShape * len(dims))()
+    for i, (r, c) in enumerate(dims):
+        S[i] = dm.DmuonShape(r, c, pdt, gdt)
+    return S
+
+
+def _ptrs(*vals):
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def _call(lib, S, n, P=None, G=None, B=None, steps=5):
+    P = P or _ptrs(*([0x10000] * n))
+    G = G or _ptrs(*([0x20000] * n))
+    B = B or _ptrs(*([0x30000] * n))
+    return lib.dmuon_muon_step_batched(P, G, B, S, n, 0.02, 0.95, 1, 0.0, steps, None)
+
+
+def test_count_zero_is_a_noop(lib):
+    assert _call(lib, _shapes((4, 4)), 0) == 0
+
+
+def test_invalid_arguments_are_rejected_on_the_host(lib):
+    assert _call(lib, _shapes((4, 4)), -1) == -1
+    assert _call(lib, _shapes((4, 4)), 1, steps=-1) == -1
+    assert _call(lib, _shapes((0, 4)), 1) == -1
+    assert "rows and cols" in dm.dmuon_last_error()
+    assert _call(lib, _shapes((4, 4)), 1, P=_ptrs(None)) == -1
+    assert _call(lib, _shapes((4, 4)), 1, B=_ptrs(None)) == -1
+    assert _call(lib, _shapes((4, 4)), 1, P=_ptrs(0x10001)) == -1      # odd bf16 address
+    assert "aligned" in dm.dmuon_last_error()
+    assert _call(lib, _shapes((4, 4), pdt=7), 1) == -2
+    assert _call(lib, _shapes((40000, 40000)), 1) == -2                # min side too large
+    assert lib.dmuon_ns_orthogonalize(None, 4, 4, 5, None) == -1
+    assert lib.dmuon_ns_orthogonalize(ctypes.c_void_p(0x1000), 4, 4, -3, None) == -1
+
+
+def test_null_gradient_is_skipped_before_any_device_work(lib):
+    # Every matrix without a gradient: nothing to do, no CUDA call, success.
+    assert _call(lib, _shapes((4, 4), (8, 8)), 2, G=_ptrs(None, None)) == 0
+
+
+def test_workspace_bytes(lib):
+    # One 256x512 bf16 matrix, 5 steps: X0 and X1 (256 x 512), A (256 x 256),
+    # 32 prologue tiles of partials, one scale; regions rounded to 1 KiB.
+    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 5) == 2 * 262144 + 131072 + 1024 + 1024
+    # Tall matrix: same m x n view.
+    assert lib.dmuon_workspace_bytes(_shapes((512, 256)), 1, 5) == 2 * 262144 + 131072 + 1024 + 1024
+    # No second iterate and no Gram for steps == 0.
+    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 0) == 262144 + 1024 + 1024
+    # Ragged shape: rows padded to 16 bytes (8 bf16 / 4 fp32).
+    assert lib.dmuon_workspace_bytes(_shapes((3, 5)), 1, 1) == 1024 + 1024 + 1024 + 1024
+    assert lib.dmuon_workspace_bytes(_shapes((0, 5)), 1, 1) == 0
+    assert lib.dmuon_ns_workspace_bytes(256, 512, dm.DMUON_F32) == 4 * 524288 + 262144 + 1024 + 1024
+
+
+def test_backend_string(lib):
+    s = dm.dmuon_backend_string()
+    assert "tcgen05" in s and "sm_100a" in s
+
+
+def test_no_cpu_fallback_without_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(ValueError):
+        dm.dmuon_ns_orthogonalize(torch.zeros(4, 4, dtype=torch.bfloat16))
