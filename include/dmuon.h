@@ -144,6 +144,30 @@ int dmuon_device_status(int clear);
  * device).  Safe to call at any time from the host. */
 void dmuon_release_cache(void);
 
+/*
+ * dmuon_ns_orthogonalize_noalloc -- same result as dmuon_ns_orthogonalize
+ * (bf16, in place), for callers that may not allocate device memory: code
+ * running inside a framework that has already reserved the device's memory
+ * for its own pool, sandboxed plugins that are not allowed to call
+ * cudaMalloc, and latency-critical paths where cudaMalloc/cudaFree could
+ * block or synchronise the device.  It calls no allocation routine.  (The
+ * pages have no counterpart of this entry point; it is a property of this
+ * library.)
+ *   Scratch: a fixed 32 MiB device array inside the library, reserved on
+ *   every device that loads the library and held until the process exits.
+ *   Matrices whose scratch (dmuon_ns_workspace_bytes(m, n, DMUON_BF16) for
+ *   steps >= 2) exceeds 32 MiB - 16 KiB are rejected with
+ *   DMUON_ERR_UNSUPPORTED; e.g. 2048 x 2048 and 1024 x 4096 fit, 4096 x 4096
+ *   does not.
+ *   Sharing: every call uses the same array, and nothing carries over from
+ *   one call to the next.  Calls that may overlap on the GPU (different
+ *   streams without ordering between them) race on it; calls on one stream
+ *   are ordered.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (once per device); make that first call before any stream capture.
+ */
+int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int steps, dmuon_stream_t stream);
+
 /* Kernel kinds reported by the timing and launch counters below. */
 enum {
   DMUON_KERNEL_PROLOGUE = 0, /* momentum, Nesterov input, norm partials, copy into X */

@@ -21,7 +21,7 @@ __all__ = [
     "dmuon_muon_step_batched", "dmuon_muon_step_batched_ex", "dmuon_workspace_bytes",
     "dmuon_last_error", "dmuon_backend_string", "dmuon_device_status", "dmuon_release_cache",
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
-    "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS",
+    "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
 ]
 
 #: Kernel kinds of dmuon_stage_times(), in order.
@@ -82,6 +82,7 @@ def load_library() -> ctypes.CDLL:
         "dmuon_stage_times": (i32, [ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int64), i32, i32]),
         "dmuon_launch_count": (ctypes.c_int64, []),
+        "dmuon_ns_orthogonalize_noalloc": (i32, [vp, i64, i64, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -277,3 +278,20 @@ def dmuon_stage_times(reset: bool = False) -> dict:
 
 def dmuon_launch_count() -> int:
     return int(load_library().dmuon_launch_count())
+
+
+def dmuon_ns_orthogonalize_noalloc(X: torch.Tensor, steps: int = 5) -> torch.Tensor:
+    """In-place cubic Newton-Schulz of one bf16 matrix without allocating
+    any device memory: the scratch is a fixed 32 MiB array inside the
+    library.  For callers that must not allocate (a framework that owns all
+    device memory, a sandbox without cudaMalloc, a path that must not block
+    on an allocation).  Calls on different streams that may overlap race on
+    the shared scratch; larger matrices are rejected (DMUON_ERR_UNSUPPORTED)."""
+    lib = load_library()
+    _cuda_matrix(X, "X")
+    if X.dtype != torch.bfloat16:
+        raise TypeError("dmuon_ns_orthogonalize_noalloc takes bf16")
+    with torch.cuda.device(X.device):
+        _check(lib.dmuon_ns_orthogonalize_noalloc(X.data_ptr(), X.shape[0], X.shape[1], steps,
+                                                  _stream(X.device)))
+    return X

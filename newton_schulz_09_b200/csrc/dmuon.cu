@@ -839,3 +839,169 @@ int dmuon_debug_wait_timeout(int limit_us, dmuon_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ======================================================================
+// Allocation-free orthogonalisation.
+//
+// Some callers may not allocate device memory at all: code that runs inside
+// a host framework which has already reserved all device memory for its own
+// pool, plugins whose sandbox forbids cudaMalloc, and latency-critical paths
+// where cudaMalloc/cudaFree may block on, or synchronise with, the device.
+// For them dmuon_ns_orthogonalize_noalloc() takes its scratch (iterates,
+// Gram matrix, norm partials and the small launch description) from the
+// fixed array below, which the CUDA module reserves on every device that
+// loads this library and keeps until the process exits.
+// ======================================================================
+namespace dmuon {
+
+constexpr size_t kStaticScratchBytes = 32ull << 20;   // 32 MiB in total
+constexpr size_t kStaticPlanBytes = 16384;            // launch description at the front
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+// Device address of g_static_scratch, fetched once per device.  The host-side
+// name of a __device__ array is only a stand-in for it, so kernels must be
+// given this address instead.
+uint8_t* g_static_addr[64] = {nullptr};
+
+int static_scratch_address(int dev, uint8_t** out) {
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_static_addr[dev];
+  return DMUON_OK;
+}
+
+// Launch description of one matrix, laid out as the device reads it.
+struct alignas(128) StaticPlan {
+  MatDesc desc;
+  int order[2];
+  int syrk_prefix[2];
+  int gemm_prefix[2];
+  int pad_[2];
+  int64_t pprefix[2];
+  alignas(64) MatMaps maps;
+};
+static_assert(sizeof(StaticPlan) <= kStaticPlanBytes, "launch description does not fit");
+
+}  // namespace
+}  // namespace dmuon
+
+extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int steps,
+                                              dmuon_stream_t stream) {
+  using namespace dmuon;
+  t_last_error.clear();
+  std::vector<MatIn> in;
+  int r = ortho_input(X, m, n, steps, DMUON_BF16, &in);
+  if (r != DMUON_OK) return r;
+  const Layout L = make_layout(in, steps);
+  const size_t room = kStaticScratchBytes - kStaticPlanBytes;
+  if (L.bytes > room)
+    return fail(DMUON_ERR_UNSUPPORTED,
+                "dmuon_ns_orthogonalize_noalloc: a %lld x %lld matrix with %d steps needs %zu "
+                "bytes of scratch; the static scratch holds %zu (use dmuon_ns_orthogonalize_ex)",
+                (long long)m, (long long)n, steps, L.bytes, room);
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  uint8_t* base = nullptr;
+  r = static_scratch_address(dev, &base);
+  if (r != DMUON_OK) return r;
+  uint8_t* ws = base + kStaticPlanBytes;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  // Host image of the launch description.
+  const MatLayout& ml = L.mats[0];
+  const GroupLayout& g = L.groups[0];
+  StaticPlan sp;
+  std::memset(&sp, 0, sizeof(sp));
+  MatDesc& d = sp.desc;
+  d.W = X; d.G = X; d.buf = nullptr;
+  d.rows = m; d.cols = n;
+  d.ldx = ml.ldx; d.lda = ml.lda;
+  d.X[0] = ws + ml.x0;
+  d.X[1] = (ml.x1 != SIZE_MAX) ? ws + ml.x1 : nullptr;
+  d.Xop[0] = d.X[0];
+  d.Xop[1] = d.X[1];
+  d.A = (ml.a != SIZE_MAX) ? ws + ml.a : nullptr;
+  d.scale = reinterpret_cast<float*>(ws + g.scales);
+  d.lr_mult = 1.0f;
+  d.m = static_cast<int>(ml.m); d.n = static_cast<int>(ml.n);
+  d.T = m > n ? 1 : 0;
+  d.mode = kModeOrtho;
+  d.g_bf16 = 1;
+  d.vec4 = (n % 4 == 0) && aligned(X, 16);
+  d.ptiles_c = static_cast<int>(ml.ptiles_c);
+  const int syrk_tiles = static_cast<int>(syrk_tiles_of(ml.m));
+  const int gemm_tiles = static_cast<int>(gemm_tiles_of(ml.m, ml.n));
+  sp.order[0] = 0;
+  sp.syrk_prefix[1] = syrk_tiles;
+  sp.gemm_prefix[1] = gemm_tiles;
+  sp.pprefix[1] = ml.ptiles;
+  const int BK = 64;   // bf16: 128-byte K slices
+  bool okm = true;
+  for (int b = 0; b < 2; ++b) {
+    void* xb = d.X[b];
+    if (!xb) { sp.maps.xk[b] = sp.maps.xk[0]; sp.maps.xmn[b] = sp.maps.xmn[0]; continue; }
+    okm &= encode_2d(&sp.maps.xk[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBM);
+    okm &= encode_2d(&sp.maps.xmn[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, BK);
+  }
+  if (d.A) okm &= encode_2d(&sp.maps.a, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+  if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  // Upload on the caller's stream: ordered after any earlier call on it.
+  cudaError_t e = cudaMemcpyAsync(base, &sp, sizeof(sp), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "uploading the launch description");
+  const StaticPlan* dsp = reinterpret_cast<const StaticPlan*>(base);
+
+  const DeviceInfo& di = g_dev[dev];
+  ElemParams ep;
+  ep.mats = &dsp->desc;
+  ep.ptile_prefix = dsp->pprefix;
+  ep.partials = reinterpret_cast<float*>(ws + g.partials);
+  ep.nmat = 1;
+  ep.ntiles = ml.ptiles;
+  ep.mu = 0.0f;
+  ep.nesterov = 0;
+  ep.lr = 0.0f;
+  ep.wd = 0.0f;
+  const int pgrid = static_cast<int>(std::min<int64_t>(ml.ptiles, static_cast<int64_t>(di.sms) * 8));
+  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, 0, st>>>(ep);
+  finalize_kernel<<<1, 32, 0, st>>>(ep);
+  g_launches += 2;
+  if (steps == 0) {
+    apply_kernel<__nv_bfloat16><<<pgrid, kPThreads, 0, st>>>(ep);
+    ++g_launches;
+  } else {
+    NsParams np;
+    np.mats = &dsp->desc;
+    np.maps = &dsp->maps;
+    np.order = dsp->order;
+    np.nmat = 1;
+    np.lr = 0.0f;
+    np.wd = 0.0f;
+    np.err = di.err;
+    np.wait_limit_ns = kWaitLimitNs;
+    for (int s = 0; s < steps; ++s) {
+      np.cur = s & 1;
+      np.first = s == 0;
+      np.last = s == steps - 1;
+      np.tile_prefix = dsp->syrk_prefix;
+      np.ntiles = syrk_tiles;
+      ns_stage_kernel<kSyrk, __nv_bfloat16><<<std::min(syrk_tiles, di.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      np.tile_prefix = dsp->gemm_prefix;
+      np.ntiles = gemm_tiles;
+      ns_stage_kernel<kGemm, __nv_bfloat16><<<std::min(gemm_tiles, di.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      g_launches += 2;
+    }
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return DMUON_OK;
+}
