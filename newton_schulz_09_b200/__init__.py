@@ -295,3 +295,4 @@ def dmuon_ns_orthogonalize_noalloc(X: torch.Tensor, steps: int = 5) -> torch.Ten
         _check(lib.dmuon_ns_orthogonalize_noalloc(X.data_ptr(), X.shape[0], X.shape[1], steps,
                                                   _stream(X.device)))
     return X
+

@@ -186,8 +186,14 @@ Layout make_layout(const std::vector<MatIn>& in, int steps) {
         if (steps >= 2) { ml.o1 = off; off = align_up(off + xb, 1024); }
       }
       if (steps >= 1) { ml.a = off; off = align_up(off + ab, 1024); }
-      ml.ptiles_c = cdiv(in[i].cols, kPT);
-      ml.ptiles = cdiv(in[i].rows, kPT) * ml.ptiles_c;
+      // Prologue work items: flat chunks, or kTR x kTC tiles when transposed.
+      if (in[i].rows > in[i].cols) {
+        ml.ptiles_c = cdiv(in[i].cols, kTC);
+        ml.ptiles = cdiv(in[i].rows, kTR) * ml.ptiles_c;
+      } else {
+        ml.ptiles_c = 0;
+        ml.ptiles = cdiv(in[i].rows * in[i].cols, kFlatChunk);
+      }
       g.ptiles += ml.ptiles;
     }
     g.partials = off; off = align_up(off + sizeof(float) * g.ptiles, 1024);
@@ -280,6 +286,8 @@ int device_setup(int dev) {
 }
 
 // SYRK tiles of an m x m Gram: column bands of 256 with row bands 0..2J+1.
+// SYRK tiles of an m x m Gram: column bands of 256 with row bands 0..2J+1
+// of 128.
 int64_t syrk_tiles_of(int64_t m) {
   const int64_t nJ = cdiv(m, kBN), nI = cdiv(m, kBM);
   return (nJ - 1) * nJ + nI;
@@ -509,6 +517,13 @@ struct LaunchScope {
   }
 };
 
+// One Newton-Schulz stage over all tiles of a group: a persistent grid of at
+// most one CTA per SM.
+template <int kMode, typename E>
+void launch_ns_stage(const NsParams& np, const DeviceInfo& d, cudaStream_t st) {
+  ns_stage_kernel<kMode, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+}
+
 template <typename E>
 void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float lr, float mu,
                   int nesterov, float wd, int steps, cudaStream_t st) {
@@ -553,14 +568,14 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float 
     np.ntiles = g.syrk_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_SYRK);
-      ns_stage_kernel<kSyrk, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      launch_ns_stage<kSyrk, E>(np, d, st);
     }
     np.order = g.gemm_order;
     np.tile_prefix = g.gemm_prefix;
     np.ntiles = g.gemm_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_GEMM);
-      ns_stage_kernel<kGemm, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      launch_ns_stage<kGemm, E>(np, d, st);
     }
   }
 }
@@ -994,10 +1009,10 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
       np.last = s == steps - 1;
       np.tile_prefix = dsp->syrk_prefix;
       np.ntiles = syrk_tiles;
-      ns_stage_kernel<kSyrk, __nv_bfloat16><<<std::min(syrk_tiles, di.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      launch_ns_stage<kSyrk, __nv_bfloat16>(np, di, st);
       np.tile_prefix = dsp->gemm_prefix;
       np.ntiles = gemm_tiles;
-      ns_stage_kernel<kGemm, __nv_bfloat16><<<std::min(gemm_tiles, di.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+      launch_ns_stage<kGemm, __nv_bfloat16>(np, di, st);
       g_launches += 2;
     }
   }

@@ -34,8 +34,11 @@ constexpr int kAStageBytes = kBM * 128;   // one 128-byte K slice of 128 rows
 constexpr int kBStageBytes = kBN * 128;   // one 128-byte K slice of 256 rows
 constexpr int kTmemCols = 2 * kBN;        // double-buffered fp32 accumulator
 constexpr int kNsThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kNsSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 256;
-constexpr int kPT = 64;            // prologue tile: 64 x 64 parameter elements
+constexpr int kEpiSlotBytes = kBM * 128;  // one 128-row x 128-byte output quarter (bf16 GEMM)
+constexpr int kEpiSlots = 2;
+constexpr int kNsSmemBytes =
+    kStages * (kAStageBytes + kBStageBytes) + kEpiSlots * kEpiSlotBytes + 1024 /*align*/ + 256;
+static_assert(kNsSmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
 constexpr int kPThreads = 256;
 
 enum { kModeMuon = 0, kModeOrtho = 1 };
@@ -59,7 +62,7 @@ struct MatDesc {
   int mode;            // kModeMuon | kModeOrtho
   int g_bf16;          // gradient / input storage: 1 bf16, 0 fp32
   int vec4;            // parameter rows allow 4-element vector access
-  int ptiles_c;        // prologue tiles per parameter row band
+  int ptiles_c;        // transposed prologue tiles per parameter row band
   int pad_;
 };
 
@@ -193,6 +196,7 @@ struct TileInfo {
   int mi, tm, tn, nkb;
 };
 
+// Tile t of a launch (128 x 256 tiles).
 template <int kMode, int BK>
 __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
   TileInfo ti;
@@ -213,7 +217,259 @@ __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
 }
 
 // ======================================================================
-// Newton-Schulz stage kernel (persistent, warp specialised).
+// Epilogue (warps 2-5): TMEM accumulators of this CTA's 128 tile rows ->
+// SYRK stores (A and its mirror), or the GEMM combine / final update.
+// The accumulator buffer is released by `release(b)` once fully read.
+// Returns false when a bounded wait gave up.
+// ======================================================================
+template <int kMode, typename E, typename Release>
+__device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_base, uint8_t* epi,
+                                             uint64_t* tfull, uint64_t* xfull, int warp, int lane,
+                                             int t0, int tstride, Release release) {
+  constexpr int EB = static_cast<int>(sizeof(E));
+  constexpr int BK = 128 / EB;
+  const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+  const int row_in_tile = q4 * 32 + lane;
+  bool ok = true;
+
+  if (kMode == kGemm && EB == 2 && !p.last) {
+    // bf16 GEMM steps: the old X arrives by TMA, 64 columns (one quarter) at
+    // a time, into a two-slot ring; each thread combines its row in place
+    // with the accumulator and the quarter leaves by TMA store.
+    const bool leader = (warp == 2 && lane == 0);
+    int ld_t = t0, ld_q = 0;               // next quarter to load (leader only)
+    uint32_t ld_g = 0;
+    bool slot_busy[kEpiSlots] = {false, false};
+    uint32_t slot_phase[kEpiSlots] = {0u, 0u};
+    auto quarters_of = [&](const TileInfo& ti) -> int {
+      const int left = p.mats[ti.mi].n - ti.tn * kBN;
+      const int nq = (left + 63) / 64;
+      return nq < 4 ? nq : 4;
+    };
+    auto load_next = [&]() {
+      if (ld_t >= p.ntiles) return;
+      const TileInfo ti = decode_tile<kMode, BK>(p, ld_t);
+      const int slot = static_cast<int>(ld_g & 1u);
+      mbar_arrive_expect_tx(&xfull[slot], kEpiSlotBytes);
+      tma_load_2d(epi + slot * kEpiSlotBytes, &p.maps[ti.mi].xk[p.cur], &xfull[slot],
+                  ti.tn * kBN + 64 * ld_q, ti.tm * kBM);
+      slot_busy[slot] = true;
+      slot_phase[slot] = (ld_g >> 1) & 1u;
+      ++ld_g;
+      if (++ld_q >= quarters_of(ti)) { ld_q = 0; ld_t += tstride; }
+    };
+    if (leader) { load_next(); load_next(); }
+    uint32_t g = 0;
+    int lt = 0;
+    for (int t = t0; t < p.ntiles && ok; t += tstride, ++lt) {
+      const TileInfo ti = decode_tile<kMode, BK>(p, t);
+      const MatDesc& md = p.mats[ti.mi];
+      const int b = lt & 1;
+      const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
+      const float cs = p.first ? *md.scale : 1.0f;
+      const int nq = quarters_of(ti);
+      bool w = mbar_wait(&tfull[b], tph, p.err, p.wait_limit_ns);
+      if (!named_bar_and(1, 128, w)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(b * kBN);
+      for (int qq = 0; qq < nq; ++qq, ++g) {
+        const int slot = static_cast<int>(g & 1u);
+        w = mbar_wait(&xfull[slot], (g >> 1) & 1u, p.err, p.wait_limit_ns);
+        if (!named_bar_and(1, 128, w)) { ok = false; break; }
+        uint32_t v0[32], v1[32];
+        tmem_ld32(taddr + qq * 64, v0);
+        tmem_ld32(taddr + qq * 64 + 32, v1);
+        tmem_ld_wait();
+        if (qq == nq - 1) release(b);
+        uint8_t* rowp = epi + slot * kEpiSlotBytes + row_in_tile * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(rowp + ((c ^ (row_in_tile & 7)) << 4));
+          uint4 u = *ptr;
+          uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 xf = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[j]));
+            const int col = c * 8 + 2 * j;
+            const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
+            const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
+            __nv_bfloat162 yv = __floats2bfloat162_rn(cs * (1.5f * xf.x - 0.5f * a0),
+                                                      cs * (1.5f * xf.y - 0.5f * a1));
+            wv[j] = *reinterpret_cast<uint32_t*>(&yv);
+          }
+          *ptr = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          tma_store_2d(&p.maps[ti.mi].xk[p.cur ^ 1], epi + slot * kEpiSlotBytes,
+                       ti.tn * kBN + 64 * qq, ti.tm * kBM);
+          bulk_commit_group();
+          bulk_wait_group_read0();               // slot read out: it may be refilled
+          slot_busy[slot] = false;
+          load_next();
+        }
+      }
+    }
+    if (leader) {
+      bulk_wait_group0();
+      if (!ok)
+        for (int e = 0; e < kEpiSlots; ++e)
+          if (slot_busy[e]) mbar_wait(&xfull[e], slot_phase[e], nullptr, p.wait_limit_ns, 1024);
+    }
+    return ok;
+  }
+
+  int lt = 0;
+  for (int t = t0; t < p.ntiles && ok; t += tstride, ++lt) {
+    const TileInfo ti = decode_tile<kMode, BK>(p, t);
+    const MatDesc& md = p.mats[ti.mi];
+    const int b = lt & 1;
+    const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
+    const float s = *md.scale;
+    bool w = mbar_wait(&tfull[b], tph, p.err, p.wait_limit_ns);
+    if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+    tc_fence_after();
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(b * kBN);
+    const int R = ti.tm * kBM + row_in_tile;
+    const int m = md.m, n = md.n;
+    if (kMode == kSyrk) {
+      const float alpha = p.first ? s * s : 1.0f;
+      E* A = reinterpret_cast<E*>(md.A);
+      const int64_t lda = md.lda;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait();
+        if (c == kBN / 32 - 1) release(b);
+        const int C0 = ti.tn * kBN + c * 32;
+        if (R < m && C0 < m && C0 + 31 >= R) {
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = op_round<E>(alpha * __uint_as_float(v[j]));
+          E* arow = A + static_cast<int64_t>(R) * lda;
+          if (C0 >= R && C0 + 32 <= m) {
+            store32<E>(arow + C0, y);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int C = C0 + j;
+              if (C < m && C >= R) arow[C] = from_f<E>(y[j]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int C = C0 + j;
+            if (C < m && C > R) A[static_cast<int64_t>(C) * lda + R] = from_f<E>(y[j]);
+          }
+        }
+      }
+    } else {
+      const float cs = p.first ? s : 1.0f;
+      const E* Xc = reinterpret_cast<const E*>(md.X[p.cur]);
+      E* Xn = reinterpret_cast<E*>(md.X[p.cur ^ 1]);
+      const int64_t ldx = md.ldx;
+      const float lr = p.lr * md.lr_mult;
+      const float decay = 1.0f - lr * p.wd;
+      E* W = reinterpret_cast<E*>(md.W);
+      const int64_t cols = md.cols;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait();
+        if (c == kBN / 32 - 1) release(b);
+        const int C0 = ti.tn * kBN + c * 32;
+        if (R < m && C0 < n) {
+          const bool full_chunk = (C0 + 32 <= n);
+          float x[32];
+          const E* xrow = Xc + static_cast<int64_t>(R) * ldx + C0;
+          if (full_chunk) {
+            load32<E>(xrow, x);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = (C0 + j < n) ? to_f<E>(xrow[j]) : 0.0f;
+          }
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = cs * (1.5f * x[j] - 0.5f * __uint_as_float(v[j]));
+          if (!p.last) {
+            E* dst = Xn + static_cast<int64_t>(R) * ldx + C0;
+            if (full_chunk) {
+              store32<E>(dst, y);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (C0 + j < n) dst[j] = from_f<E>(y[j]);
+            }
+            if (EB == 4) {
+              E* odst = reinterpret_cast<E*>(md.Xop[p.cur ^ 1]) + static_cast<int64_t>(R) * ldx + C0;
+              float yr[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) yr[j] = op_round<E>(y[j]);
+              if (full_chunk) {
+                store32<E>(odst, yr);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (C0 + j < n) odst[j] = from_f<E>(yr[j]);
+              }
+            }
+          } else if (!md.T) {
+            E* wrow = W + static_cast<int64_t>(R) * cols + C0;
+            if (md.mode == kModeOrtho) {
+              if (full_chunk && md.vec4 && (cols % (16 / EB) == 0)) {
+                store32<E>(wrow, y);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (C0 + j < n) wrow[j] = from_f<E>(y[j]);
+              }
+            } else {
+              if (full_chunk && md.vec4 && (cols % (16 / EB) == 0)) {
+                float wv[32];
+                load32<E>(wrow, wv);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) wv[j] = fmaf(wv[j], decay, -lr * y[j]);
+                store32<E>(wrow, wv);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (C0 + j < n) wrow[j] = from_f<E>(fmaf(to_f<E>(wrow[j]), decay, -lr * y[j]));
+              }
+            }
+          } else {
+            // Transposed parameter: X[R][C] is W[C][R]; a warp's lanes hold
+            // consecutive R, so each j touches one contiguous run.  All
+            // loads are issued before any store so they overlap.
+            E* wcol = W + static_cast<int64_t>(C0) * cols + R;
+            if (md.mode == kModeOrtho) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (C0 + j < n) wcol[static_cast<int64_t>(j) * cols] = from_f<E>(y[j]);
+            } else {
+              float wv[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                wv[j] = (C0 + j < n) ? to_f<E>(wcol[static_cast<int64_t>(j) * cols]) : 0.0f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (C0 + j < n)
+                  wcol[static_cast<int64_t>(j) * cols] = from_f<E>(fmaf(wv[j], decay, -lr * y[j]));
+            }
+          }
+        }
+      }
+    }
+  }
+  return ok;
+}
+
+// ======================================================================
+// Newton-Schulz stage kernel, one CTA per 128 x 256 tile.
+// Persistent and warp specialised: warp 0 TMA producer, warp 1 UMMA issuer,
+// warps 2-5 epilogue.
 // ======================================================================
 template <int kMode, typename E>
 __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_constant__ NsParams p) {
@@ -231,11 +487,13 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sa = smem;
   uint8_t* sb = smem + kStages * kAStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kStages * kBStageBytes);
+  uint8_t* epi = sb + kStages * kBStageBytes;          // GEMM output quarters (bf16)
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiSlots * kEpiSlotBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* xfull = tempty + 2;                          // [kEpiSlots]
+  uint64_t* drain = xfull + kEpiSlots;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -250,6 +508,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4 * 32);
     }
+    for (int e = 0; e < kEpiSlots; ++e) mbar_init(&xfull[e], 1);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -362,144 +621,11 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------ epilogue (4 warps)
-    const int q = warp & 3;                 // TMEM lane quarter of this warp
-    const int row_in_tile = q * 32 + lane;
-    int lt = 0;
-    for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
-      const TileInfo ti = decode_tile<kMode, BK>(p, t);
-      const MatDesc& md = p.mats[ti.mi];
-      const int b = lt & 1;
-      const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
-      const float s = *md.scale;
-      bool w = mbar_wait(&tfull[b], tph, p.err, p.wait_limit_ns);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * kBN);
-      const int R = ti.tm * kBM + row_in_tile;
-      const int m = md.m, n = md.n;
-      if (kMode == kSyrk) {
-        const float alpha = p.first ? s * s : 1.0f;
-        E* A = reinterpret_cast<E*>(md.A);
-        const int64_t lda = md.lda;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_ld_wait();
-          const int C0 = ti.tn * kBN + c * 32;
-          if (R < m && C0 < m && C0 + 31 >= R) {
-            float y[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = op_round<E>(alpha * __uint_as_float(v[j]));
-            E* arow = A + static_cast<int64_t>(R) * lda;
-            if (C0 >= R && C0 + 32 <= m) {
-              store32<E>(arow + C0, y);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int C = C0 + j;
-                if (C < m && C >= R) arow[C] = from_f<E>(y[j]);
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int C = C0 + j;
-              if (C < m && C > R) A[static_cast<int64_t>(C) * lda + R] = from_f<E>(y[j]);
-            }
-          }
-        }
-      } else {
-        const float cs = p.first ? s : 1.0f;
-        const E* Xc = reinterpret_cast<const E*>(md.X[p.cur]);
-        E* Xn = reinterpret_cast<E*>(md.X[p.cur ^ 1]);
-        const int64_t ldx = md.ldx;
-        const float lr = p.lr * md.lr_mult;
-        const float decay = 1.0f - lr * p.wd;
-        E* W = reinterpret_cast<E*>(md.W);
-        const int64_t cols = md.cols;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_ld_wait();
-          const int C0 = ti.tn * kBN + c * 32;
-          if (R < m && C0 < n) {
-            const bool full_chunk = (C0 + 32 <= n);
-            float x[32];
-            const E* xrow = Xc + static_cast<int64_t>(R) * ldx + C0;
-            if (full_chunk) {
-              load32<E>(xrow, x);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) x[j] = (C0 + j < n) ? to_f<E>(xrow[j]) : 0.0f;
-            }
-            float y[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = cs * (1.5f * x[j] - 0.5f * __uint_as_float(v[j]));
-            if (!p.last) {
-              E* dst = Xn + static_cast<int64_t>(R) * ldx + C0;
-              if (full_chunk) {
-                store32<E>(dst, y);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (C0 + j < n) dst[j] = from_f<E>(y[j]);
-              }
-              if (EB == 4) {
-                E* odst = reinterpret_cast<E*>(md.Xop[p.cur ^ 1]) + static_cast<int64_t>(R) * ldx + C0;
-                float yr[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) yr[j] = op_round<E>(y[j]);
-                if (full_chunk) {
-                  store32<E>(odst, yr);
-                } else {
-#pragma unroll
-                  for (int j = 0; j < 32; ++j)
-                    if (C0 + j < n) odst[j] = from_f<E>(yr[j]);
-                }
-              }
-            } else if (!md.T) {
-              E* wrow = W + static_cast<int64_t>(R) * cols + C0;
-              if (md.mode == kModeOrtho) {
-                if (full_chunk && md.vec4 && (cols % (16 / EB) == 0)) {
-                  store32<E>(wrow, y);
-                } else {
-#pragma unroll
-                  for (int j = 0; j < 32; ++j)
-                    if (C0 + j < n) wrow[j] = from_f<E>(y[j]);
-                }
-              } else {
-                if (full_chunk && md.vec4 && (cols % (16 / EB) == 0)) {
-                  float wv[32];
-                  load32<E>(wrow, wv);
-#pragma unroll
-                  for (int j = 0; j < 32; ++j) wv[j] = fmaf(wv[j], decay, -lr * y[j]);
-                  store32<E>(wrow, wv);
-                } else {
-#pragma unroll
-                  for (int j = 0; j < 32; ++j)
-                    if (C0 + j < n) wrow[j] = from_f<E>(fmaf(to_f<E>(wrow[j]), decay, -lr * y[j]));
-                }
-              }
-            } else {
-              // Transposed parameter: X[R][C] is W[C][R]; a warp's lanes hold
-              // consecutive R, so each j writes one contiguous run.
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int C = C0 + j;
-                if (C < n) {
-                  E* wp = W + static_cast<int64_t>(C) * cols + R;
-                  if (md.mode == kModeOrtho) *wp = from_f<E>(y[j]);
-                  else *wp = from_f<E>(fmaf(to_f<E>(*wp), decay, -lr * y[j]));
-                }
-              }
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[b]);
-    }
+    ok = run_epilogue<kMode, E>(p, tmem_base, epi, tfull, xfull, warp, lane, blockIdx.x, gridDim.x,
+                                [&](int b) {
+                                         tc_fence_before();
+                                         mbar_arrive(&tempty[b]);
+                                       });
   }
 
   __syncthreads();
@@ -510,149 +636,224 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 }
 
 // ======================================================================
-// Prologue: momentum + Nesterov + sum of squares + copy into X (transposed
-// when rows > cols).  One 64 x 64 parameter tile per iteration.
+// Prologue: momentum + Nesterov + sum of squares + copy of M into X.
+// Work items: a matrix that is not transposed is streamed flat, kFlatChunk
+// consecutive elements per item (X has the parameter's layout); a transposed
+// matrix is cut into kTR x kTC parameter tiles that are transposed through
+// shared memory.  One partial sum of squares per item.
 // ======================================================================
-template <typename E>
-__device__ __forceinline__ void load4_in(const MatDesc& md, int64_t idx, bool vec, int valid,
-                                         float (&g)[4]) {
+constexpr int kFlatChunk = 8192;       // elements per flat item (256 threads x 4 x 8)
+constexpr int kTR = 64, kTC = 128;     // transposed item: 64 parameter rows x 128 columns
+
+// 8 consecutive input elements (bf16 or fp32), 16-byte aligned when vec.
+__device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool vec, int valid, float (&g)[8]) {
   if (md.g_bf16) {
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(md.G) + idx;
     if (vec) {
-      uint2 u = *reinterpret_cast<const uint2*>(src);
-      float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
-      float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
-      g[0] = a.x; g[1] = a.y; g[2] = b.x; g[3] = b.y;
+      const uint4 u = *reinterpret_cast<const uint4*>(src);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        g[2 * j] = f.x;
+        g[2 * j + 1] = f.y;
+      }
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) g[e] = (e < valid) ? __bfloat162float(src[e]) : 0.0f;
+      for (int e = 0; e < 8; ++e) g[e] = (e < valid) ? __bfloat162float(src[e]) : 0.0f;
     }
   } else {
     const float* src = reinterpret_cast<const float*>(md.G) + idx;
     if (vec) {
-      float4 u = *reinterpret_cast<const float4*>(src);
-      g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w;
+      g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) g[e] = (e < valid) ? src[e] : 0.0f;
+      for (int e = 0; e < 8; ++e) g[e] = (e < valid) ? src[e] : 0.0f;
+    }
+  }
+}
+__device__ __forceinline__ void load8_f32(const float* src, bool vec, int valid, float (&b)[8]) {
+  if (vec) {
+    const float4 x = *reinterpret_cast<const float4*>(src);
+    const float4 y = *reinterpret_cast<const float4*>(src + 4);
+    b[0] = x.x; b[1] = x.y; b[2] = x.z; b[3] = x.w;
+    b[4] = y.x; b[5] = y.y; b[6] = y.z; b[7] = y.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b[e] = (e < valid) ? src[e] : 0.0f;
+  }
+}
+__device__ __forceinline__ void store8_f32(float* dst, bool vec, int valid, const float (&b)[8]) {
+  if (vec) {
+    *reinterpret_cast<float4*>(dst) = make_float4(b[0], b[1], b[2], b[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(b[4], b[5], b[6], b[7]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < valid) dst[e] = b[e];
+  }
+}
+// 8 consecutive X elements (16-byte aligned when vec).
+template <typename E>
+__device__ __forceinline__ void store8_x(E* dst, bool vec, int valid, const float (&v)[8]) {
+  if (vec && sizeof(E) == 2) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if (vec) {
+    float* d = reinterpret_cast<float*>(dst);
+    *reinterpret_cast<float4*>(d) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < valid) dst[e] = from_f<E>(v[e]);
+  }
+}
+
+// Momentum / Nesterov on 8 values; returns M, updates b in place.
+__device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, const float (&g)[8],
+                                          float (&b)[8], float (&M)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (has_buf) {
+      // buf <- fl(fl(mu * buf) + g): two roundings, never fused.
+      b[e] = __fadd_rn(__fmul_rn(p.mu, b[e]), g[e]);
+      M[e] = p.nesterov ? fmaf(p.mu, b[e], g[e]) : b[e];
+    } else {
+      M[e] = g[e];
     }
   }
 }
 
 template <typename E>
+__device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDesc& md, int64_t item) {
+  const int tid = threadIdx.x;
+  const int64_t numel = md.rows * md.cols;
+  const int64_t e_begin = item * kFlatChunk;
+  const bool has_buf = md.buf != nullptr;
+  const bool flat_x = (md.ldx == md.cols);
+  E* X = reinterpret_cast<E*>(md.X[0]);
+  E* Xo = reinterpret_cast<E*>(md.Xop[0]);
+  float ss = 0.0f;
+  // Four rounds of 8 consecutive elements per thread; latency is hidden by
+  // occupancy (few registers per thread).
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    const int64_t e = e_begin + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+    if (e >= numel) break;
+    const int valid = static_cast<int>(numel - e < 8 ? numel - e : 8);
+    const bool vec = md.vec4 && valid == 8;
+    float g[8], b[8], M[8];
+    load8_in(md, e, vec, valid, g);
+    if (has_buf) load8_f32(md.buf + e, vec, valid, b);
+    momentum8(p, has_buf, g, b, M);
+    if (has_buf) store8_f32(md.buf + e, vec, valid, b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= valid) M[k] = 0.0f;
+      ss = fmaf(M[k], M[k], ss);
+    }
+    if (flat_x) {
+      store8_x<E>(X + e, valid == 8, valid, M);
+      if (sizeof(E) == 4 && Xo != X) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) M[k] = op_round<E>(M[k]);
+        store8_x<E>(Xo + e, valid == 8, valid, M);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < valid) {
+          const int64_t r = (e + k) / md.cols, c = (e + k) - r * md.cols;
+          X[r * md.ldx + c] = from_f<E>(M[k]);
+          if (sizeof(E) == 4 && Xo != X) Xo[r * md.ldx + c] = from_f<E>(op_round<E>(M[k]));
+        }
+      }
+    }
+  }
+  return ss;
+}
+
+template <typename E>
+__device__ __forceinline__ float prologue_transposed(const ElemParams& p, const MatDesc& md, int64_t item,
+                                                     float (*sM)[kTC + 1]) {
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4;      // 0..15: parameter rows ty + 16 i
+  const int tx = tid & 15;      // 0..15: 8 consecutive parameter columns
+  const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+  const int64_t r0 = tr * kTR, c0 = tc * kTC;
+  const int64_t rows = md.rows, cols = md.cols;
+  const bool has_buf = md.buf != nullptr;
+  const int64_t c = c0 + tx * 8;
+  float ss = 0.0f;
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + ty + 16 * i;
+    const int valid = (r < rows && c < cols) ? static_cast<int>(cols - c < 8 ? cols - c : 8) : 0;
+    float g[8], b[8], M[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { g[k] = 0.0f; b[k] = 0.0f; }
+    const int64_t idx = r * cols + c;
+    const bool vec = md.vec4 && valid == 8 && ((idx & 7) == 0);
+    if (valid > 0) {
+      load8_in(md, idx, vec, valid, g);
+      if (has_buf) load8_f32(md.buf + idx, vec, valid, b);
+    }
+    momentum8(p, has_buf, g, b, M);
+    if (valid > 0 && has_buf) store8_f32(md.buf + idx, vec, valid, b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= valid) M[k] = 0.0f;
+      ss = fmaf(M[k], M[k], ss);
+      sM[ty + 16 * i][tx * 8 + k] = M[k];
+    }
+  }
+  __syncthreads();
+  // X row = parameter column (128 of them), X columns = the 64 parameter rows.
+  E* X = reinterpret_cast<E*>(md.X[0]);
+  E* Xo = reinterpret_cast<E*>(md.Xop[0]);
+  const int xc8 = tid & 7;      // 8 threads x 8 elements = the 64 rows
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int cc = (tid >> 3) + 32 * pass;   // parameter column within the tile
+    const int64_t xr = c0 + cc;
+    const int64_t xc = r0 + xc8 * 8;
+    if (xr < cols && xc < rows) {
+      const int valid = (rows - xc >= 8) ? 8 : static_cast<int>(rows - xc);
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = sM[xc8 * 8 + k][cc];
+      store8_x<E>(X + xr * md.ldx + xc, valid == 8, valid, v);
+      if (sizeof(E) == 4 && Xo != X) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = op_round<E>(v[k]);
+        store8_x<E>(Xo + xr * md.ldx + xc, valid == 8, valid, v);
+      }
+    }
+  }
+  __syncthreads();
+  return ss;
+}
+
+template <typename E>
 __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
-  __shared__ float sM[kPT][kPT + 1];
+  __shared__ float sM[kTR][kTC + 1];
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
-  const int ty = tid >> 4;  // 0..15
-  const int tx = tid & 15;  // 0..15: 4 consecutive columns each
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
     const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
     const MatDesc& md = p.mats[mi];
-    const int64_t local = t - __ldg(p.ptile_prefix + mi);
-    const int64_t tr = local / md.ptiles_c, tc = local - tr * md.ptiles_c;
-    const int64_t r0 = tr * kPT, c0 = tc * kPT;
-    const int64_t rows = md.rows, cols = md.cols;
-    E* X = reinterpret_cast<E*>(md.X[0]);
-    E* Xo = reinterpret_cast<E*>(md.Xop[0]);
-    float ss = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t r = r0 + ty + 16 * i;
-      const int64_t c = c0 + tx * 4;
-      float M[4] = {0.f, 0.f, 0.f, 0.f};
-      if (r < rows && c < cols) {
-        const int valid = (cols - c >= 4) ? 4 : static_cast<int>(cols - c);
-        const bool vec = md.vec4 && valid == 4;
-        const int64_t idx = r * cols + c;
-        float g[4];
-        load4_in<E>(md, idx, vec, valid, g);
-        if (md.buf != nullptr) {
-          float* bp = md.buf + idx;
-          float b[4];
-          if (vec) {
-            float4 u = *reinterpret_cast<const float4*>(bp);
-            b[0] = u.x; b[1] = u.y; b[2] = u.z; b[3] = u.w;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) b[e] = (e < valid) ? bp[e] : 0.0f;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            // buf <- fl(fl(mu * buf) + g): two roundings, never fused.
-            b[e] = __fadd_rn(__fmul_rn(p.mu, b[e]), g[e]);
-            M[e] = p.nesterov ? fmaf(p.mu, b[e], g[e]) : b[e];
-          }
-          if (vec) {
-            *reinterpret_cast<float4*>(bp) = make_float4(b[0], b[1], b[2], b[3]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (e < valid) bp[e] = b[e];
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) M[e] = g[e];
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (e >= valid) M[e] = 0.0f;
-          ss = fmaf(M[e], M[e], ss);
-        }
-        if (!md.T) {
-          E* dst = X + r * md.ldx + c;
-          if (valid == 4 && sizeof(E) == 2) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(M[0], M[1]);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(M[2], M[3]);
-            uint2 u;
-            u.x = *reinterpret_cast<uint32_t*>(&lo);
-            u.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(dst) = u;
-          } else if (valid == 4) {
-            *reinterpret_cast<float4*>(dst) = make_float4(M[0], M[1], M[2], M[3]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (e < valid) dst[e] = from_f<E>(M[e]);
-          }
-          if (sizeof(E) == 4 && Xo != X) {
-            E* odst = Xo + r * md.ldx + c;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (e < valid) odst[e] = from_f<E>(op_round<E>(M[e]));
-          }
-        }
-      }
-      if (md.T) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sM[ty + 16 * i][tx * 4 + e] = M[e];
-      }
-    }
-    if (md.T) {
-      __syncthreads();
-      // X row = parameter column, X columns = parameter rows.
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int cc = ty + 16 * i;
-        const int64_t xr = c0 + cc;
-        const int64_t xc = r0 + tx * 4;
-        if (xr < cols && xc < rows) {
-          E* dst = X + xr * md.ldx + xc;
-          const int valid = (rows - xc >= 4) ? 4 : static_cast<int>(rows - xc);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (e < valid) dst[e] = from_f<E>(sM[tx * 4 + e][cc]);
-          if (sizeof(E) == 4 && Xo != X) {
-            E* odst = Xo + xr * md.ldx + xc;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (e < valid) odst[e] = from_f<E>(op_round<E>(sM[tx * 4 + e][cc]));
-          }
-        }
-      }
-      __syncthreads();
-    }
-    // Fixed-order block reduction of the tile's sum of squares.
+    const int64_t item = t - __ldg(p.ptile_prefix + mi);
+    float ss = md.T ? prologue_transposed<E>(p, md, item, sM) : prologue_flat<E>(p, md, item);
+    // Fixed-order block reduction of the item's sum of squares.
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
@@ -680,22 +881,36 @@ __global__ void finalize_kernel(const __grid_constant__ ElemParams p) {
   if (lane == 0) *p.mats[mi].scale = static_cast<float>(1.0 / (sqrt(acc) + 1e-7));
 }
 
-// ns_steps == 0: the result is X0 = s M itself.
+// ns_steps == 0: the result is X0 = s M itself.  Same work items as the
+// prologue.
 template <typename E>
 __global__ void __launch_bounds__(kPThreads) apply_kernel(const __grid_constant__ ElemParams p) {
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
     const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
     const MatDesc& md = p.mats[mi];
-    const int64_t local = t - __ldg(p.ptile_prefix + mi);
-    const int64_t tr = local / md.ptiles_c, tc = local - tr * md.ptiles_c;
+    const int64_t item = t - __ldg(p.ptile_prefix + mi);
     const float s = *md.scale;
     const float lr = p.lr * md.lr_mult;
     const float decay = 1.0f - lr * p.wd;
     const E* X = reinterpret_cast<const E*>(md.X[0]);
     E* W = reinterpret_cast<E*>(md.W);
-    for (int k = threadIdx.x; k < kPT * kPT; k += blockDim.x) {
-      const int64_t r = tr * kPT + k / kPT, c = tc * kPT + k % kPT;
-      if (r >= md.rows || c >= md.cols) continue;
+    int64_t r0, c0, nr, nc;
+    if (md.T) {
+      const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+      r0 = tr * kTR; c0 = tc * kTC; nr = kTR; nc = kTC;
+    } else {
+      r0 = 0; c0 = item * kFlatChunk; nr = 1; nc = kFlatChunk;   // flat element range
+    }
+    for (int k = threadIdx.x; k < nr * nc; k += blockDim.x) {
+      int64_t r, c;
+      if (md.T) {
+        r = r0 + k / nc; c = c0 + k % nc;
+        if (r >= md.rows || c >= md.cols) continue;
+      } else {
+        const int64_t e = c0 + k;
+        if (e >= md.rows * md.cols) continue;
+        r = e / md.cols; c = e - r * md.cols;
+      }
       const float x = s * to_f<E>(md.T ? X[c * md.ldx + r] : X[r * md.ldx + c]);
       E* wp = W + r * md.cols + c;
       if (md.mode == kModeOrtho) *wp = from_f<E>(x);
