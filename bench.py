@@ -33,6 +33,12 @@ sys.path.insert(0, HERE)
 METRIC = "Muon-step ms & NS TFLOP/s (Llama-8B shapes), % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage per full
+# Llama-8B launch: the one-layer ncu capture (--workload llama8b_layer) scaled by 32 identical
+# layers; valid only for the kernel source it was measured on.
+PROFILED_TRAFFIC = {"kernels_sha256_prefix": "da9e8cb50425422a", "workload": "llama8b",
+                    "gemm_bytes_per_launch": 32 * 1.282e9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -47,6 +53,19 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     return ap.parse_args()
+
+
+def profiled_traffic(workload: str):
+    """The profiled DRAM bytes per GEMM launch, or None when the kernels changed since."""
+    import hashlib
+    path = os.path.join(HERE, "newton_schulz_09_b200", "csrc", "kernels.cuh")
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if sha.startswith(PROFILED_TRAFFIC["kernels_sha256_prefix"]) and workload == PROFILED_TRAFFIC["workload"]:
+        return PROFILED_TRAFFIC["gemm_bytes_per_launch"]
+    return None
 
 
 def load_peaks():
@@ -292,7 +311,8 @@ def run_ours(args):
     roofline = {
         "kernel": "ns_stage_kernel<GEMM, bf16>", "bound": "tensor",
         "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
-        "frac": (gemm_tf / peak) if gemm_tf else None, "traffic": None,
+        "frac": (gemm_tf / peak) if gemm_tf else None, "traffic": profiled_traffic(wl.name),
+        "traffic_unit": "bytes per launch (ncu, one-layer capture x 32)",
         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
         "syrk": {"achieved": syrk_tf, "frac": (syrk_tf / peak) if syrk_tf else None},
         "stage_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},

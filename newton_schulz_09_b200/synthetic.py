@@ -115,12 +115,15 @@ def workload(name: str) -> Workload:
                         weight_decay=0.01, seed=2)
     if name == "llama8b":
         return Workload(name, torch.bfloat16, _llama8b_specs(), grad_std=1e-4, seed=3)
+    if name == "llama8b_layer":
+        # one layer of the stack: the small case for profiler captures
+        return Workload(name, torch.bfloat16, _llama8b_specs(1), grad_std=1e-4, seed=3)
     if name == "mixed1024":
         return Workload(name, torch.bfloat16, mixed_shapes(), grad_std=1.0, seed=4)
     raise KeyError(name)
 
 
-WORKLOADS = ("fp32_256x512", "tinymlp", "square4096", "llama8b", "mixed1024")
+WORKLOADS = ("fp32_256x512", "tinymlp", "square4096", "llama8b", "mixed1024", "llama8b_layer")
 
 
 def _gen(seed: int, device) -> torch.Generator:
