@@ -122,6 +122,46 @@ int dmuon_muon_step_batched_ex(void* const params[], const void* const grads[], 
                                int nesterov, float weight_decay, int ns_steps, void* workspace,
                                size_t ws_bytes, dmuon_stream_t stream);
 
+/*
+ * Options of dmuon_muon_step_batched_opts.  Fill with
+ * dmuon_step_options_default() (the pages' defaults: lr 0.02, momentum 0.95,
+ * Nesterov, 5 steps of the cubic 1.5 / -0.5 iteration, no weight decay, no lr
+ * scaling, no clipping), then change fields.
+ *   ns_a, ns_b      coefficients of the cubic step X <- a X + b (X X^T) X
+ *                   (the training guide's custom NewtonSchulz coefficients,
+ *                   "超参数指南"; the blog's step is a = 1.5, b = -0.5).
+ *   lr_scale        DMUON_LR_PLAIN: lr as given.  DMUON_LR_SQRT_MAX: each
+ *                   matrix uses lr * 0.2 * sqrt(max(rows, cols)) in place of lr
+ *                   everywhere in its update (the guide's "internally scaled
+ *                   per-param" note), weight decay included.
+ *   max_grad_norm   > 0: Muon-only gradient clipping before the momentum
+ *                   update (the guide's "梯度裁剪" section): with
+ *                   ||g|| = sqrt(sum of g^2 over every matrix of the call),
+ *                   each gradient enters the momentum as fl32(g * c),
+ *                   c = fl32(min(1, max_grad_norm / (||g|| + 1e-6))).  The
+ *                   gradient tensors themselves are not modified.
+ *   grad_norm_out   optional DEVICE pointer (fp32): receives ||g|| when
+ *                   clipping is on.
+ */
+enum { DMUON_LR_PLAIN = 0, DMUON_LR_SQRT_MAX = 1 };
+typedef struct {
+  size_t struct_size; /* sizeof(dmuon_step_options) */
+  float lr, momentum, weight_decay;
+  int nesterov, ns_steps;
+  float ns_a, ns_b;
+  int lr_scale;
+  float max_grad_norm;
+  float* grad_norm_out;
+} dmuon_step_options;
+void dmuon_step_options_default(dmuon_step_options* opts);
+
+/* One Muon update of `count` matrices with options (arguments otherwise as
+ * dmuon_muon_step_batched).  workspace may be NULL (library arena) or a
+ * caller buffer of ws_bytes >= dmuon_workspace_bytes(). */
+int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[], float* const bufs[],
+                                 const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
+                                 void* workspace, size_t ws_bytes, dmuon_stream_t stream);
+
 /* Scratch bytes needed by dmuon_muon_step_batched_ex for these shapes
  * (matrices with a NULL gradient may be left out or counted; counting them
  * over-estimates).  Returns 0 for invalid shapes. */

@@ -22,6 +22,7 @@ __all__ = [
     "dmuon_last_error", "dmuon_backend_string", "dmuon_device_status", "dmuon_release_cache",
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
+    "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
 ]
 
 #: Kernel kinds of dmuon_stage_times(), in order.
@@ -46,6 +47,18 @@ class DmuonError(RuntimeError):
 class DmuonShape(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("param_dtype", ctypes.c_int32), ("grad_dtype", ctypes.c_int32)]
+
+
+DMUON_LR_PLAIN = 0
+DMUON_LR_SQRT_MAX = 1
+
+
+class DmuonStepOptions(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_size_t), ("lr", ctypes.c_float),
+                ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("nesterov", ctypes.c_int), ("ns_steps", ctypes.c_int),
+                ("ns_a", ctypes.c_float), ("ns_b", ctypes.c_float), ("lr_scale", ctypes.c_int),
+                ("max_grad_norm", ctypes.c_float), ("grad_norm_out", ctypes.c_void_p)]
 
 
 def library_path() -> str:
@@ -83,6 +96,9 @@ def load_library() -> ctypes.CDLL:
                                     ctypes.POINTER(ctypes.c_int64), i32, i32]),
         "dmuon_launch_count": (ctypes.c_int64, []),
         "dmuon_ns_orthogonalize_noalloc": (i32, [vp, i64, i64, i32, vp]),
+        "dmuon_step_options_default": (None, [ctypes.POINTER(DmuonStepOptions)]),
+        "dmuon_muon_step_batched_opts": (i32, [pp, pp, pp, sp, i32, ctypes.POINTER(DmuonStepOptions),
+                                               vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -215,6 +231,42 @@ def dmuon_muon_step_batched(params, grads, bufs, lr: float = 0.02, momentum: flo
     with torch.cuda.device(b.device):
         _check(lib.dmuon_muon_step_batched(*b.args(), lr, momentum, 1 if nesterov else 0,
                                            weight_decay, ns_steps, _stream(b.device)))
+
+
+def dmuon_muon_step_batched_opts(params, grads, bufs, lr: float = 0.02, momentum: float = 0.95,
+                                 nesterov: bool = True, weight_decay: float = 0.0,
+                                 ns_steps: int = 5, ns_coefficients=(1.5, -0.5),
+                                 lr_scale: str = "plain", max_grad_norm: float = 0.0,
+                                 grad_norm_out: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None) -> None:
+    """One Muon update with the options of dmuon_step_options: custom cubic
+    coefficients (a, b), per-matrix lr scale ("plain" or "sqrt_max":
+    lr * 0.2 * sqrt(max(rows, cols))), Muon-only global-norm gradient
+    clipping (max_grad_norm > 0; the pre-clip norm goes to ``grad_norm_out``,
+    a one-element fp32 CUDA tensor, when given).  Scratch from ``workspace``
+    or the library arena."""
+    lib = load_library()
+    b = _Batch(params, grads, bufs)
+    if b.n == 0:
+        return
+    o = DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
+    o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
+    o.ns_a, o.ns_b = ns_coefficients
+    o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
+    o.max_grad_norm = max_grad_norm
+    if grad_norm_out is not None:
+        if (grad_norm_out.dtype != torch.float32 or not grad_norm_out.is_cuda
+                or grad_norm_out.numel() < 1):
+            raise ValueError("grad_norm_out must be a CUDA fp32 tensor with one element")
+        o.grad_norm_out = grad_norm_out.data_ptr()
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    with torch.cuda.device(b.device):
+        _check(lib.dmuon_muon_step_batched_opts(*b.args(), ctypes.byref(o), ws_ptr, ws_bytes,
+                                                _stream(b.device)))
 
 
 def dmuon_muon_step_batched_ex(params, grads, bufs, lr: float = 0.02, momentum: float = 0.95,

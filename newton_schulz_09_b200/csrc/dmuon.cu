@@ -105,6 +105,17 @@ struct MatIn {
   int64_t rows, cols;
   int pdt, gdt;
   int mode;
+  float lr_mult = 1.0f;   // per-matrix factor on lr
+};
+
+// Scalars and switches of one call.
+struct StepOpts {
+  float lr = 0.0f, mu = 0.0f, wd = 0.0f;
+  int nesterov = 0, steps = 0;
+  float ca = 1.5f, cb = -0.5f;      // cubic coefficients
+  int lr_scale = DMUON_LR_PLAIN;
+  float max_norm = 0.0f;            // > 0: global-norm gradient clipping
+  float* norm_out = nullptr;        // device pointer for the pre-clip norm
 };
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -148,11 +159,13 @@ struct GroupLayout {
   int dtype;
   std::vector<int> idx;    // indices into the input matrix array
   size_t partials, scales; // byte offsets
+  size_t gpartials;        // byte offset of the gradient-norm partials (double per item)
   int64_t ptiles;
 };
 struct Layout {
   std::vector<MatLayout> mats;   // parallel to the input matrices
   std::vector<GroupLayout> groups;
+  size_t clip = 0;               // byte offset of {clip coefficient, gradient norm}
   size_t bytes = 0;
 };
 
@@ -198,8 +211,10 @@ Layout make_layout(const std::vector<MatIn>& in, int steps) {
     }
     g.partials = off; off = align_up(off + sizeof(float) * g.ptiles, 1024);
     g.scales = off; off = align_up(off + sizeof(float) * g.idx.size(), 1024);
+    g.gpartials = off; off = align_up(off + sizeof(double) * g.ptiles, 1024);
     L.groups.push_back(std::move(g));
   }
+  L.clip = off; off = align_up(off + 2 * sizeof(float), 1024);
   L.bytes = off;
   return L;
 }
@@ -215,6 +230,7 @@ struct GroupPlan {
   const int* gemm_order; const int* gemm_prefix;
   const int64_t* pprefix;
   float* partials;
+  double* gpartials;
 };
 
 struct Plan {
@@ -224,6 +240,7 @@ struct Plan {
   void* dmem = nullptr;
   const MatDesc* d_mats = nullptr;
   const MatMaps* d_maps = nullptr;
+  float* clip = nullptr;          // workspace: {clip coefficient, gradient norm}
   std::vector<GroupPlan> groups;
   ~Plan() {
     if (dmem) cudaFree(dmem);
@@ -305,7 +322,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   for (const MatIn& x : in) {
     put(key, x.W); put(key, x.G); put(key, x.buf);
     put(key, x.rows); put(key, x.cols);
-    put(key, x.pdt); put(key, x.gdt); put(key, x.mode);
+    put(key, x.pdt); put(key, x.gdt); put(key, x.mode); put(key, x.lr_mult);
   }
   const uint64_t h = fnv1a(key.data(), key.size());
   for (auto it = g_plans.begin(); it != g_plans.end(); ++it) {
@@ -363,7 +380,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
       d.Xop[1] = (ml.o1 != SIZE_MAX) ? wsb + ml.o1 : nullptr;
       d.A = (ml.a != SIZE_MAX) ? wsb + ml.a : nullptr;
       d.scale = reinterpret_cast<float*>(wsb + g.scales) + k;
-      d.lr_mult = 1.0f;
+      d.lr_mult = x.lr_mult;
       d.m = static_cast<int>(ml.m); d.n = static_cast<int>(ml.n);
       d.T = x.rows > x.cols ? 1 : 0;
       d.mode = x.mode;
@@ -416,6 +433,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     gp.syrk_tiles = static_cast<int>(st);
     gp.gemm_tiles = static_cast<int>(gt);
     gp.partials = reinterpret_cast<float*>(wsb + g.partials);
+    gp.gpartials = reinterpret_cast<double*>(wsb + g.gpartials);
     P->groups.push_back(gp);
     first += gp.nmat;
   }
@@ -458,6 +476,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     gp.gemm_order = reinterpret_cast<const int*>(base + o_g[gi * 5 + 3]);
     gp.gemm_prefix = reinterpret_cast<const int*>(base + o_g[gi * 5 + 4]);
   }
+  P->clip = reinterpret_cast<float*>(wsb + L.clip);
   P->d_mats = reinterpret_cast<const MatDesc*>(base + o_desc);
   P->d_maps = reinterpret_cast<const MatMaps*>(base + o_maps);
   g_plans.emplace_front(std::move(P));
@@ -525,18 +544,37 @@ void launch_ns_stage(const NsParams& np, const DeviceInfo& d, cudaStream_t st) {
 }
 
 template <typename E>
-void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float lr, float mu,
-                  int nesterov, float wd, int steps, cudaStream_t st) {
+ElemParams elem_params(const Plan& P, const GroupPlan& g, const StepOpts& o) {
   ElemParams ep;
   ep.mats = P.d_mats + g.first;
   ep.ptile_prefix = g.pprefix;
   ep.partials = g.partials;
   ep.nmat = g.nmat;
   ep.ntiles = g.ptiles;
-  ep.mu = mu;
-  ep.nesterov = nesterov;
-  ep.lr = lr;
-  ep.wd = wd;
+  ep.mu = o.mu;
+  ep.nesterov = o.nesterov;
+  ep.lr = o.lr;
+  ep.wd = o.wd;
+  ep.clip = o.max_norm > 0.0f ? P.clip : nullptr;
+  ep.gpartials = g.gpartials;
+  return ep;
+}
+
+template <typename E>
+void launch_grad_norm(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const StepOpts& o,
+                      cudaStream_t st) {
+  const ElemParams ep = elem_params<E>(P, g, o);
+  const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
+  LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
+  grad_norm_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+}
+
+template <typename E>
+void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const StepOpts& o,
+                  cudaStream_t st) {
+  const float lr = o.lr, wd = o.wd;
+  const int steps = o.steps;
+  const ElemParams ep = elem_params<E>(P, g, o);
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
@@ -557,6 +595,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float 
   np.nmat = g.nmat;
   np.lr = lr;
   np.wd = wd;
+  np.ca = o.ca;
+  np.cb = o.cb;
   np.err = d.err;
   np.wait_limit_ns = kWaitLimitNs;
   for (int s = 0; s < steps; ++s) {
@@ -580,12 +620,30 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, float 
   }
 }
 
-int launch_plan(const Plan& P, float lr, float mu, int nesterov, float wd, int steps,
-                cudaStream_t st) {
+int launch_plan(const Plan& P, const StepOpts& o, cudaStream_t st) {
   const DeviceInfo& d = g_dev[P.device];
+  if (o.max_norm > 0.0f) {
+    // Global gradient norm over every matrix of the call, then the clip
+    // coefficient that the prologues apply.
+    ClipParams cp;
+    cp.part[0] = cp.part[1] = nullptr;
+    cp.count[0] = cp.count[1] = 0;
+    for (size_t gi = 0; gi < P.groups.size() && gi < 2; ++gi) {
+      const GroupPlan& g = P.groups[gi];
+      if (g.dtype == DMUON_BF16) launch_grad_norm<__nv_bfloat16>(P, g, d, o, st);
+      else launch_grad_norm<float>(P, g, d, o, st);
+      cp.part[gi] = g.gpartials;
+      cp.count[gi] = g.ptiles;
+    }
+    cp.max_norm = o.max_norm;
+    cp.coef = P.clip;
+    cp.norm_out = o.norm_out;
+    LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
+    clip_coef_kernel<<<1, 256, 0, st>>>(cp);
+  }
   for (const GroupPlan& g : P.groups) {
-    if (g.dtype == DMUON_BF16) launch_group<__nv_bfloat16>(P, g, d, lr, mu, nesterov, wd, steps, st);
-    else launch_group<float>(P, g, d, lr, mu, nesterov, wd, steps, st);
+    if (g.dtype == DMUON_BF16) launch_group<__nv_bfloat16>(P, g, d, o, st);
+    else launch_group<float>(P, g, d, o, st);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -622,7 +680,8 @@ int arena_get(int dev, cudaStream_t st, size_t bytes, void** out) {
 }
 
 int gather(void* const params[], const void* const grads[], float* const bufs[],
-           const dmuon_shape shapes[], int count, int ns_steps, std::vector<MatIn>* in) {
+           const dmuon_shape shapes[], int count, int ns_steps, int lr_scale,
+           std::vector<MatIn>* in) {
   if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count must be >= 0");
   if (ns_steps < 0 || ns_steps > DMUON_MAX_STEPS)
     return fail(DMUON_ERR_INVALID_ARG, "ns_steps must be in [0, %d]", DMUON_MAX_STEPS);
@@ -641,6 +700,9 @@ int gather(void* const params[], const void* const grads[], float* const bufs[],
     x.pdt = shapes[i].param_dtype;
     x.gdt = shapes[i].grad_dtype;
     x.mode = kModeMuon;
+    x.lr_mult = 1.0f;
+    if (lr_scale == DMUON_LR_SQRT_MAX)
+      x.lr_mult = static_cast<float>(0.2 * std::sqrt(static_cast<double>(std::max(x.rows, x.cols))));
     const int r = check_matrix(x, i);
     if (r != DMUON_OK) return r;
     in->push_back(x);
@@ -648,8 +710,9 @@ int gather(void* const params[], const void* const grads[], float* const bufs[],
   return DMUON_OK;
 }
 
-int run(const std::vector<MatIn>& in, int steps, void* ws, size_t ws_bytes, bool own_ws,
-        float lr, float mu, int nesterov, float wd, cudaStream_t st) {
+int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, const StepOpts& o,
+        cudaStream_t st) {
+  const int steps = o.steps;
   if (in.empty()) return DMUON_OK;
   std::lock_guard<std::mutex> lk(g_api_mu);
   int dev = 0;
@@ -669,7 +732,28 @@ int run(const std::vector<MatIn>& in, int steps, void* ws, size_t ws_bytes, bool
   Plan* plan = nullptr;
   r = get_plan(in, steps, ws, dev, &plan);
   if (r != DMUON_OK) return r;
-  return launch_plan(*plan, lr, mu, nesterov, wd, steps, st);
+  return launch_plan(*plan, o, st);
+}
+
+int check_opts(const StepOpts& o) {
+  if (!std::isfinite(o.lr) || !std::isfinite(o.mu) || !std::isfinite(o.wd) || !std::isfinite(o.ca) ||
+      !std::isfinite(o.cb))
+    return fail(DMUON_ERR_INVALID_ARG, "lr, momentum, weight_decay and the NS coefficients must be finite");
+  if (!(o.max_norm >= 0.0f) || !std::isfinite(o.max_norm))
+    return fail(DMUON_ERR_INVALID_ARG, "max_grad_norm must be finite and >= 0");
+  if (o.lr_scale != DMUON_LR_PLAIN && o.lr_scale != DMUON_LR_SQRT_MAX)
+    return fail(DMUON_ERR_INVALID_ARG, "unknown lr_scale %d", o.lr_scale);
+  return DMUON_OK;
+}
+
+StepOpts plain_opts(float lr, float momentum, int nesterov, float wd, int steps) {
+  StepOpts o;
+  o.lr = lr;
+  o.mu = momentum;
+  o.nesterov = nesterov ? 1 : 0;
+  o.wd = wd;
+  o.steps = steps;
+  return o;
 }
 
 }  // namespace
@@ -684,22 +768,65 @@ int dmuon_muon_step_batched_ex(void* const params[], const void* const grads[], 
                                int nesterov, float weight_decay, int ns_steps, void* workspace,
                                size_t ws_bytes, dmuon_stream_t stream) {
   t_last_error.clear();
-  std::vector<MatIn> in;
-  int r = gather(params, grads, bufs, shapes, count, ns_steps, &in);
+  const StepOpts o = plain_opts(lr, momentum, nesterov, weight_decay, ns_steps);
+  int r = check_opts(o);
   if (r != DMUON_OK) return r;
-  return run(in, ns_steps, workspace, ws_bytes, false, lr, momentum, nesterov ? 1 : 0, weight_decay,
-             reinterpret_cast<cudaStream_t>(stream));
+  std::vector<MatIn> in;
+  r = gather(params, grads, bufs, shapes, count, ns_steps, DMUON_LR_PLAIN, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, workspace, ws_bytes, false, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dmuon_muon_step_batched(void* const params[], const void* const grads[], float* const bufs[],
                             const dmuon_shape shapes[], int count, float lr, float momentum,
                             int nesterov, float weight_decay, int ns_steps, dmuon_stream_t stream) {
   t_last_error.clear();
-  std::vector<MatIn> in;
-  int r = gather(params, grads, bufs, shapes, count, ns_steps, &in);
+  const StepOpts o = plain_opts(lr, momentum, nesterov, weight_decay, ns_steps);
+  int r = check_opts(o);
   if (r != DMUON_OK) return r;
-  return run(in, ns_steps, nullptr, 0, true, lr, momentum, nesterov ? 1 : 0, weight_decay,
-             reinterpret_cast<cudaStream_t>(stream));
+  std::vector<MatIn> in;
+  r = gather(params, grads, bufs, shapes, count, ns_steps, DMUON_LR_PLAIN, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, nullptr, 0, true, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+void dmuon_step_options_default(dmuon_step_options* o) {
+  if (!o) return;
+  std::memset(o, 0, sizeof(*o));
+  o->struct_size = sizeof(dmuon_step_options);
+  o->lr = 0.02f;
+  o->momentum = 0.95f;
+  o->nesterov = 1;
+  o->weight_decay = 0.0f;
+  o->ns_steps = 5;
+  o->ns_a = 1.5f;
+  o->ns_b = -0.5f;
+  o->lr_scale = DMUON_LR_PLAIN;
+  o->max_grad_norm = 0.0f;
+  o->grad_norm_out = nullptr;
+}
+
+int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[], float* const bufs[],
+                                 const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
+                                 void* workspace, size_t ws_bytes, dmuon_stream_t stream) {
+  t_last_error.clear();
+  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
+  if (opts->struct_size != sizeof(dmuon_step_options))
+    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
+                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
+  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
+  o.ca = opts->ns_a;
+  o.cb = opts->ns_b;
+  o.lr_scale = opts->lr_scale;
+  o.max_norm = opts->max_grad_norm;
+  o.norm_out = opts->grad_norm_out;
+  int r = check_opts(o);
+  if (r != DMUON_OK) return r;
+  if (o.norm_out && !aligned(o.norm_out, 4)) return fail(DMUON_ERR_INVALID_ARG, "grad_norm_out misaligned");
+  std::vector<MatIn> in;
+  r = gather(params, grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
+  if (r != DMUON_OK) return r;
+  return run(in, workspace, ws_bytes, workspace == nullptr, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps) {
@@ -743,7 +870,7 @@ int dmuon_ns_orthogonalize_ex(void* X, int64_t m, int64_t n, int steps, int dtyp
   std::vector<MatIn> in;
   int r = ortho_input(X, m, n, steps, dtype, &in);
   if (r != DMUON_OK) return r;
-  return run(in, steps, workspace, ws_bytes, false, 0.0f, 0.0f, 0, 0.0f,
+  return run(in, workspace, ws_bytes, false, plain_opts(0.0f, 0.0f, 0, 0.0f, steps),
              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -752,7 +879,7 @@ int dmuon_ns_orthogonalize(void* X, int64_t m, int64_t n, int steps, dmuon_strea
   std::vector<MatIn> in;
   int r = ortho_input(X, m, n, steps, DMUON_BF16, &in);
   if (r != DMUON_OK) return r;
-  return run(in, steps, nullptr, 0, true, 0.0f, 0.0f, 0, 0.0f,
+  return run(in, nullptr, 0, true, plain_opts(0.0f, 0.0f, 0, 0.0f, steps),
              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -986,6 +1113,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   ep.nesterov = 0;
   ep.lr = 0.0f;
   ep.wd = 0.0f;
+  ep.clip = nullptr;
+  ep.gpartials = nullptr;
   const int pgrid = static_cast<int>(std::min<int64_t>(ml.ptiles, static_cast<int64_t>(di.sms) * 8));
   prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, 0, st>>>(ep);
   finalize_kernel<<<1, 32, 0, st>>>(ep);
@@ -1001,6 +1130,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     np.nmat = 1;
     np.lr = 0.0f;
     np.wd = 0.0f;
+    np.ca = 1.5f;
+    np.cb = -0.5f;
     np.err = di.err;
     np.wait_limit_ns = kWaitLimitNs;
     for (int s = 0; s < steps; ++s) {

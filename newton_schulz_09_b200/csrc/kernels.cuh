@@ -83,6 +83,7 @@ struct NsParams {
   int first;               // fold s into this stage (first NS step)
   int last;                // GEMM writes the final result (last NS step)
   float lr, wd;            // update scalars (used when last)
+  float ca, cb;            // cubic coefficients: X <- ca X + cb (X X^T) X
   int* err;                // device error word
   uint64_t wait_limit_ns;
 };
@@ -96,6 +97,8 @@ struct ElemParams {
   float mu;
   int nesterov;
   float lr, wd;                 // apply_kernel only
+  const float* clip;            // gradient scale (global-norm clipping) or nullptr
+  double* gpartials;            // grad_norm_kernel: one partial sum of g^2 per item
 };
 
 // ------------------------------------------------------------------ helpers
@@ -293,8 +296,8 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
             const int col = c * 8 + 2 * j;
             const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
             const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
-            __nv_bfloat162 yv = __floats2bfloat162_rn(cs * (1.5f * xf.x - 0.5f * a0),
-                                                      cs * (1.5f * xf.y - 0.5f * a1));
+            __nv_bfloat162 yv = __floats2bfloat162_rn(cs * (p.ca * xf.x + p.cb * a0),
+                                                      cs * (p.ca * xf.y + p.cb * a1));
             wv[j] = *reinterpret_cast<uint32_t*>(&yv);
           }
           *ptr = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -393,7 +396,7 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
           }
           float y[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = cs * (1.5f * x[j] - 0.5f * __uint_as_float(v[j]));
+          for (int j = 0; j < 32; ++j) y[j] = cs * (p.ca * x[j] + p.cb * __uint_as_float(v[j]));
           if (!p.last) {
             E* dst = Xn + static_cast<int64_t>(R) * ldx + C0;
             if (full_chunk) {
@@ -718,9 +721,15 @@ __device__ __forceinline__ void store8_x(E* dst, bool vec, int valid, const floa
   }
 }
 
-// Momentum / Nesterov on 8 values; returns M, updates b in place.
-__device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, const float (&g)[8],
+// Momentum / Nesterov on 8 values; returns M, updates b in place.  With
+// gradient clipping the gradient enters as fl32(g * c).
+__device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, float (&g)[8],
                                           float (&b)[8], float (&M)[8]) {
+  if (p.clip != nullptr) {
+    const float c = *p.clip;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(g[e], c);
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     if (has_buf) {
@@ -865,6 +874,89 @@ __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_consta
       p.partials[t] = acc;
     }
     __syncthreads();
+  }
+}
+
+// Sum of squares of the gradients (fp64 accumulation), one partial per
+// prologue work item (the items cover every gradient element exactly once).
+template <typename E>
+__global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_constant__ ElemParams p) {
+  __shared__ double red[kPThreads / 32];
+  const int tid = threadIdx.x;
+  for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
+    const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
+    const MatDesc& md = p.mats[mi];
+    const int64_t item = t - __ldg(p.ptile_prefix + mi);
+    double ss = 0.0;
+    const int64_t rows = md.rows, cols = md.cols;
+    if (!md.T) {
+      const int64_t numel = rows * cols;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int64_t e = item * kFlatChunk + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+        if (e >= numel) break;
+        const int valid = static_cast<int>(numel - e < 8 ? numel - e : 8);
+        float g[8];
+        load8_in(md, e, md.vec4 && valid == 8, valid, g);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += static_cast<double>(g[k]) * g[k];
+      }
+    } else {
+      const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+      const int64_t c = tc * kTC + (tid & 15) * 8;
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        const int64_t r = tr * kTR + (tid >> 4) + 16 * i;
+        if (r >= rows || c >= cols) continue;
+        const int valid = static_cast<int>(cols - c < 8 ? cols - c : 8);
+        const int64_t idx = r * cols + c;
+        float g[8];
+        load8_in(md, idx, md.vec4 && valid == 8 && ((idx & 7) == 0), valid, g);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += static_cast<double>(g[k]) * g[k];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      double acc = 0.0;
+#pragma unroll
+      for (int w = 0; w < kPThreads / 32; ++w) acc += red[w];
+      p.gpartials[t] = acc;
+    }
+    __syncthreads();
+  }
+}
+
+// Global-norm clipping coefficient over all gradients of a call (one block,
+// fixed-order sums): c = min(1, max_norm / (||g|| + 1e-6)); optionally also
+// the norm itself.
+struct ClipParams {
+  const double* part[2];   // per dtype group: partial sums of g^2
+  int64_t count[2];
+  float max_norm;
+  float* coef;             // out: device scalar read by the prologue
+  float* norm_out;         // out (optional): the gradient norm before clipping
+};
+
+__global__ void clip_coef_kernel(const __grid_constant__ ClipParams cp) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int gi = 0; gi < 2; ++gi)
+    for (int64_t i = threadIdx.x; i < cp.count[gi]; i += blockDim.x) acc += cp.part[gi][i];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+    const double nrm = sqrt(tot);
+    const double c = static_cast<double>(cp.max_norm) / (nrm + 1e-6);
+    *cp.coef = static_cast<float>(c < 1.0 ? c : 1.0);
+    if (cp.norm_out) *cp.norm_out = static_cast<float>(nrm);
   }
 }
 

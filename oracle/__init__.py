@@ -8,7 +8,9 @@ from .muon_oracle import (  # noqa: F401
     NORM_EPS,
     NS_A,
     NS_B,
+    clip_coefficient,
     frobenius_normalize,
+    lr_scale_factor,
     momentum_update,
     muon_step,
     muon_weight_update,

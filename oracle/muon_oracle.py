@@ -27,7 +27,12 @@ Readings where the pages are silent (each listed in the design doc):
 * Weight decay is decoupled and uses the pre-update weight:
   W' = W (1 - lr wd) - lr X.
 * The per-parameter lr scale "0.2 sqrt(max(m, n))" mentioned in the guide's
-  hyper-parameter table is not applied (the blog's step uses plain ``-lr``).
+  hyper-parameter table is off by default (the blog's step uses plain
+  ``-lr``); when requested it replaces lr in the whole update, weight decay
+  included.
+* Gradient clipping (guide, "梯度裁剪") scales every gradient of the call by
+  c = min(1, max_norm / (||g|| + 1e-6)) before the momentum update, with the
+  2-norm over all of them; the gradient enters as fl32(g * c).
 * The transpose test is strict (rows > cols), as in the blog listing.
 
 All pins that tie these functions to the pages and to mathematics live in
@@ -78,17 +83,20 @@ def frobenius_normalize(G: np.ndarray) -> np.ndarray:
     return G / (norm + NORM_EPS)
 
 
-def ns_iteration(X: np.ndarray) -> np.ndarray:
-    """One cubic step X <- 1.5 X - 0.5 (X X^T) X  (blog, "Muon 核心")."""
+def ns_iteration(X: np.ndarray, a: float = NS_A, b: float = NS_B) -> np.ndarray:
+    """One cubic step X <- a X + b (X X^T) X; the blog's step ("Muon 核心")
+    is a = 1.5, b = -0.5, other (a, b) are the training guide's custom
+    coefficients ("超参数指南", ns_backend row)."""
     A = X @ X.T
-    return NS_A * X + NS_B * (A @ X)
+    return a * X + b * (A @ X)
 
 
-def newton_schulz(G: np.ndarray, steps: int) -> np.ndarray:
+def newton_schulz(G: np.ndarray, steps: int, coeffs=(NS_A, NS_B)) -> np.ndarray:
     """Orthogonalise one 2-D matrix with ``steps`` cubic Newton-Schulz steps.
 
     Blog, "Muon 核心" listing: transpose when rows > cols, normalise, iterate,
-    transpose back.  Returns fp64 with the input's shape.
+    transpose back.  Returns fp64 with the input's shape.  ``coeffs`` are the
+    float32 values (a, b) the caller passes through the C ABI.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
@@ -98,8 +106,9 @@ def newton_schulz(G: np.ndarray, steps: int) -> np.ndarray:
     transposed = G.shape[0] > G.shape[1]
     X = G.T.copy() if transposed else G.copy()
     X = frobenius_normalize(X)
+    a, b = (float(np.float32(c)) for c in coeffs)
     for _ in range(steps):
-        X = ns_iteration(X)
+        X = ns_iteration(X, a, b)
     return X.T.copy() if transposed else X
 
 
@@ -112,17 +121,47 @@ def muon_weight_update(W: np.ndarray, X: np.ndarray, lr: float, wd: float) -> np
     return np.asarray(W, dtype=np.float64) * (1.0 - lr64 * wd64) - lr64 * X
 
 
+def lr_scale_factor(rows: int, cols: int) -> float:
+    """Per-parameter lr factor 0.2 sqrt(max(m, n)) (training guide,
+    "超参数指南", lr row), as the float32 the library multiplies lr by."""
+    return float(np.float32(0.2 * np.sqrt(float(max(rows, cols)))))
+
+
+def clip_coefficient(grads, max_norm: float):
+    """Muon-only global-norm clipping (training guide, "梯度裁剪": global
+    p-norm clipping of the Muon gradients before momentum and NS), with p = 2:
+    ||g|| over every gradient, c = min(1, max_norm / (||g|| + 1e-6)) rounded
+    to float32.  Returns (c, ||g||)."""
+    tot = 0.0
+    for g in grads:
+        g64 = np.asarray(g, dtype=np.float64)
+        tot += float(np.sum(g64 * g64))
+    norm = float(np.sqrt(tot))
+    c = min(1.0, float(np.float32(max_norm)) / (norm + 1e-6))
+    return np.float32(c), norm
+
+
 def muon_step(W, g, buf, *, lr: float, momentum: float, nesterov: bool,
-              weight_decay: float, ns_steps: int):
+              weight_decay: float, ns_steps: int, ns_coeffs=(NS_A, NS_B),
+              lr_scale: bool = False, grad_scale=None):
     """One Muon update of one matrix.
 
     Inputs are numpy arrays: ``W`` and ``g`` as float32 (bf16 values widen
-    exactly), ``buf`` float32.  Returns ``(buf_new float32, X fp64, W_new fp64)``.
+    exactly), ``buf`` float32.  ``grad_scale`` (a float32 clip coefficient)
+    makes the gradient enter as fl32(g * c).  ``lr_scale`` multiplies lr by
+    0.2 sqrt(max(rows, cols)) in the whole update.  Returns
+    ``(buf_new float32, X fp64, W_new fp64)``.
     """
-    buf_new = momentum_update(buf, g, momentum)
-    M = nesterov_input(g, buf_new, momentum, nesterov)
-    X = newton_schulz(M, ns_steps)
-    W_new = muon_weight_update(W, X, lr, weight_decay)
+    g32 = np.asarray(g, dtype=np.float32)
+    if grad_scale is not None:
+        g32 = np.multiply(g32, np.float32(grad_scale), dtype=np.float32)
+    buf_new = momentum_update(buf, g32, momentum)
+    M = nesterov_input(g32, buf_new, momentum, nesterov)
+    X = newton_schulz(M, ns_steps, ns_coeffs)
+    lr_eff = lr
+    if lr_scale:
+        lr_eff = float(np.float32(np.float32(lr) * np.float32(lr_scale_factor(*np.shape(g32)))))
+    W_new = muon_weight_update(W, X, lr_eff, weight_decay)
     return buf_new, X, W_new
 
 

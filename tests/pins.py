@@ -258,6 +258,83 @@ def pin_update_closed_form(o, seed: int = 17) -> None:
         assert np.max(np.abs(Wn - Ww)) <= 1e-15
 
 
+def pin_custom_coefficients(o, seed: int = 18) -> None:
+    """Custom cubic coefficients (a, b): a 1x1 input follows s <- a s + b s^3
+    and the spectral map holds with f(s) = a s + b s^3 (float32 a, b)."""
+    rng = np.random.default_rng(seed)
+    for (a, b) in ((1.875, -0.875), (2.0, -1.0)):
+        a32, b32 = float(np.float32(a)), float(np.float32(b))
+        for x in (0.8, -3.0, 1e-6):
+            s_ = x / (abs(x) + EPS)
+            for _ in range(4):
+                s_ = a32 * s_ + b32 * s_ ** 3
+            got = o.newton_schulz(np.array([[x]]), 4, (a, b))[0, 0]
+            assert abs(got - s_) <= 1e-14 * max(1.0, abs(s_)), (a, b, x, got, s_)
+        G = rng.standard_normal((9, 21))
+        U, sig, V = jacobi_svd(G)
+        nrm = math.sqrt(float(np.sum(G * G)))
+        fs = []
+        for sv in sig:
+            t = sv / (nrm + EPS)
+            for _ in range(3):
+                t = a32 * t + b32 * t ** 3
+            fs.append(t)
+        want = (U * np.array(fs)) @ V.T
+        assert _rel(o.newton_schulz(G, 3, (a, b)), want) <= 1e-12
+        assert _rel(o.newton_schulz(G.T, 3, (a, b)), want.T) <= 1e-12
+
+
+def pin_lr_scale(o, seed: int = 19) -> None:
+    """lr scaled by 0.2 sqrt(max(rows, cols)) in the whole update: with the
+    Hadamard input of pin_update_closed_form, W' = W (1 - lr_s wd) - lr_s c_k Q
+    where lr_s = fl32(lr * fl32(0.2 * 4)) for 16 columns."""
+    rng = np.random.default_rng(seed)
+    H = _hadamard(16) / 4.0
+    Q = H[:8].copy()
+    c = 2.0 ** -9
+    g = (c * Q).astype(np.float32)
+    W = (rng.standard_normal(g.shape) * 0.02).astype(np.float32)
+    lr, mu, wd, k = 0.02, 0.95, 0.01, 5
+    _, X, Wn = o.muon_step(W, g, np.zeros_like(g), lr=lr, momentum=mu, nesterov=True,
+                           weight_decay=wd, ns_steps=k, lr_scale=True)
+    alpha = c + float(np.float32(mu)) * c
+    Xw = cubic_map(alpha / (alpha * math.sqrt(8.0) + EPS), k) * Q
+    assert _rel(X, Xw) <= 1e-13
+    lr_s = float(np.float32(np.float32(lr) * np.float32(0.2 * 4.0)))
+    Ww = W.astype(np.float64) * (1.0 - lr_s * float(np.float32(wd))) - lr_s * Xw
+    assert np.max(np.abs(Wn - Ww)) <= 1e-15
+    assert abs(o.lr_scale_factor(14336, 4096) - 0.2 * math.sqrt(14336.0)) < 1e-6
+
+
+def pin_gradient_clipping(o) -> None:
+    """Global-norm clipping before the momentum update: two matrices of +-1/4
+    entries (Hadamard rows) have ||g|| = sqrt(64/16 + 256/16) = sqrt(20) ...
+    here chosen as 4 x 16 and 16 x 16 blocks, ||g||^2 = 4 + 16 = 20.  With
+    max_norm = 1 the coefficient is fl32(1 / (sqrt(20) + 1e-6)), and the new
+    buffer is fl32(fl32(mu buf) + fl32(g c)), checked with exact arithmetic
+    (a nonzero buffer distinguishes clipping before from after momentum)."""
+    H = _hadamard(16) / 4.0
+    g1 = H[:4].astype(np.float32)
+    g2 = H.astype(np.float32)
+    c32, norm = o.clip_coefficient([g1, g2], 1.0)
+    assert abs(norm - math.sqrt(20.0)) <= 1e-15
+    want_c = exact_f32_round(Fraction(1) / (Fraction(math.sqrt(20.0)) + Fraction(1e-6)))
+    assert c32 == want_c
+    assert o.clip_coefficient([g1], 100.0)[0] == np.float32(1.0)       # no clipping below the bound
+    buf = (np.arange(64, dtype=np.float32).reshape(4, 16) - 31.0) * np.float32(0.01)
+    mu = 0.9
+    buf_new, _, _ = o.muon_step(np.zeros_like(g1), g1, buf, lr=0.0, momentum=mu, nesterov=False,
+                                weight_decay=0.0, ns_steps=0, grad_scale=c32)
+    mu32 = Fraction(float(np.float32(mu)))
+    for i in range(4):
+        for j in range(16):
+            gc = exact_f32_round(Fraction(float(g1[i, j])) * Fraction(float(c32)))
+            p = exact_f32_round(mu32 * Fraction(float(buf[i, j])))
+            want = exact_f32_round(Fraction(float(p)) + Fraction(float(gc)))
+            assert buf_new[i, j] == want, (i, j)
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
-            pin_nesterov_post_update, pin_update_closed_form)
+            pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
+            pin_lr_scale, pin_gradient_clipping)

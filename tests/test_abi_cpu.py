@@ -86,16 +86,41 @@ def test_null_gradient_is_skipped_before_any_device_work(lib):
 
 def test_workspace_bytes(lib):
     # One 256x512 bf16 matrix, 5 steps: X0 and X1 (256 x 512), A (256 x 256),
-    # 32 prologue tiles of partials, one scale; regions rounded to 1 KiB.
-    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 5) == 2 * 262144 + 131072 + 1024 + 1024
+    # then 1 KiB regions: norm partials, scales, gradient-norm partials and the
+    # clip scalars (every region rounded up to 1 KiB).
+    small = 4 * 1024
+    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 5) == 2 * 262144 + 131072 + small
     # Tall matrix: same m x n view.
-    assert lib.dmuon_workspace_bytes(_shapes((512, 256)), 1, 5) == 2 * 262144 + 131072 + 1024 + 1024
+    assert lib.dmuon_workspace_bytes(_shapes((512, 256)), 1, 5) == 2 * 262144 + 131072 + small
     # No second iterate and no Gram for steps == 0.
-    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 0) == 262144 + 1024 + 1024
+    assert lib.dmuon_workspace_bytes(_shapes((256, 512)), 1, 0) == 262144 + small
     # Ragged shape: rows padded to 16 bytes (8 bf16 / 4 fp32).
-    assert lib.dmuon_workspace_bytes(_shapes((3, 5)), 1, 1) == 1024 + 1024 + 1024 + 1024
+    assert lib.dmuon_workspace_bytes(_shapes((3, 5)), 1, 1) == 1024 + 1024 + small
     assert lib.dmuon_workspace_bytes(_shapes((0, 5)), 1, 1) == 0
-    assert lib.dmuon_ns_workspace_bytes(256, 512, dm.DMUON_F32) == 4 * 524288 + 262144 + 1024 + 1024
+    assert lib.dmuon_ns_workspace_bytes(256, 512, dm.DMUON_F32) == 4 * 524288 + 262144 + small
+    # Two dtype groups: per-group regions, one clip region.
+    S = (dm.DmuonShape * 2)(dm.DmuonShape(256, 512, dm.DMUON_BF16, dm.DMUON_BF16),
+                            dm.DmuonShape(256, 512, dm.DMUON_F32, dm.DMUON_F32))
+    assert lib.dmuon_workspace_bytes(S, 2, 5) == (2 * 262144 + 131072) + (4 * 524288 + 262144) + 7 * 1024
+
+
+def test_step_options_defaults_and_checks(lib):
+    o = dm.DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    assert o.struct_size == ctypes.sizeof(dm.DmuonStepOptions)
+    assert abs(o.lr - 0.02) < 1e-9 and abs(o.momentum - 0.95) < 1e-7 and o.nesterov == 1
+    assert o.ns_steps == 5 and o.ns_a == 1.5 and o.ns_b == -0.5
+    assert o.lr_scale == dm.DMUON_LR_PLAIN and o.max_grad_norm == 0.0
+    P, G, B = _ptrs(0x10000), _ptrs(0x20000), _ptrs(0x30000)
+    S = _shapes((4, 4))
+    bad = dm.DmuonStepOptions(); lib.dmuon_step_options_default(ctypes.byref(bad)); bad.struct_size = 8
+    assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, ctypes.byref(bad), None, 0, None) == -1
+    assert "struct_size" in dm.dmuon_last_error()
+    for field, value in (("max_grad_norm", -1.0), ("lr_scale", 7), ("ns_a", float("nan"))):
+        x = dm.DmuonStepOptions(); lib.dmuon_step_options_default(ctypes.byref(x))
+        setattr(x, field, value)
+        assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, ctypes.byref(x), None, 0, None) == -1
+    assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, None, None, 0, None) == -1
 
 
 def test_backend_string(lib):

@@ -45,20 +45,28 @@ def _mutant(**overrides):
     for k, v in overrides.items():
         setattr(m, k, v)
     # rebind the module-level helpers so that replaced pieces are used
-    def newton_schulz(G, steps):
+    def newton_schulz(G, steps, coeffs=(1.5, -0.5)):
         G = np.asarray(G, dtype=np.float64)
         transposed = G.shape[0] > G.shape[1]
         X = G.T.copy() if transposed else G.copy()
         X = m.frobenius_normalize(X)
+        a, b = (float(np.float32(c)) for c in coeffs)
         for _ in range(steps):
-            X = m.ns_iteration(X)
+            X = m.ns_iteration(X, a, b)
         return X.T.copy() if transposed else X
 
-    def muon_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps):
-        buf_new = m.momentum_update(buf, g, momentum)
-        M = m.nesterov_input(g, buf_new, momentum, nesterov)
-        X = m.newton_schulz(M, ns_steps)
-        return buf_new, X, m.muon_weight_update(W, X, lr, weight_decay)
+    def muon_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps,
+                  ns_coeffs=(1.5, -0.5), lr_scale=False, grad_scale=None):
+        g32 = np.asarray(g, dtype=np.float32)
+        if grad_scale is not None:
+            g32 = np.multiply(g32, np.float32(grad_scale), dtype=np.float32)
+        buf_new = m.momentum_update(buf, g32, momentum)
+        M = m.nesterov_input(g32, buf_new, momentum, nesterov)
+        X = m.newton_schulz(M, ns_steps, ns_coeffs)
+        lr_eff = lr
+        if lr_scale:
+            lr_eff = float(np.float32(np.float32(lr) * np.float32(m.lr_scale_factor(*np.shape(g32)))))
+        return buf_new, X, m.muon_weight_update(W, X, lr_eff, weight_decay)
 
     if "newton_schulz" not in overrides:
         m.newton_schulz = newton_schulz
@@ -74,12 +82,12 @@ def _no_eps(G):
 
 
 MUTANTS = {
-    "sign_of_cubic_term": dict(ns_iteration=lambda X: 1.5 * X + 0.5 * (X @ X.T) @ X),
-    "coefficient_3_not_1.5": dict(ns_iteration=lambda X: 3.0 * X - 0.5 * (X @ X.T) @ X),
+    "sign_of_cubic_term": dict(ns_iteration=lambda X, a=1.5, b=-0.5: a * X - b * (X @ X.T) @ X),
+    "coefficient_3_not_1.5": dict(ns_iteration=lambda X, a=1.5, b=-0.5: 2 * a * X + b * (X @ X.T) @ X),
     # X^T X in place of X X^T: only expressible for square X (otherwise the
     # shapes do not conform), where it differs unless X is normal.
-    "gram_of_columns": dict(ns_iteration=lambda X: 1.5 * X - 0.5 * ((X.T @ X) @ X if X.shape[0] == X.shape[1] else (X @ X.T) @ X)),
-    "one_step_short": dict(ns_iteration=lambda X: X),
+    "gram_of_columns": dict(ns_iteration=lambda X, a=1.5, b=-0.5: a * X + b * ((X.T @ X) @ X if X.shape[0] == X.shape[1] else (X @ X.T) @ X)),
+    "one_step_short": dict(ns_iteration=lambda X, a=1.5, b=-0.5: X),
     "dropped_norm_eps": dict(frobenius_normalize=_no_eps),
     "eps_on_squared_norm": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64) / np.sqrt(np.sum(np.asarray(G, np.float64) ** 2) + 1e-7)),
     "no_normalisation": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64)),
@@ -91,14 +99,49 @@ MUTANTS = {
 }
 
 
-def _pre_update_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps):
-    M = muon_oracle.nesterov_input(g, buf, momentum, nesterov)       # old buffer
-    buf_new = muon_oracle.momentum_update(buf, g, momentum)
-    X = muon_oracle.newton_schulz(M, ns_steps)
-    return buf_new, X, muon_oracle.muon_weight_update(W, X, lr, weight_decay)
+def _pre_update_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps,
+                     ns_coeffs=(1.5, -0.5), lr_scale=False, grad_scale=None):
+    g32 = np.asarray(g, dtype=np.float32)
+    if grad_scale is not None:
+        g32 = np.multiply(g32, np.float32(grad_scale), dtype=np.float32)
+    M = muon_oracle.nesterov_input(g32, buf, momentum, nesterov)       # old buffer
+    buf_new = muon_oracle.momentum_update(buf, g32, momentum)
+    X = muon_oracle.newton_schulz(M, ns_steps, ns_coeffs)
+    lr_eff = lr
+    if lr_scale:
+        lr_eff = float(np.float32(np.float32(lr) * np.float32(muon_oracle.lr_scale_factor(*np.shape(g32)))))
+    return buf_new, X, muon_oracle.muon_weight_update(W, X, lr_eff, weight_decay)
 
 
 MUTANTS["nesterov_pre_update"] = dict(muon_step=_pre_update_step)
+
+
+def _clip_after_momentum(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps,
+                         ns_coeffs=(1.5, -0.5), lr_scale=False, grad_scale=None):
+    buf_new = muon_oracle.momentum_update(buf, g, momentum)
+    if grad_scale is not None:
+        buf_new = np.multiply(buf_new, np.float32(grad_scale), dtype=np.float32)
+    M = muon_oracle.nesterov_input(g, buf_new, momentum, nesterov)
+    X = muon_oracle.newton_schulz(M, ns_steps, ns_coeffs)
+    return buf_new, X, muon_oracle.muon_weight_update(W, X, lr, weight_decay)
+
+
+def _lr_scale_min_side(W, g, buf, **kw):
+    if kw.get("lr_scale"):
+        kw = dict(kw)
+        kw["lr_scale"] = False
+        kw["lr"] = float(np.float32(kw["lr"] * 0.2 * np.sqrt(min(np.shape(g)))))
+    return muon_oracle.muon_step(W, g, buf, **kw)
+
+
+def _coeffs_ignored(G, steps, coeffs=(1.5, -0.5)):
+    return muon_oracle.newton_schulz(G, steps)
+
+
+MUTANTS["clip_after_momentum"] = dict(muon_step=_clip_after_momentum)
+MUTANTS["lr_scale_min_side"] = dict(muon_step=_lr_scale_min_side)
+MUTANTS["custom_coefficients_ignored"] = dict(newton_schulz=_coeffs_ignored)
+MUTANTS["clip_no_eps"] = dict(clip_coefficient=lambda grads, mx: (np.float32(min(1.0, float(np.float32(mx)) / np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))), float(np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))))
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
