@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-adamw", action="store_true")
     return ap.parse_args()
 
 
@@ -242,6 +243,41 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- ours
+def measure_adamw(dm, dev, stream, world, peaks, steps):
+    """AdamW over the Llama-8B parameters that are not 2-D projections: token
+    embedding and LM head (128256 x 4096 each) and 65 norm weights (4096),
+    bf16 parameters and gradients, fp32 moments; 22 algorithmic bytes per
+    element (p read+write 4, g 2, m and v read+write 16)."""
+    import torch
+    shapes = [(128256 * 4096,), (128256 * 4096,)] + [(4096,)] * 65
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    ps = [(torch.randn(s, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for s in shapes]
+    gs = [(torch.randn(s, generator=gen, device=dev) * 1e-3).to(torch.bfloat16) for s in shapes]
+    ms = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    vs = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    n = sum(s[0] for s in shapes)
+    for t in range(1, 4):
+        dm.dmuon_adamw_step_batched(ps, gs, ms, vs, step=t)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(4, 4 + steps):
+        dm.dmuon_adamw_step_batched(ps, gs, ms, vs, step=t)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    gbs = 22.0 * n / (ms_step * 1e-3) / 1e9
+    out = {"elements": n, "ms_per_step": ms_step, "achieved": gbs, "unit": "GB/s",
+           "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "bound": "hbm",
+           "bytes_per_element": 22}
+    del ps, gs, ms, vs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import newton_schulz_09_b200 as dm
@@ -318,6 +354,11 @@ def run_ours(args):
         "stage_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
     }
 
+    # ---- AdamW of the model's non-orthogonalised parameters (HBM-bound leg)
+    adamw = None
+    if not args.no_adamw and wl.name == "llama8b":
+        adamw = measure_adamw(dm, dev, stream, world, peaks, args.steps)
+
     # ---- end to end through the public API: pinned host grads in, weights out
     e2e = None
     if not args.no_e2e:
@@ -367,7 +408,7 @@ def run_ours(args):
                        "useful_ns_flops_per_step_per_gpu": fl,
                        "l2": f"inputs larger than L2 ({wl.numel * 8 / 1e9:.0f} GB per GPU)",
                        "parallelism": f"replicas x{world}"},
-            "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "adamw": adamw,
             "roofline": roofline, "cpu_baseline": cpu,
         }
         print(json.dumps(line))

@@ -162,6 +162,31 @@ int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[]
                                  const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
                                  void* workspace, size_t ws_bytes, dmuon_stream_t stream);
 
+/*
+ * dmuon_adamw_step_batched -- AdamW for the parameters the Muon path does
+ * not orthogonalise (the training guide's second parameter group of
+ * dmuon.Muon, "第 4 步：创建优化器": adamw_lr, adamw_betas, adamw_eps,
+ * adamw_weight_decay), all tensors of the call in one launch.  Per element,
+ * with c1 = fl32(1 - beta1), c2 = fl32(1 - beta2), bc1 = 1 - beta1^step,
+ * bc2 = 1 - beta2^step:
+ *   m <- fl(fl(beta1 m) + fl(c1 g))                 (two roundings, bit-exact)
+ *   v <- fl(fl(beta2 v) + fl(fl(c2 g) g))
+ *   p <- p (1 - lr wd) - (lr / bc1) m / (sqrt(v) / sqrt(bc2) + eps)   (fp32)
+ *   params[i], grads[i]: device pointers of descs[i].numel elements
+ *   (param_dtype / grad_dtype: DMUON_BF16 or DMUON_F32), any shape, flat;
+ *   grads[i] == NULL skips tensor i.  exp_avgs[i], exp_avg_sqs[i]: fp32
+ *   device buffers of the same length, updated in place.  step >= 1 is the
+ *   step count including this one.  No scratch memory is used.
+ */
+typedef struct {
+  int64_t numel;
+  int32_t param_dtype, grad_dtype;
+} dmuon_tensor_desc;
+int dmuon_adamw_step_batched(void* const params[], const void* const grads[], float* const exp_avgs[],
+                             float* const exp_avg_sqs[], const dmuon_tensor_desc descs[], int count,
+                             float lr, float beta1, float beta2, float eps, float weight_decay,
+                             int64_t step, dmuon_stream_t stream);
+
 /* Scratch bytes needed by dmuon_muon_step_batched_ex for these shapes
  * (matrices with a NULL gradient may be left out or counted; counting them
  * over-estimates).  Returns 0 for invalid shapes. */
@@ -215,7 +240,8 @@ enum {
   DMUON_KERNEL_SYRK = 2,     /* A = X X^T (upper tiles) */
   DMUON_KERNEL_GEMM = 3,     /* X <- 1.5 X - 0.5 A X, last step fused with the update */
   DMUON_KERNEL_APPLY = 4,    /* update for ns_steps == 0 */
-  DMUON_KERNEL_KINDS = 5
+  DMUON_KERNEL_ADAMW = 5,    /* AdamW of the non-orthogonalised parameters */
+  DMUON_KERNEL_KINDS = 6
 };
 
 /* Per-kernel timing: while enabled, every launch is bracketed by CUDA events

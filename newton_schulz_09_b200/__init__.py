@@ -23,10 +23,11 @@ __all__ = [
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
     "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
+    "dmuon_adamw_step_batched", "DmuonTensorDesc",
 ]
 
 #: Kernel kinds of dmuon_stage_times(), in order.
-KERNEL_KINDS = ("prologue", "finalize", "syrk", "gemm", "apply")
+KERNEL_KINDS = ("prologue", "finalize", "syrk", "gemm", "apply", "adamw")
 
 DMUON_F32 = 0
 DMUON_BF16 = 1
@@ -51,6 +52,11 @@ class DmuonShape(ctypes.Structure):
 
 DMUON_LR_PLAIN = 0
 DMUON_LR_SQRT_MAX = 1
+
+
+class DmuonTensorDesc(ctypes.Structure):
+    _fields_ = [("numel", ctypes.c_int64), ("param_dtype", ctypes.c_int32),
+                ("grad_dtype", ctypes.c_int32)]
 
 
 class DmuonStepOptions(ctypes.Structure):
@@ -97,6 +103,8 @@ def load_library() -> ctypes.CDLL:
         "dmuon_launch_count": (ctypes.c_int64, []),
         "dmuon_ns_orthogonalize_noalloc": (i32, [vp, i64, i64, i32, vp]),
         "dmuon_step_options_default": (None, [ctypes.POINTER(DmuonStepOptions)]),
+        "dmuon_adamw_step_batched": (i32, [pp, pp, pp, pp, ctypes.POINTER(DmuonTensorDesc), i32,
+                                           f32, f32, f32, f32, f32, i64, vp]),
         "dmuon_muon_step_batched_opts": (i32, [pp, pp, pp, sp, i32, ctypes.POINTER(DmuonStepOptions),
                                                vp, sz, vp]),
     }
@@ -348,3 +356,44 @@ def dmuon_ns_orthogonalize_noalloc(X: torch.Tensor, steps: int = 5) -> torch.Ten
                                                   _stream(X.device)))
     return X
 
+
+
+def dmuon_adamw_step_batched(params, grads, exp_avgs, exp_avg_sqs, lr: float = 1e-3,
+                             betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.01,
+                             step: int = 1) -> None:
+    """AdamW of the tensors the Muon path does not orthogonalise (any shape,
+    contiguous; bf16 or fp32 parameters and gradients, fp32 states), one
+    launch for all of them.  ``step`` counts this step (>= 1).  A None
+    gradient skips its tensor."""
+    lib = load_library()
+    n = len(params)
+    if not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == n):
+        raise ValueError("params, grads, exp_avgs and exp_avg_sqs must have the same length")
+    if n == 0:
+        return
+    P = (ctypes.c_void_p * n)()
+    G = (ctypes.c_void_p * n)()
+    M = (ctypes.c_void_p * n)()
+    V = (ctypes.c_void_p * n)()
+    D = (DmuonTensorDesc * n)()
+    dev = None
+    for i, (p, g, m, v) in enumerate(zip(params, grads, exp_avgs, exp_avg_sqs)):
+        for t, what in ((p, "params"), (m, "exp_avgs"), (v, "exp_avg_sqs")) + (((g, "grads"),) if g is not None else ()):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{what}[{i}] must be a contiguous CUDA tensor")
+            if t.numel() != p.numel():
+                raise ValueError(f"{what}[{i}] must have the parameter's number of elements")
+            dev = dev or t.device
+            if t.device != dev:
+                raise ValueError("all tensors must be on one device")
+        if m.dtype != torch.float32 or v.dtype != torch.float32:
+            raise ValueError(f"exp_avgs[{i}] and exp_avg_sqs[{i}] must be fp32")
+        P[i], M[i], V[i] = p.data_ptr(), m.data_ptr(), v.data_ptr()
+        G[i] = g.data_ptr() if g is not None else None
+        D[i] = DmuonTensorDesc(p.numel(), _dtype_code(p.dtype),
+                               _dtype_code(g.dtype) if g is not None else _dtype_code(p.dtype))
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    with torch.cuda.device(dev):
+        _check(lib.dmuon_adamw_step_batched(ctypes.cast(P, pp), ctypes.cast(G, pp), ctypes.cast(M, pp),
+                                            ctypes.cast(V, pp), D, n, lr, betas[0], betas[1], eps,
+                                            weight_decay, step, _stream(dev)))

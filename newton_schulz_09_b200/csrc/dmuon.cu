@@ -924,6 +924,80 @@ void dmuon_release_cache(void) {
   g_arenas.clear();
 }
 
+int dmuon_adamw_step_batched(void* const params[], const void* const grads[], float* const exp_avgs[],
+                             float* const exp_avg_sqs[], const dmuon_tensor_desc descs[], int count,
+                             float lr, float beta1, float beta2, float eps, float weight_decay,
+                             int64_t step, dmuon_stream_t stream) {
+  t_last_error.clear();
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count must be >= 0");
+  if (count == 0) return DMUON_OK;
+  if (!params || !grads || !exp_avgs || !exp_avg_sqs || !descs)
+    return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  if (!std::isfinite(lr) || !std::isfinite(weight_decay) || !(beta1 >= 0.0f && beta1 < 1.0f) ||
+      !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps > 0.0f) || !std::isfinite(eps))
+    return fail(DMUON_ERR_INVALID_ARG, "need finite lr and weight_decay, betas in [0, 1), eps > 0");
+  if (step < 1) return fail(DMUON_ERR_INVALID_ARG, "step must be >= 1");
+  std::vector<AdamTensor> ts;
+  ts.reserve(count);
+  for (int i = 0; i < count; ++i) {
+    if (grads[i] == nullptr) continue;
+    const dmuon_tensor_desc& d = descs[i];
+    if (d.numel < 1) return fail(DMUON_ERR_INVALID_ARG, "tensor %d: numel must be >= 1", i);
+    if ((d.param_dtype != DMUON_BF16 && d.param_dtype != DMUON_F32) ||
+        (d.grad_dtype != DMUON_BF16 && d.grad_dtype != DMUON_F32))
+      return fail(DMUON_ERR_UNSUPPORTED, "tensor %d: dtype must be DMUON_BF16 or DMUON_F32", i);
+    if (!params[i] || !exp_avgs[i] || !exp_avg_sqs[i])
+      return fail(DMUON_ERR_INVALID_ARG, "tensor %d: NULL pointer", i);
+    if (!aligned(params[i], elem_bytes(d.param_dtype)) || !aligned(grads[i], elem_bytes(d.grad_dtype)) ||
+        !aligned(exp_avgs[i], 4) || !aligned(exp_avg_sqs[i], 4))
+      return fail(DMUON_ERR_INVALID_ARG, "tensor %d: pointer not aligned to its element size", i);
+    AdamTensor t;
+    t.p = params[i];
+    t.g = grads[i];
+    t.m = exp_avgs[i];
+    t.v = exp_avg_sqs[i];
+    t.numel = d.numel;
+    t.item0 = 0;
+    t.p_bf16 = d.param_dtype == DMUON_BF16;
+    t.g_bf16 = d.grad_dtype == DMUON_BF16;
+    ts.push_back(t);
+  }
+  if (ts.empty()) return DMUON_OK;
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  int r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const double bc1 = 1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step));
+  const double bc2 = 1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step));
+  std::unique_ptr<AdamParams> ap(new AdamParams());
+  ap->b1 = beta1;
+  ap->b2 = beta2;
+  ap->c1 = 1.0f - beta1;
+  ap->c2 = 1.0f - beta2;
+  ap->eps = eps;
+  ap->decay = 1.0f - lr * weight_decay;
+  ap->step_size = static_cast<float>(static_cast<double>(lr) / bc1);
+  ap->inv_bc2_sqrt = static_cast<float>(1.0 / std::sqrt(bc2));
+  for (size_t first = 0; first < ts.size(); first += kAdamMaxTensors) {
+    const int n = static_cast<int>(std::min<size_t>(kAdamMaxTensors, ts.size() - first));
+    int64_t items = 0;
+    for (int k = 0; k < n; ++k) {
+      ap->t[k] = ts[first + k];
+      ap->t[k].item0 = items;
+      items += cdiv(ap->t[k].numel, kAdamChunk);
+    }
+    ap->count = n;
+    ap->nitems = items;
+    const int grid = static_cast<int>(std::min<int64_t>(items, static_cast<int64_t>(g_dev[dev].sms) * 8));
+    LaunchScope ls(st, DMUON_KERNEL_ADAMW);
+    adamw_kernel<<<grid, kPThreads, 0, st>>>(*ap);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return DMUON_OK;
+}
+
 int dmuon_stage_timing(int enable) {
   std::lock_guard<std::mutex> lk(g_api_mu);
   g_timing = enable != 0;

@@ -1011,6 +1011,96 @@ __global__ void __launch_bounds__(kPThreads) apply_kernel(const __grid_constant_
   }
 }
 
+// ======================================================================
+// AdamW for the parameters that are not orthogonalised (the training
+// guide's second group: biases, norms, embeddings, heads), all tensors of a
+// call in one launch.  Per element, with c1 = fl32(1 - beta1),
+// c2 = fl32(1 - beta2):
+//   m <- fl(fl(beta1 m) + fl(c1 g))
+//   v <- fl(fl(beta2 v) + fl(fl(c2 g) g))
+//   p <- p (1 - lr wd) - (lr / bc1) m / (sqrt(v) / sqrt(bc2) + eps)
+// with bc1 = 1 - beta1^t, bc2 = 1 - beta2^t (fp32 arithmetic for p).
+// ======================================================================
+constexpr int kAdamMaxTensors = 512;
+constexpr int kAdamChunk = 8192;            // elements per work item (256 threads x 4 x 8)
+
+struct AdamTensor {
+  void* p;
+  const void* g;
+  float* m;
+  float* v;
+  int64_t numel;
+  int64_t item0;     // first work item of this tensor
+  int32_t p_bf16, g_bf16;
+};
+
+struct AdamParams {
+  AdamTensor t[kAdamMaxTensors];
+  int count;
+  int64_t nitems;
+  float b1, b2, c1, c2, eps, decay, step_size, inv_bc2_sqrt;
+};
+
+__device__ __forceinline__ void load8_any(const void* base, bool bf16, int64_t idx, bool vec, int valid,
+                                          float (&x)[8]) {
+  if (bf16) {
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(base) + idx;
+    if (vec) {
+      const uint4 u = *reinterpret_cast<const uint4*>(src);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+        x[2 * j] = f.x;
+        x[2 * j + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = (e < valid) ? __bfloat162float(src[e]) : 0.0f;
+    }
+  } else {
+    load8_f32(reinterpret_cast<const float*>(base) + idx, vec, valid, x);
+  }
+}
+
+__global__ void __launch_bounds__(kPThreads) adamw_kernel(const __grid_constant__ AdamParams p) {
+  for (int64_t it = blockIdx.x; it < p.nitems; it += gridDim.x) {
+    int lo = 0, hi = p.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.t[mid].item0 <= it) lo = mid; else hi = mid - 1;
+    }
+    const AdamTensor& T = p.t[lo];
+    const int64_t base = (it - T.item0) * kAdamChunk;
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + threadIdx.x) * 8;
+      if (e >= T.numel) break;
+      const int valid = static_cast<int>(T.numel - e < 8 ? T.numel - e : 8);
+      const bool vp = valid == 8 && ((reinterpret_cast<uintptr_t>(T.p) & 15) == 0);
+      const bool vg = valid == 8 && ((reinterpret_cast<uintptr_t>(T.g) & 15) == 0);
+      const bool vs = valid == 8 && ((reinterpret_cast<uintptr_t>(T.m) & 15) == 0) &&
+                      ((reinterpret_cast<uintptr_t>(T.v) & 15) == 0);
+      float g[8], m[8], v[8], w[8];
+      load8_any(T.g, T.g_bf16, e, vg, valid, g);
+      load8_f32(T.m + e, vs, valid, m);
+      load8_f32(T.v + e, vs, valid, v);
+      load8_any(T.p, T.p_bf16, e, vp, valid, w);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        m[k] = __fadd_rn(__fmul_rn(p.b1, m[k]), __fmul_rn(p.c1, g[k]));
+        v[k] = __fadd_rn(__fmul_rn(p.b2, v[k]), __fmul_rn(__fmul_rn(p.c2, g[k]), g[k]));
+        const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v[k]), p.inv_bc2_sqrt), p.eps);
+        w[k] = __fsub_rn(__fmul_rn(w[k], p.decay), __fmul_rn(p.step_size, __fdiv_rn(m[k], denom)));
+      }
+      store8_f32(T.m + e, vs, valid, m);
+      store8_f32(T.v + e, vs, valid, v);
+      if (T.p_bf16) store8_x<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(T.p) + e, vp, valid, w);
+      else store8_f32(reinterpret_cast<float*>(T.p) + e, vp, valid, w);
+    }
+  }
+}
+
 // Test kernel: waits on a barrier that nothing arrives at; the bounded wait
 // gives up after `limit_ns` and records kErrTimeout.
 __global__ void wait_timeout_kernel(int* err, uint64_t limit_ns) {

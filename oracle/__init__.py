@@ -8,6 +8,7 @@ from .muon_oracle import (  # noqa: F401
     NORM_EPS,
     NS_A,
     NS_B,
+    adamw_step,
     clip_coefficient,
     frobenius_normalize,
     lr_scale_factor,

@@ -195,3 +195,31 @@ def ns_flops(rows: int, cols: int, steps: int) -> float:
     symmetric product X X^T and 2 m^2 n for (X X^T) X, m = min, n = max."""
     m, n = min(rows, cols), max(rows, cols)
     return float(steps) * 3.0 * m * m * n
+
+
+def adamw_step(p, g, m, v, *, lr: float, beta1: float, beta2: float, eps: float,
+               weight_decay: float, step: int):
+    """AdamW of one tensor (training guide, "第 4 步：创建优化器": the second
+    parameter group of dmuon.Muon, with adamw_lr / adamw_betas / adamw_eps /
+    adamw_weight_decay; decoupled weight decay, bias-corrected moments).
+
+    The moments follow an exact float32 sequence, c1 = fl32(1 - beta1),
+    c2 = fl32(1 - beta2):  m' = fl(fl(beta1 m) + fl(c1 g)),
+    v' = fl(fl(beta2 v) + fl(fl(c2 g) g)).  The parameter is computed in fp64:
+    p' = p (1 - lr wd) - (lr / bc1) m' / (sqrt(v') / sqrt(bc2) + eps),
+    bc1 = 1 - beta1^step, bc2 = 1 - beta2^step.  Returns (m', v', p')."""
+    f32 = np.float32
+    g32 = np.asarray(g, dtype=np.float32)
+    b1, b2 = f32(beta1), f32(beta2)
+    c1, c2 = f32(f32(1.0) - b1), f32(f32(1.0) - b2)
+    m_new = np.add(np.multiply(np.asarray(m, np.float32), b1, dtype=np.float32),
+                   np.multiply(g32, c1, dtype=np.float32), dtype=np.float32)
+    v_new = np.add(np.multiply(np.asarray(v, np.float32), b2, dtype=np.float32),
+                   np.multiply(np.multiply(g32, c2, dtype=np.float32), g32, dtype=np.float32),
+                   dtype=np.float32)
+    bc1 = 1.0 - float(b1) ** step
+    bc2 = 1.0 - float(b2) ** step
+    lr64, wd64, eps64 = float(f32(lr)), float(f32(weight_decay)), float(f32(eps))
+    denom = np.sqrt(v_new.astype(np.float64)) / np.sqrt(bc2) + eps64
+    p_new = np.asarray(p, np.float64) * (1.0 - lr64 * wd64) - (lr64 / bc1) * m_new.astype(np.float64) / denom
+    return m_new, v_new, p_new

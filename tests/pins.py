@@ -334,7 +334,55 @@ def pin_gradient_clipping(o) -> None:
             assert buf_new[i, j] == want, (i, j)
 
 
+def pin_adamw(o, seed: int = 20) -> None:
+    """AdamW (decoupled decay, bias-corrected moments):
+    * first step from zero moments moves each element by lr g / (|g| + eps)
+      (the bias corrections cancel 1 - beta exactly), i.e. lr sign(g) far
+      above eps and lr / 2 at |g| = eps;
+    * a constant gradient keeps that step size at every later step;
+    * a zero gradient leaves the moments at zero and only decays p;
+    * the moments follow fl(fl(beta m) + fl((1 - beta) g)) exactly."""
+    rng = np.random.default_rng(seed)
+    lr, b1, b2, wd = 1e-3, 0.9, 0.999, 0.0
+    eps = 1e-8
+    g = np.array([3.0, -0.25, 1e-8, -1e-8, 7e-3], dtype=np.float32)
+    p0 = rng.standard_normal(5).astype(np.float32)
+    m = np.zeros(5, np.float32)
+    v = np.zeros(5, np.float32)
+    p = p0.astype(np.float64)
+    for t in range(1, 4):
+        m, v, p = o.adamw_step(p, g, m, v, lr=lr, beta1=b1, beta2=b2, eps=eps, weight_decay=wd, step=t)
+        g64 = g.astype(np.float64)
+        step_want = float(np.float32(lr)) * g64 / (np.abs(g64) + float(np.float32(eps)))
+        moved = p0.astype(np.float64) - p
+        assert np.allclose(moved, t * step_want, rtol=2e-6, atol=0), (t, moved, t * step_want)
+    # zero gradient: moments stay zero, p decays only
+    w = rng.standard_normal(6).astype(np.float32)
+    m1, v1, p1 = o.adamw_step(w, np.zeros(6, np.float32), np.zeros(6, np.float32),
+                              np.zeros(6, np.float32), lr=0.1, beta1=b1, beta2=b2, eps=eps,
+                              weight_decay=0.05, step=4)
+    assert not m1.any() and not v1.any()
+    assert np.array_equal(p1, w.astype(np.float64) * (1.0 - float(np.float32(0.1)) * float(np.float32(0.05))))
+    # exact moment rounding
+    gm = (rng.standard_normal(40) * 10.0 ** rng.integers(-6, 2, 40)).astype(np.float32)
+    mm = (rng.standard_normal(40) * 1e-3).astype(np.float32)
+    vv = (rng.random(40) * 1e-5).astype(np.float32)
+    m2, v2, _ = o.adamw_step(np.zeros(40), gm, mm, vv, lr=lr, beta1=b1, beta2=b2, eps=eps,
+                             weight_decay=0.0, step=2)
+    B1, B2 = Fraction(float(np.float32(b1))), Fraction(float(np.float32(b2)))
+    C1 = exact_f32_round(Fraction(1) - B1)
+    C2 = exact_f32_round(Fraction(1) - B2)
+    for i in range(40):
+        G = Fraction(float(gm[i]))
+        want_m = exact_f32_round(Fraction(float(exact_f32_round(B1 * Fraction(float(mm[i]))))) +
+                                 Fraction(float(exact_f32_round(Fraction(float(C1)) * G))))
+        cg = exact_f32_round(Fraction(float(C2)) * G)
+        want_v = exact_f32_round(Fraction(float(exact_f32_round(B2 * Fraction(float(vv[i]))))) +
+                                 Fraction(float(exact_f32_round(Fraction(float(cg)) * G))))
+        assert m2[i] == want_m and v2[i] == want_v, i
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
-            pin_lr_scale, pin_gradient_clipping)
+            pin_lr_scale, pin_gradient_clipping, pin_adamw)

@@ -138,6 +138,29 @@ def _coeffs_ignored(G, steps, coeffs=(1.5, -0.5)):
     return muon_oracle.newton_schulz(G, steps)
 
 
+def _adamw_variant(kind):
+    def step_fn(p, g, m, v, *, lr, beta1, beta2, eps, weight_decay, step):
+        f32 = np.float32
+        g32 = np.asarray(g, np.float32)
+        if kind == "l2_decay":
+            g32 = (g32 + f32(weight_decay) * np.asarray(p, np.float32)).astype(np.float32)
+        m_new = (f32(beta1) * np.asarray(m, np.float32) + (f32(1) - f32(beta1)) * g32).astype(np.float32)
+        v_new = (f32(beta2) * np.asarray(v, np.float32) + (f32(1) - f32(beta2)) * g32 * g32).astype(np.float32)
+        bc1 = 1.0 - float(f32(beta1)) ** step if kind != "no_bias_correction" else 1.0
+        bc2 = 1.0 - float(f32(beta2)) ** step if kind != "no_bias_correction" else 1.0
+        if kind == "eps_inside_sqrt":
+            denom = np.sqrt(v_new.astype(np.float64) / bc2 + float(f32(eps)))
+        else:
+            denom = np.sqrt(v_new.astype(np.float64)) / np.sqrt(bc2) + float(f32(eps))
+        wd = 0.0 if kind == "l2_decay" else float(f32(weight_decay))
+        p_new = np.asarray(p, np.float64) * (1.0 - float(f32(lr)) * wd) - (float(f32(lr)) / bc1) * m_new / denom
+        return m_new, v_new, p_new
+    return step_fn
+
+
+MUTANTS["adamw_no_bias_correction"] = dict(adamw_step=_adamw_variant("no_bias_correction"))
+MUTANTS["adamw_l2_decay"] = dict(adamw_step=_adamw_variant("l2_decay"))
+MUTANTS["adamw_eps_inside_sqrt"] = dict(adamw_step=_adamw_variant("eps_inside_sqrt"))
 MUTANTS["clip_after_momentum"] = dict(muon_step=_clip_after_momentum)
 MUTANTS["lr_scale_min_side"] = dict(muon_step=_lr_scale_min_side)
 MUTANTS["custom_coefficients_ignored"] = dict(newton_schulz=_coeffs_ignored)
