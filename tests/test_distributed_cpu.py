@@ -1,0 +1,110 @@
+"""Owner-partitioned Muon over data-parallel ranks, on CPU (gloo, 2 ranks).
+
+The per-owner update is the fp64 oracle (injected as the step function), so
+these tests check the partition, the reduction to owners, the owners' batched
+step and the broadcast: the result on every rank must equal one step of the
+oracle on the rank-averaged gradients.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from newton_schulz_09_b200 import distributed as dmd
+from newton_schulz_09_b200 import synthetic
+
+SHAPES = [(48, 96), (96, 48), (64, 64), (32, 128), (24, 40), (128, 32), (16, 16)]
+HP = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.01)
+
+
+def oracle_step_fn(ps, gs, bs, *, lr, momentum, nesterov, weight_decay, ns_steps):
+    for p, g, b in zip(ps, gs, bs):
+        buf_new, X, W_new = oracle.muon_step(p.numpy(), g.numpy(), b.numpy(), lr=lr, momentum=momentum,
+                                             nesterov=nesterov, weight_decay=weight_decay,
+                                             ns_steps=ns_steps)
+        b.copy_(torch.from_numpy(buf_new))
+        p.copy_(torch.from_numpy(W_new.astype(np.float32)))
+
+
+def _params():
+    gen = torch.Generator().manual_seed(5)
+    return [torch.randn(s, generator=gen) * 0.02 for s in SHAPES]
+
+
+def _grads(rank, step):
+    gen = torch.Generator().manual_seed(1000 * step + rank)
+    gs = [torch.randn(s, generator=gen) * 1e-3 for s in SHAPES]
+    gs[4] = None if step == 1 else gs[4]          # no gradient for one matrix on step 1
+    return gs
+
+
+def _worker(rank, world, port, out_dir):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        params = _params()
+        opt = dmd.OwnerPartitionedMuon(params, ns_steps=3, step_fn=oracle_step_fn)
+        for step in range(2):
+            opt.step(_grads(rank, step), **HP)
+        torch.save({"params": [p.clone() for p in params], "owner": opt.owner,
+                    "owned": opt.owned, "bufs": {i: b.clone() for i, b in opt.bufs.items()}},
+                   os.path.join(out_dir, f"rank{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_lpt_partition_is_deterministic_and_balanced():
+    wl = synthetic.workload("llama8b")
+    costs = [dmd.ns_cost(s.rows, s.cols) for s in wl.specs]
+    for world in (2, 4, 8):
+        owner = dmd.lpt_partition(costs, world)
+        assert owner == dmd.lpt_partition(costs, world)
+        assert set(owner) == set(range(world))
+        assert dmd.imbalance(costs, owner, world) < 0.02
+    # one dominant item: it sits alone on its rank
+    owner = dmd.lpt_partition([100.0, 1.0, 1.0, 1.0], 2)
+    assert owner[0] != owner[1] and owner[1] == owner[2] == owner[3]
+    assert dmd.lpt_partition([3.0, 2.0], 1) == [0, 0]
+    with pytest.raises(ValueError):
+        dmd.lpt_partition([1.0], 0)
+
+
+def test_two_ranks_match_one_step_on_averaged_gradients(tmp_path):
+    world = 2
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    res = [torch.load(tmp_path / f"rank{r}.pt") for r in range(world)]
+    # both ranks hold identical weights after the broadcast
+    for a, b in zip(res[0]["params"], res[1]["params"]):
+        assert torch.equal(a, b)
+    # every matrix has exactly one owner, and only owners keep buffers
+    assert sorted(res[0]["owned"] + res[1]["owned"]) == list(range(len(SHAPES)))
+    # reference: two oracle steps on the mean gradient (sum in fp32, then / 2)
+    W = [p.numpy().copy() for p in _params()]
+    bufs = [np.zeros(s, np.float32) for s in SHAPES]
+    for step in range(2):
+        g0, g1 = _grads(0, step), _grads(1, step)
+        for i in range(len(SHAPES)):
+            if g0[i] is None:
+                continue
+            gm = ((g0[i] + g1[i]) / 2).numpy()
+            bufs[i], _, Wn = oracle.muon_step(W[i], gm, bufs[i], ns_steps=3, **HP)
+            W[i] = Wn.astype(np.float32)
+    for i in range(len(SHAPES)):
+        got = res[0]["params"][i].numpy()
+        assert np.array_equal(got, W[i]), i
+        owner = res[0]["owner"][i]
+        assert np.array_equal(res[owner]["bufs"][i].numpy(), bufs[i])

@@ -1,0 +1,44 @@
+"""The owner-partitioned step on the GPU through NCCL with one rank: the
+reduction and broadcast are no-ops, so the result must equal a direct
+batched step bit for bit (needs a B200)."""
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+
+from newton_schulz_09_b200 import distributed as dmd
+
+pytestmark = pytest.mark.gpu
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_single_rank_nccl_matches_direct_step(cuda_lib):
+    dm = cuda_lib
+    dev = torch.device("cuda:0")
+    gen = torch.Generator(device=dev).manual_seed(3)
+    shapes = [(512, 1536), (1536, 512), (256, 256)]
+    pa = [(torch.randn(s, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for s in shapes]
+    pb = [p.clone() for p in pa]
+    grads = [(torch.randn(s, generator=gen, device=dev) * 1e-3).to(torch.bfloat16) for s in shapes]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        opt = dmd.OwnerPartitionedMuon(pa)
+        assert opt.owned == [0, 1, 2]
+        opt.step([g.clone() for g in grads], lr=0.02, weight_decay=0.01)
+        bufs = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+        dm.dmuon_muon_step_batched(pb, grads, bufs, lr=0.02, weight_decay=0.01)
+        torch.cuda.synchronize()
+        for a, b in zip(pa, pb):
+            assert torch.equal(a, b)
+        for i in range(3):
+            assert torch.equal(opt.bufs[i], bufs[i])
+    finally:
+        dist.destroy_process_group()
