@@ -359,31 +359,51 @@ def run_ours(args):
     if not args.no_adamw and wl.name == "llama8b":
         adamw = measure_adamw(dm, dev, stream, world, peaks, args.steps)
 
-    # ---- end to end through the public API: pinned host grads in, weights out
+    # ---- end to end through the public API: pinned host grads in, weights out.
+    # dmuon_muon_step_batched_host uploads each group's gradients, updates it
+    # and downloads its weights, with the copies overlapped with the kernels.
     e2e = None
     if not args.no_e2e:
         pflat, gflat, _ = t.flat
         h_g = torch.empty(gflat.shape, dtype=gflat.dtype, pin_memory=True)
         h_g.copy_(gflat)
         h_w = torch.empty(pflat.shape, dtype=pflat.dtype, pin_memory=True)
+
+        def host_view(flat_h, flat_d, views):
+            out = []
+            for v in views:
+                off = (v.data_ptr() - flat_d.data_ptr()) // v.element_size()
+                out.append(flat_h[off:off + v.numel()].view(v.shape))
+            return out
+
+        hg = host_view(h_g, gflat, t.grads)
+        hw = host_view(h_w, pflat, t.params)
+
+        def host_step():
+            dm.dmuon_muon_step_batched_host(t.params, t.grads, t.bufs, hg, hw, lr=wl.lr,
+                                            momentum=wl.momentum, nesterov=wl.nesterov,
+                                            weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+
+        host_step()                                  # plans and copy streams
         barrier(world)
         torch.cuda.synchronize(dev)
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for _ in range(args.e2e_steps):
-            gflat.copy_(h_g, non_blocking=True)
-            step()
-            h_w.copy_(pflat, non_blocking=True)
+            host_step()
         a1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
+        if not torch.equal(h_w[:4096], pflat[:4096].cpu()):
+            raise RuntimeError("downloaded weights differ from the device weights")
         e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps, world, dev)
         e2e = {"value": fl * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": gflat.numel() * gflat.element_size(),
-               "d2h_bytes_per_step": pflat.numel() * pflat.element_size()}
-        del h_g, h_w
+               "d2h_bytes_per_step": pflat.numel() * pflat.element_size(),
+               "api": "dmuon_muon_step_batched_host (pinned host buffers, copies overlapped)"}
+        del h_g, h_w, hg, hw
 
     status = dm.dmuon_device_status()
     if status != 0:

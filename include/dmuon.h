@@ -25,7 +25,8 @@
  *   - Matrices are dense and row-major: element (r, c) at base[r * cols + c].
  *   - Every pointer argument is a DEVICE pointer owned by the caller, except
  *     the arrays of pointers / shapes themselves, which are HOST arrays read
- *     during the call only.  Updated tensors are written in place.
+ *     during the call only, and the page-locked host buffers named host_* of
+ *     dmuon_muon_step_batched_host.  Updated tensors are written in place.
  *   - Calls are asynchronous: they only enqueue work on `stream` (a
  *     cudaStream_t; NULL is the legacy default stream).  Device pointers must
  *     stay valid until the stream reaches that work.
@@ -161,6 +162,48 @@ void dmuon_step_options_default(dmuon_step_options* opts);
 int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[], float* const bufs[],
                                  const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
                                  void* workspace, size_t ws_bytes, dmuon_stream_t stream);
+
+/*
+ * dmuon_muon_step_batched_host -- the same Muon update (the blog's Vanilla
+ * Muon step, "代码实现" section) for a caller whose gradients arrive in, and
+ * whose updated weights must return to, page-locked host memory.  The
+ * transfers overlap the update: the matrices are cut, in order, into
+ * `chunks` consecutive groups of about equal gradient bytes (chunks <= 0:
+ * one group per ~64 MiB of gradients; at most DMUON_MAX_CHUNKS and at most
+ * one group per matrix).  Every group's gradients are uploaded on a library
+ * copy stream; group c is updated on `stream` as soon as its upload has
+ * landed (while later groups upload) and its weights are downloaded on a
+ * second library copy stream while later groups compute.  The copy schedule
+ * is this library's; the pages have no counterpart of it.  Device results
+ * are bit-identical to dmuon_muon_step_batched_opts on the same tensors.
+ *   params[i]       device W_i, updated in place (the resident weights).
+ *   grads[i]        device staging buffer for g_i (rows x cols, grad_dtype),
+ *                   overwritten with host_grads[i].
+ *   bufs[i]         device fp32 momentum buffer, updated in place.
+ *   host_grads[i]   page-locked host g_i (cudaHostAlloc or cudaHostRegister
+ *                   memory), read only; NULL skips matrix i entirely.
+ *   host_params[i]  page-locked host buffer of W_i's size that receives the
+ *                   updated W_i; NULL: matrix i is not downloaded.
+ *   opts            as for dmuon_muon_step_batched_opts, but max_grad_norm
+ *                   must be 0: a global norm needs every gradient before the
+ *                   first update, which would serialise the uploads.
+ * Ordering: the uploads start after the work enqueued on `stream` before the
+ * call; work enqueued on `stream` after the call starts after the last
+ * download.  The host buffers must not be touched until then.  The two copy
+ * streams are created on a device's first call and kept.  Errors: pageable
+ * host memory or max_grad_norm > 0 -> DMUON_ERR_UNSUPPORTED, chunks >
+ * DMUON_MAX_CHUNKS -> DMUON_ERR_INVALID_ARG, otherwise as
+ * dmuon_muon_step_batched_opts; after an argument or allocation error nothing
+ * is enqueued (a DMUON_ERR_CUDA from a copy or a launch may leave the groups
+ * before it enqueued).  workspace:
+ * NULL (library arena) or ws_bytes >= dmuon_workspace_bytes() of the whole
+ * set (which covers every group).
+ */
+#define DMUON_MAX_CHUNKS 32
+int dmuon_muon_step_batched_host(void* const params[], void* const grads[], float* const bufs[],
+                                 const void* const host_grads[], void* const host_params[],
+                                 const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
+                                 int chunks, void* workspace, size_t ws_bytes, dmuon_stream_t stream);
 
 /*
  * dmuon_adamw_step_batched -- AdamW for the parameters the Muon path does

@@ -23,7 +23,8 @@ __all__ = [
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
     "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
-    "dmuon_adamw_step_batched", "DmuonTensorDesc",
+    "dmuon_adamw_step_batched", "DmuonTensorDesc", "dmuon_muon_step_batched_host",
+    "DMUON_MAX_CHUNKS",
 ]
 
 #: Kernel kinds of dmuon_stage_times(), in order.
@@ -52,6 +53,7 @@ class DmuonShape(ctypes.Structure):
 
 DMUON_LR_PLAIN = 0
 DMUON_LR_SQRT_MAX = 1
+DMUON_MAX_CHUNKS = 32
 
 
 class DmuonTensorDesc(ctypes.Structure):
@@ -107,6 +109,8 @@ def load_library() -> ctypes.CDLL:
                                            f32, f32, f32, f32, f32, i64, vp]),
         "dmuon_muon_step_batched_opts": (i32, [pp, pp, pp, sp, i32, ctypes.POINTER(DmuonStepOptions),
                                                vp, sz, vp]),
+        "dmuon_muon_step_batched_host": (i32, [pp, pp, pp, pp, pp, sp, i32,
+                                               ctypes.POINTER(DmuonStepOptions), i32, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -274,6 +278,58 @@ def dmuon_muon_step_batched_opts(params, grads, bufs, lr: float = 0.02, momentum
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
     with torch.cuda.device(b.device):
         _check(lib.dmuon_muon_step_batched_opts(*b.args(), ctypes.byref(o), ws_ptr, ws_bytes,
+                                                _stream(b.device)))
+
+
+def dmuon_muon_step_batched_host(params, grads, bufs, host_grads, host_params=None,
+                                 lr: float = 0.02, momentum: float = 0.95, nesterov: bool = True,
+                                 weight_decay: float = 0.0, ns_steps: int = 5,
+                                 ns_coefficients=(1.5, -0.5), lr_scale: str = "plain",
+                                 chunks: int = 0, workspace: Optional[torch.Tensor] = None) -> None:
+    """One Muon update whose gradients come from page-locked host tensors
+    (``host_grads``, copied into the device tensors ``grads``) and whose
+    updated weights are copied back into page-locked host tensors
+    (``host_params``, optional), with the copies overlapped with the update in
+    ``chunks`` groups (0: the library picks).  ``params`` and ``bufs`` stay on
+    the device.  Asynchronous on the current stream: synchronise it before
+    reading ``host_params`` or reusing ``host_grads``."""
+    lib = load_library()
+    n = len(params)
+    if len(host_grads) != n or (host_params is not None and len(host_params) != n):
+        raise ValueError("host_grads and host_params must have one entry per parameter")
+    dev_grads = [g if hg is not None else None for g, hg in zip(grads, host_grads)]
+    b = _Batch(params, dev_grads, bufs)
+    if b.n == 0:
+        return
+    HG = (ctypes.c_void_p * n)()
+    HP = (ctypes.c_void_p * n)()
+    for i, (p, g, hg) in enumerate(zip(params, grads, host_grads)):
+        if hg is None:
+            continue
+        hp = host_params[i] if host_params is not None else None
+        for t, what, ref in ((hg, "host_grads", g), (hp, "host_params", p)):
+            if t is None:
+                continue
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+                raise ValueError(f"{what}[{i}] must be a contiguous page-locked (pinned) CPU tensor")
+            if t.dtype != ref.dtype or t.shape != ref.shape:
+                raise ValueError(f"{what}[{i}] must match the device tensor's dtype and shape")
+        HG[i] = hg.data_ptr()
+        HP[i] = hp.data_ptr() if hp is not None else None
+    o = DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
+    o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
+    o.ns_a, o.ns_b = ns_coefficients
+    o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    P, G, B, S, cnt = b.args()
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    with torch.cuda.device(b.device):
+        _check(lib.dmuon_muon_step_batched_host(P, G, B, ctypes.cast(HG, pp), ctypes.cast(HP, pp), S,
+                                                cnt, ctypes.byref(o), chunks, ws_ptr, ws_bytes,
                                                 _stream(b.device)))
 
 

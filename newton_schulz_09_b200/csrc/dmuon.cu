@@ -254,7 +254,7 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[64];
 std::list<std::unique_ptr<Plan>> g_plans;   // most recently used first
-constexpr size_t kMaxPlans = 16;
+constexpr size_t kMaxPlans = 64;   // > DMUON_MAX_CHUNKS: one host-buffer call never evicts its own plans
 
 struct Arena {
   void* ptr = nullptr;
@@ -756,6 +756,144 @@ StepOpts plain_opts(float lr, float momentum, int nesterov, float wd, int steps)
   return o;
 }
 
+// ------------------------------------------------------------------ host-buffer step
+// Two copy streams (upload, download) and a fixed set of events per device,
+// created on the device's first host-buffer call and kept.  Events are
+// re-recorded by later calls: a stream wait binds to the record that precedes
+// it, so reuse is safe.
+struct CopyLanes {
+  bool ready = false;
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev[2 * DMUON_MAX_CHUNKS + 1] = {};
+};
+CopyLanes g_lanes[64];
+
+int copy_lanes(int dev, CopyLanes** out) {
+  CopyLanes& L = g_lanes[dev];
+  if (!L.ready) {
+    cudaError_t e = cudaStreamCreateWithFlags(&L.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L.down, cudaStreamNonBlocking);
+    for (cudaEvent_t& ev : L.ev)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "copy stream set-up");
+    L.ready = true;
+  }
+  *out = &L;
+  return DMUON_OK;
+}
+
+bool page_locked(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+// Cut [0, n) into at most `chunks` runs of about equal `bytes`; returns the
+// run boundaries (first 0, last n).
+std::vector<int> chunk_bounds(const std::vector<size_t>& bytes, int chunks) {
+  const int n = static_cast<int>(bytes.size());
+  size_t total = 0;
+  for (size_t b : bytes) total += b;
+  std::vector<int> bnd(1, 0);
+  size_t acc = 0;
+  int c = 1;
+  for (int i = 0; i + 1 < n; ++i) {
+    acc += bytes[i];
+    if (c < chunks && static_cast<double>(acc) * chunks >= static_cast<double>(total) * c) {
+      bnd.push_back(i + 1);
+      while (c < chunks && static_cast<double>(acc) * chunks >= static_cast<double>(total) * c) ++c;
+    }
+  }
+  bnd.push_back(n);
+  return bnd;
+}
+
+constexpr size_t kChunkTargetBytes = size_t(64) << 20;
+
+// in[k] are the matrices with a gradient; hg/hp/stage are parallel to in.
+int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
+             const std::vector<void*>& hp, const std::vector<void*>& stage, int chunks, void* ws,
+             size_t ws_bytes, bool own_ws, const StepOpts& o, cudaStream_t st) {
+  if (in.empty()) return DMUON_OK;
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  int r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  const int n = static_cast<int>(in.size());
+  std::vector<size_t> gb(n), pb(n);
+  size_t total = 0;
+  for (int k = 0; k < n; ++k) {
+    const size_t numel = static_cast<size_t>(in[k].rows) * static_cast<size_t>(in[k].cols);
+    gb[k] = numel * elem_bytes(in[k].gdt);
+    pb[k] = numel * elem_bytes(in[k].pdt);
+    total += gb[k];
+  }
+  if (chunks <= 0)
+    chunks = static_cast<int>(std::min<size_t>(DMUON_MAX_CHUNKS,
+                                               std::max<size_t>(1, (total + kChunkTargetBytes - 1) /
+                                                                       kChunkTargetBytes)));
+  chunks = std::min(chunks, n);
+  const std::vector<int> bnd = chunk_bounds(gb, chunks);
+  const int nc = static_cast<int>(bnd.size()) - 1;
+  std::vector<std::vector<MatIn>> sub(nc);
+  size_t need = 0;
+  for (int c = 0; c < nc; ++c) {
+    sub[c].assign(in.begin() + bnd[c], in.begin() + bnd[c + 1]);
+    need = std::max(need, make_layout(sub[c], o.steps).bytes);
+  }
+  if (own_ws) {
+    r = arena_get(dev, st, need, &ws);
+    if (r != DMUON_OK) return r;
+  } else {
+    if (!ws) return fail(DMUON_ERR_INVALID_ARG, "NULL workspace");
+    if (ws_bytes < need)
+      return fail(DMUON_ERR_NO_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed",
+                  ws_bytes, need);
+    if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  // Every group's plan before anything is enqueued.  The cache holds more
+  // plans than DMUON_MAX_CHUNKS, so none of these is evicted by the others.
+  std::vector<Plan*> plans(nc, nullptr);
+  for (int c = 0; c < nc; ++c) {
+    r = get_plan(sub[c], o.steps, ws, dev, &plans[c]);
+    if (r != DMUON_OK) return r;
+  }
+  CopyLanes* L = nullptr;
+  r = copy_lanes(dev, &L);
+  if (r != DMUON_OK) return r;
+
+  cudaEvent_t start = L->ev[2 * DMUON_MAX_CHUNKS];
+  cudaError_t e = cudaEventRecord(start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(L->up, start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(L->down, start, 0);
+  // All uploads back to back on one copy engine, one event per group.
+  for (int c = 0; c < nc && e == cudaSuccess; ++c) {
+    for (int k = bnd[c]; k < bnd[c + 1] && e == cudaSuccess; ++k)
+      e = cudaMemcpyAsync(stage[k], hg[k], gb[k], cudaMemcpyHostToDevice, L->up);
+    if (e == cudaSuccess) e = cudaEventRecord(L->ev[c], L->up);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "upload");
+  for (int c = 0; c < nc; ++c) {
+    e = cudaStreamWaitEvent(st, L->ev[c], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    r = launch_plan(*plans[c], o, st);
+    if (r != DMUON_OK) return r;
+    e = cudaEventRecord(L->ev[DMUON_MAX_CHUNKS + c], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->down, L->ev[DMUON_MAX_CHUNKS + c], 0);
+    for (int k = bnd[c]; k < bnd[c + 1] && e == cudaSuccess; ++k)
+      if (hp[k]) e = cudaMemcpyAsync(hp[k], in[k].W, pb[k], cudaMemcpyDeviceToHost, L->down);
+    if (e != cudaSuccess) return cuda_fail(e, "download");
+  }
+  // `stream` continues after the last download.
+  e = cudaEventRecord(start, L->down);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, start, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "download completion");
+  return DMUON_OK;
+}
+
 }  // namespace
 }  // namespace dmuon
 
@@ -827,6 +965,55 @@ int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[]
   r = gather(params, grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
   if (r != DMUON_OK) return r;
   return run(in, workspace, ws_bytes, workspace == nullptr, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dmuon_muon_step_batched_host(void* const params[], void* const grads[], float* const bufs[],
+                                 const void* const host_grads[], void* const host_params[],
+                                 const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
+                                 int chunks, void* workspace, size_t ws_bytes, dmuon_stream_t stream) {
+  t_last_error.clear();
+  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
+  if (opts->struct_size != sizeof(dmuon_step_options))
+    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
+                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
+  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
+  o.ca = opts->ns_a;
+  o.cb = opts->ns_b;
+  o.lr_scale = opts->lr_scale;
+  int r = check_opts(o);
+  if (r != DMUON_OK) return r;
+  if (opts->max_grad_norm != 0.0f)
+    return fail(DMUON_ERR_UNSUPPORTED, "gradient clipping needs every gradient before the first "
+                "update; use dmuon_muon_step_batched_opts");
+  if (chunks > DMUON_MAX_CHUNKS)
+    return fail(DMUON_ERR_INVALID_ARG, "chunks must be <= %d", DMUON_MAX_CHUNKS);
+  if (count > 0 && (!host_grads || !host_params || !grads))
+    return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  std::vector<MatIn> in;
+  // Checked as given, then the device staging buffers stand for the
+  // gradients in the update.
+  r = gather(params, host_grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
+  if (r != DMUON_OK) return r;
+  std::vector<const void*> hg;
+  std::vector<void*> hp, stage;
+  for (int i = 0; i < count; ++i) {
+    if (!host_grads[i]) continue;
+    if (!grads[i]) return fail(DMUON_ERR_INVALID_ARG, "matrix %d: NULL device gradient buffer", i);
+    if (!page_locked(host_grads[i]))
+      return fail(DMUON_ERR_UNSUPPORTED, "matrix %d: host gradient is not page-locked memory", i);
+    if (host_params[i] && !page_locked(host_params[i]))
+      return fail(DMUON_ERR_UNSUPPORTED, "matrix %d: host parameter buffer is not page-locked memory", i);
+    const size_t eb = elem_bytes(shapes[i].grad_dtype);
+    if (!aligned(grads[i], eb))
+      return fail(DMUON_ERR_INVALID_ARG, "matrix %d: device gradient buffer misaligned", i);
+    MatIn& x = in[hg.size()];
+    x.G = grads[i];
+    hg.push_back(host_grads[i]);
+    hp.push_back(host_params[i]);
+    stage.push_back(grads[i]);
+  }
+  return run_host(in, hg, hp, stage, chunks, workspace, ws_bytes, workspace == nullptr, o,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps) {

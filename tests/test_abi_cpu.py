@@ -134,3 +134,25 @@ def test_no_cpu_fallback_without_device():
         pytest.skip("a GPU is present")
     with pytest.raises(ValueError):
         dm.dmuon_ns_orthogonalize(torch.zeros(4, 4, dtype=torch.bfloat16))
+
+
+def test_host_buffer_step_rejects_bad_arguments_on_the_host(lib):
+    o = dm.DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    P, G, B = _ptrs(0x10000), _ptrs(0x20000), _ptrs(0x30000)
+    HG, HP = _ptrs(0x40000), _ptrs(0x50000)
+    S = _shapes((4, 4))
+    call = lambda opts, chunks=0, hg=HG, n=1: lib.dmuon_muon_step_batched_host(
+        P, G, B, hg, HP, S, n, opts, chunks, None, 0, None)
+    assert call(ctypes.byref(o), n=0) == 0
+    assert call(None) == -1
+    assert call(ctypes.byref(o), chunks=dm.DMUON_MAX_CHUNKS + 1) == -1
+    clip = dm.DmuonStepOptions(); lib.dmuon_step_options_default(ctypes.byref(clip))
+    clip.max_grad_norm = 1.0
+    assert call(ctypes.byref(clip)) == -2
+    assert "clipping" in dm.dmuon_last_error()
+    # no host gradient at all: nothing to do, no CUDA call
+    assert call(ctypes.byref(o), hg=_ptrs(None)) == 0
+    # pointers that are not page-locked host memory are refused
+    assert call(ctypes.byref(o)) == -2
+    assert "page-locked" in dm.dmuon_last_error()
