@@ -37,8 +37,8 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage per full
 # Llama-8B launch: the one-layer ncu capture (--workload llama8b_layer) scaled by 32 identical
 # layers; valid only for the kernel source it was measured on.
-PROFILED_TRAFFIC = {"kernels_sha256_prefix": "da9e8cb50425422a", "workload": "llama8b",
-                    "gemm_bytes_per_launch": 32 * 1.282e9}
+PROFILED_TRAFFIC = {"kernels_sha256_prefix": "a5feef2896f3af76", "workload": "llama8b",
+                    "gemm_bytes_per_launch": 32 * 1.2086e9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
