@@ -149,6 +149,10 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def min_over_ranks(x: float, world: int, device) -> float:
+    return -max_over_ranks(-x, world, device)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -363,7 +367,20 @@ def run_ours(args):
     # dmuon_muon_step_batched_host uploads each group's gradients, updates it
     # and downloads its weights, with the copies overlapped with the kernels.
     e2e = None
-    if not args.no_e2e:
+    e2e_ok = not args.no_e2e
+    if e2e_ok:
+        # Every rank of this node pins its own gradient and weight copies; skip
+        # the leg (on every rank alike) when the host cannot hold them all.
+        import psutil
+        pflat, gflat, _ = t.flat
+        pin_bytes = pflat.numel() * pflat.element_size() + gflat.numel() * gflat.element_size()
+        local_ranks = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+        fits = psutil.virtual_memory().available > 1.3 * pin_bytes * local_ranks
+        if min_over_ranks(1.0 if fits else 0.0, world, dev) < 1.0:
+            e2e_ok = False
+            e2e = {"value": None, "skipped": f"host memory: {local_ranks} ranks x {pin_bytes / 1e9:.0f} GB "
+                                             f"pinned exceeds the available RAM"}
+    if e2e_ok:
         pflat, gflat, _ = t.flat
         h_g = torch.empty(gflat.shape, dtype=gflat.dtype, pin_memory=True)
         h_g.copy_(gflat)
