@@ -297,6 +297,12 @@ int device_setup(int dev) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
   }
+  const void* pk[] = {reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16>),
+                      reinterpret_cast<const void*>(&prologue_kernel<float>)};
+  for (const void* k : pk) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kProSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prologue smem)");
+  }
   if (!encode_fn()) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   d.ready = true;
   return DMUON_OK;
@@ -578,7 +584,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-    prologue_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+    prologue_kernel<E><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
@@ -1377,7 +1383,7 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   ep.clip = nullptr;
   ep.gpartials = nullptr;
   const int pgrid = static_cast<int>(std::min<int64_t>(ml.ptiles, static_cast<int64_t>(di.sms) * 8));
-  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, 0, st>>>(ep);
+  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
   finalize_kernel<<<1, 32, 0, st>>>(ep);
   g_launches += 2;
   if (steps == 0) {

@@ -647,6 +647,53 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 // ======================================================================
 constexpr int kFlatChunk = 8192;       // elements per flat item (256 threads x 4 x 8)
 constexpr int kTR = 64, kTC = 128;     // transposed item: 64 parameter rows x 128 columns
+// Dynamic shared memory of the prologue: the staged gradient (room for fp32)
+// and momentum of one item; a transposed item reuses it as its 64 x 129
+// fp32 transpose tile once every thread has read its staged inputs.
+constexpr int kProStageG = kFlatChunk * 4;
+constexpr int kProSmemBytes = kFlatChunk * 8;
+static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes, "transpose tile must fit the staging area");
+
+// Stage 8 consecutive input elements (one thread's segment) into shared
+// memory with 16-byte asynchronous copies: the gradient at sg (2 or 4 bytes
+// an element), the momentum at sb.  Only whole, 16-byte aligned segments.
+__device__ __forceinline__ void stage8(const MatDesc& md, int64_t idx, bool has_buf, uint8_t* sg, float* sb) {
+  if (md.g_bf16) {
+    cp_async16(sg, reinterpret_cast<const __nv_bfloat16*>(md.G) + idx);
+  } else {
+    const float* g = reinterpret_cast<const float*>(md.G) + idx;
+    cp_async16(sg, g);
+    cp_async16(sg + 16, g + 4);
+  }
+  if (has_buf) {
+    cp_async16(sb, md.buf + idx);
+    cp_async16(sb + 4, md.buf + idx + 4);
+  }
+}
+__device__ __forceinline__ void unstage8(const MatDesc& md, bool has_buf, const uint8_t* sg, const float* sb,
+                                         float (&g)[8], float (&b)[8]) {
+  if (md.g_bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(sg);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      g[2 * j] = f.x;
+      g[2 * j + 1] = f.y;
+    }
+  } else {
+    const float4 x = *reinterpret_cast<const float4*>(sg);
+    const float4 y = *reinterpret_cast<const float4*>(sg + 16);
+    g[0] = x.x; g[1] = x.y; g[2] = x.z; g[3] = x.w;
+    g[4] = y.x; g[5] = y.y; g[6] = y.z; g[7] = y.w;
+  }
+  if (has_buf) {
+    const float4 x = *reinterpret_cast<const float4*>(sb);
+    const float4 y = *reinterpret_cast<const float4*>(sb + 4);
+    b[0] = x.x; b[1] = x.y; b[2] = x.z; b[3] = x.w;
+    b[4] = y.x; b[5] = y.y; b[6] = y.z; b[7] = y.w;
+  }
+}
 
 // 8 consecutive input elements (bf16 or fp32), 16-byte aligned when vec.
 __device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool vec, int valid, float (&g)[8]) {
@@ -743,7 +790,8 @@ __device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, flo
 }
 
 template <typename E>
-__device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDesc& md, int64_t item) {
+__device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDesc& md, int64_t item,
+                                               uint8_t* stage) {
   const int tid = threadIdx.x;
   const int64_t numel = md.rows * md.cols;
   const int64_t e_begin = item * kFlatChunk;
@@ -751,18 +799,35 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
   const bool flat_x = (md.ldx == md.cols);
   E* X = reinterpret_cast<E*>(md.X[0]);
   E* Xo = reinterpret_cast<E*>(md.Xop[0]);
+  const int gb = md.g_bf16 ? 2 : 4;
+  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
+  // Four rounds of 8 consecutive elements per thread.  The whole, aligned
+  // segments of all four rounds are staged into shared memory first, so
+  // 4 x (8 g + 8 buf) elements per thread are in flight at once; each thread
+  // reads back only what it staged itself.
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int le = (j * kPThreads + tid) * 8;
+    const int64_t e = e_begin + le;
+    if (md.vec4 && e + 8 <= numel) stage8(md, e, has_buf, stage + le * gb, sbuf + le);
+  }
+  cp_async_commit();
+  cp_async_wait_all();
   float ss = 0.0f;
-  // Four rounds of 8 consecutive elements per thread; latency is hidden by
-  // occupancy (few registers per thread).
 #pragma unroll 1
   for (int j = 0; j < 4; ++j) {
-    const int64_t e = e_begin + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+    const int le = (j * kPThreads + tid) * 8;
+    const int64_t e = e_begin + le;
     if (e >= numel) break;
     const int valid = static_cast<int>(numel - e < 8 ? numel - e : 8);
     const bool vec = md.vec4 && valid == 8;
     float g[8], b[8], M[8];
-    load8_in(md, e, vec, valid, g);
-    if (has_buf) load8_f32(md.buf + e, vec, valid, b);
+    if (vec) {
+      unstage8(md, has_buf, stage + le * gb, sbuf + le, g, b);
+    } else {
+      load8_in(md, e, vec, valid, g);
+      if (has_buf) load8_f32(md.buf + e, vec, valid, b);
+    }
     momentum8(p, has_buf, g, b, M);
     if (has_buf) store8_f32(md.buf + e, vec, valid, b);
 #pragma unroll
@@ -793,7 +858,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
 
 template <typename E>
 __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const MatDesc& md, int64_t item,
-                                                     float (*sM)[kTC + 1]) {
+                                                     uint8_t* stage) {
   const int tid = threadIdx.x;
   const int ty = tid >> 4;      // 0..15: parameter rows ty + 16 i
   const int tx = tid & 15;      // 0..15: 8 consecutive parameter columns
@@ -802,29 +867,52 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   const int64_t rows = md.rows, cols = md.cols;
   const bool has_buf = md.buf != nullptr;
   const int64_t c = c0 + tx * 8;
+  const int gb = md.g_bf16 ? 2 : 4;
+  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
+  // Stage this thread's four row segments (whole, aligned ones) first.
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + ty + 16 * i;
+    const int64_t idx = r * cols + c;
+    const int slot = (i * kPThreads + tid) * 8;
+    if (md.vec4 && r < rows && c + 8 <= cols && (idx & 7) == 0)
+      stage8(md, idx, has_buf, stage + slot * gb, sbuf + slot);
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  float Mv[4][8];
   float ss = 0.0f;
-#pragma unroll 1
+#pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t r = r0 + ty + 16 * i;
     const int valid = (r < rows && c < cols) ? static_cast<int>(cols - c < 8 ? cols - c : 8) : 0;
-    float g[8], b[8], M[8];
+    float g[8], b[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) { g[k] = 0.0f; b[k] = 0.0f; }
     const int64_t idx = r * cols + c;
     const bool vec = md.vec4 && valid == 8 && ((idx & 7) == 0);
-    if (valid > 0) {
+    if (vec) {
+      const int slot = (i * kPThreads + tid) * 8;
+      unstage8(md, has_buf, stage + slot * gb, sbuf + slot, g, b);
+    } else if (valid > 0) {
       load8_in(md, idx, vec, valid, g);
       if (has_buf) load8_f32(md.buf + idx, vec, valid, b);
     }
-    momentum8(p, has_buf, g, b, M);
+    momentum8(p, has_buf, g, b, Mv[i]);
     if (valid > 0 && has_buf) store8_f32(md.buf + idx, vec, valid, b);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      if (k >= valid) M[k] = 0.0f;
-      ss = fmaf(M[k], M[k], ss);
-      sM[ty + 16 * i][tx * 8 + k] = M[k];
+      if (k >= valid) Mv[i][k] = 0.0f;
+      ss = fmaf(Mv[i][k], Mv[i][k], ss);
     }
   }
+  // Every thread has read its staged inputs: the area becomes the transpose tile.
+  __syncthreads();
+  float (*sM)[kTC + 1] = reinterpret_cast<float (*)[kTC + 1]>(stage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sM[ty + 16 * i][tx * 8 + k] = Mv[i][k];
   __syncthreads();
   // X row = parameter column (128 of them), X columns = the 64 parameter rows.
   E* X = reinterpret_cast<E*>(md.X[0]);
@@ -854,14 +942,14 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
 
 template <typename E>
 __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
-  __shared__ float sM[kTR][kTC + 1];
+  extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
     const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
     const MatDesc& md = p.mats[mi];
     const int64_t item = t - __ldg(p.ptile_prefix + mi);
-    float ss = md.T ? prologue_transposed<E>(p, md, item, sM) : prologue_flat<E>(p, md, item);
+    float ss = md.T ? prologue_transposed<E>(p, md, item, pro_stage) : prologue_flat<E>(p, md, item, pro_stage);
     // Fixed-order block reduction of the item's sum of squares.
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
