@@ -186,7 +186,9 @@ __device__ __forceinline__ int find_slot64(const int64_t* prefix, int n, int64_t
 
 // Upper-triangle SYRK tiles of one matrix, enumerated column-band major:
 // column band J (256 wide) holds row bands I = 0 .. 2J+1 (128 tall), so band
-// J starts at J (J + 1).
+// J starts at J (J + 1).  The last tile of a band, I = 2J+1, lies on the
+// diagonal with its left 128 columns wholly below it: that tile is computed
+// as a 128 x 128 half tile (UMMA N = 128) over the band's right 128 columns.
 __device__ __forceinline__ void syrk_tile_coords(int local, int& I, int& J) {
   int j = static_cast<int>((sqrtf(4.0f * static_cast<float>(local) + 1.0f) - 1.0f) * 0.5f);
   while ((j + 1) * (j + 2) <= local) ++j;
@@ -197,6 +199,7 @@ __device__ __forceinline__ void syrk_tile_coords(int local, int& I, int& J) {
 
 struct TileInfo {
   int mi, tm, tn, nkb;
+  int half;   // SYRK: 128 x 128 tile over columns tn * 256 + 128 ..
 };
 
 // Tile t of a launch (128 x 256 tiles).
@@ -207,9 +210,11 @@ __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
   ti.mi = __ldg(p.order + slot);
   const int local = t - __ldg(p.tile_prefix + slot);
   const MatDesc& md = p.mats[ti.mi];
+  ti.half = 0;
   if (kMode == kSyrk) {
     syrk_tile_coords(local, ti.tm, ti.tn);
     ti.nkb = (md.n + BK - 1) / BK;
+    ti.half = (ti.tm == 2 * ti.tn + 1) ? 1 : 0;
   } else {
     const int nI = (md.m + kBM - 1) / kBM;
     ti.tn = local / nI;
@@ -340,13 +345,15 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
       const float alpha = p.first ? s * s : 1.0f;
       E* A = reinterpret_cast<E*>(md.A);
       const int64_t lda = md.lda;
+      const int nch = ti.half ? kBN / 64 : kBN / 32;
+      const int col0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < nch; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait();
-        if (c == kBN / 32 - 1) release(b);
-        const int C0 = ti.tn * kBN + c * 32;
+        if (c == nch - 1) release(b);
+        const int C0 = col0 + c * 32;
         if (R < m && C0 < m && C0 + 31 >= R) {
           float y[32];
 #pragma unroll
@@ -482,6 +489,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   constexpr int KSTEPS = BK / MMA_K;        // = 4
   constexpr uint32_t FMT = (EB == 2) ? 1u : 2u;
   constexpr uint32_t IDESC = make_idesc(FMT, 0u, kMode == kGemm ? 1u : 0u, kBM, kBN);
+  constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);   // SYRK half tiles
   constexpr int NBOX_B = (kMode == kGemm) ? kBN / BK : 2;
   constexpr uint32_t BOX_B_BYTES = (kMode == kGemm) ? BK * 128 : kAStageBytes;
 
@@ -540,8 +548,9 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const CUtensorMap* mapA = (kMode == kSyrk) ? &mp.xk[p.cur] : &mp.a;
       const CUtensorMap* mapB = (kMode == kSyrk) ? &mp.xk[p.cur] : &mp.xmn[p.cur];
       int nb = 0;
+      const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK B operand rows
       if (kMode == kSyrk) {
-        nb = (ti.tn * kBN + 128 < md.m) ? 2 : 1;
+        nb = (ti.half || ti.tn * kBN + 128 >= md.m) ? 1 : 2;
       } else {
         const int left = md.n - ti.tn * kBN;
         nb = (left + BK - 1) / BK;
@@ -558,7 +567,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
           for (int j = 0; j < nb; ++j) {
             if (kMode == kSyrk)
-              tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, ti.tn * kBN + j * 128);
+              tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
             else
               tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);
           }
@@ -587,6 +596,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
+      const uint32_t idesc = (kMode == kSyrk && ti.half) ? IDESC_HALF : IDESC;
       for (int kb = 0; kb < ti.nkb; ++kb) {
         w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
@@ -605,8 +615,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
                     : sw128_desc(b_base + k * MMA_K * 128, BK * 128, EB == 2 ? 1024 : 512,
                                  EB == 2 ? kSwizzle128B : kSwizzle128B32);
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-            if (EB == 2) umma_f16(d_tmem, ad, bd, IDESC, acc);
-            else umma_tf32(d_tmem, ad, bd, IDESC, acc);
+            if (EB == 2) umma_f16(d_tmem, ad, bd, idesc, acc);
+            else umma_tf32(d_tmem, ad, bd, idesc, acc);
           }
           umma_commit(&empty[stage]);
         }
