@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama8b")
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--impl", choices=["ours", "reference", "torch"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -455,10 +455,84 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------- torch eager
+def run_torch(args):
+    """Context arm, not the product: the same step written as plain PyTorch
+    eager code, the per-parameter loop of the blog's Vanilla Muon with the
+    Newton-Schulz products in bf16 through torch.matmul (cuBLAS).  It forms
+    the full X X^T (4 m^2 n FLOPs per step); the rate below still counts the
+    3 m^2 n useful FLOPs, as for the product."""
+    import torch
+    from newton_schulz_09_b200 import synthetic
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    wl = synthetic.workload(args.workload)
+    t = synthetic.make_tensors(wl, device=dev, flat=True, seed_offset=rank)
+    fl = synthetic.ns_flops(wl)
+    mu, lr, wd, k = wl.momentum, wl.lr, wl.weight_decay, wl.ns_steps
+
+    @torch.no_grad()
+    def step():
+        for p, g, buf in zip(t.params, t.grads, t.bufs):
+            buf.mul_(mu).add_(g)
+            M = g.float().add(buf, alpha=mu) if wl.nesterov else buf
+            X = M.to(torch.bfloat16)
+            tall = X.shape[0] > X.shape[1]
+            if tall:
+                X = X.T
+            X = X / (X.norm() + 1e-7)
+            for _ in range(k):
+                A = X @ X.T
+                X = 1.5 * X - 0.5 * (A @ X)
+            if tall:
+                X = X.T
+            p.mul_(1.0 - lr * wd).add_(X.to(p.dtype), alpha=-lr)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if rank == 0:
+        print(json.dumps({
+            "impl": "torch-eager", "metric": METRIC, "value": fl * world / (ms * 1e-3) / 1e12,
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "dtype": "bf16",
+            "data": "synthetic", "clocks": clocks,
+            "config": {"workload": wl.name, "matrices": len(wl.specs), "ns_steps": k,
+                       "note": "per-matrix torch eager loop, NS products by torch.matmul (cuBLAS)"}}))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.impl == "torch":
+        return run_torch(args)
     return run_ours(args)
 
 
