@@ -37,8 +37,11 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage per full
 # Llama-8B launch: the one-layer ncu capture (--workload llama8b_layer) scaled by 32 identical
 # layers; valid only for the kernel source it was measured on.
-PROFILED_TRAFFIC = {"kernels_sha256_prefix": "a5feef2896f3af76", "workload": "llama8b",
-                    "gemm_bytes_per_launch": 32 * 1.2086e9}
+# ncu capture of the GEMM stage on one Llama-8B layer (1.339 GB of DRAM traffic for
+# 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so
+# its traffic is this ratio times the useful FLOPs of that launch.
+PROFILED_TRAFFIC = {"kernels_sha256_prefix": "1d289bbf78e598ca", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 1.339e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -57,7 +60,7 @@ def parse_args():
 
 
 def profiled_traffic(workload: str):
-    """The profiled DRAM bytes per GEMM launch, or None when the kernels changed since."""
+    """The profiled DRAM bytes per useful GEMM FLOP, or None when the kernels changed since."""
     import hashlib
     path = os.path.join(HERE, "newton_schulz_09_b200", "csrc", "kernels.cuh")
     try:
@@ -65,7 +68,7 @@ def profiled_traffic(workload: str):
     except OSError:
         return None
     if sha.startswith(PROFILED_TRAFFIC["kernels_sha256_prefix"]) and workload == PROFILED_TRAFFIC["workload"]:
-        return PROFILED_TRAFFIC["gemm_bytes_per_launch"]
+        return PROFILED_TRAFFIC["gemm_bytes_per_useful_flop"]
     return None
 
 
@@ -340,19 +343,27 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, world, dev)
     value = fl * world / (ms * 1e-3) / 1e12
 
-    # ---- roofline of the dominant kernel (the GEMM stage: 2 m^2 n per step)
+    # ---- roofline of the dominant kernel (the GEMM stage: 2 m^2 n per NS step).
+    # The library runs a large call as groups of matrices, so a step has several
+    # GEMM launches per NS step; rates use the step's totals (= the launches'
+    # FLOP-weighted average), traffic is per average launch.
     gemm_ms, gemm_n = stages["gemm"]
     syrk_ms, syrk_n = stages["syrk"]
-    gemm_fl_per_launch = sum(2.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
-    syrk_fl_per_launch = sum(1.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
+    gemm_fl_step = wl.ns_steps * sum(2.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
+    syrk_fl_step = wl.ns_steps * sum(1.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) for s in wl.specs)
     peak = peaks["bf16_tflops_sustained"]
-    gemm_tf = gemm_fl_per_launch / (gemm_ms / gemm_n * 1e-3) / 1e12 if gemm_n else None
-    syrk_tf = syrk_fl_per_launch / (syrk_ms / syrk_n * 1e-3) / 1e12 if syrk_n else None
+    gemm_tf = gemm_fl_step / (gemm_ms / args.steps * 1e-3) / 1e12 if gemm_n else None
+    syrk_tf = syrk_fl_step / (syrk_ms / args.steps * 1e-3) / 1e12 if syrk_n else None
+    gemm_launches_step = gemm_n / args.steps if gemm_n else None
+    fl_per_launch = gemm_fl_step / gemm_launches_step if gemm_n else None
+    bpf = profiled_traffic(wl.name)
     roofline = {
         "kernel": "ns_stage_kernel<GEMM, bf16>", "bound": "tensor",
         "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
-        "frac": (gemm_tf / peak) if gemm_tf else None, "traffic": profiled_traffic(wl.name),
-        "traffic_unit": "bytes per launch (ncu, one-layer capture x 32)",
+        "frac": (gemm_tf / peak) if gemm_tf else None,
+        "traffic": (bpf * fl_per_launch) if (bpf and fl_per_launch) else None,
+        "traffic_unit": "DRAM bytes per average launch (ncu one-layer capture, scaled by useful FLOPs)",
+        "launches_per_step": gemm_launches_step, "useful_flop_per_launch": fl_per_launch,
         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
         "syrk": {"achieved": syrk_tf, "frac": (syrk_tf / peak) if syrk_tf else None},
         "stage_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},

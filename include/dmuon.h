@@ -99,8 +99,12 @@ size_t dmuon_ns_workspace_bytes(int64_t m, int64_t n, int dtype);
 
 /*
  * dmuon_muon_step_batched -- one Muon update of `count` matrices, with one
- * launch per stage for all of them (the per-parameter loop of the blog's
- * Vanilla Muon, "代码实现" section, done as grouped kernels).
+ * launch per stage for a whole group of them (the per-parameter loop of the
+ * blog's Vanilla Muon, "代码实现" section, done as grouped kernels).  A call
+ * of more than 2^30 elements runs as consecutive groups of at most about
+ * that many (in the order given, at most 32 groups, one after the other on
+ * the stream and sharing one scratch region); the result of each matrix does
+ * not depend on the grouping.  With gradient clipping the call is one group.
  *   params[i]  device pointer to W_i (rows x cols, param_dtype), updated in place.
  *   grads[i]   device pointer to g_i (rows x cols, grad_dtype), read only; NULL
  *              skips matrix i entirely (no momentum, no update), as the blog
@@ -230,9 +234,10 @@ int dmuon_adamw_step_batched(void* const params[], const void* const grads[], fl
                              float lr, float beta1, float beta2, float eps, float weight_decay,
                              int64_t step, dmuon_stream_t stream);
 
-/* Scratch bytes needed by dmuon_muon_step_batched_ex for these shapes
+/* Scratch bytes that suffice for dmuon_muon_step_batched_ex on these shapes
  * (matrices with a NULL gradient may be left out or counted; counting them
- * over-estimates).  Returns 0 for invalid shapes. */
+ * over-estimates): the need of the whole set as one group, which covers any
+ * grouping of it.  Returns 0 for invalid shapes. */
 size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps);
 
 /* Last error message of the calling host thread ("" if none). */

@@ -254,7 +254,7 @@ struct DeviceInfo {
 };
 DeviceInfo g_dev[64];
 std::list<std::unique_ptr<Plan>> g_plans;   // most recently used first
-constexpr size_t kMaxPlans = 64;   // > DMUON_MAX_CHUNKS: one host-buffer call never evicts its own plans
+constexpr size_t kMaxPlans = 64;   // > the groups of one call (<= 32): a call never evicts its own plans
 
 struct Arena {
   void* ptr = nullptr;
@@ -716,6 +716,32 @@ int gather(void* const params[], const void* const grads[], float* const bufs[],
   return DMUON_OK;
 }
 
+// A large call runs as consecutive groups of matrices, one after the other on
+// the stream, sharing one scratch region.  Measured on the Llama-8B stack
+// (224 matrices, 7e9 elements): groups of ~2^30 elements (four layers) run
+// at a higher SM clock under the power cap than one launch per stage over
+// every matrix (413 ms against 440 ms per step); the arithmetic of each
+// matrix does not depend on the grouping.
+constexpr int64_t kGroupElems = int64_t(1) << 30;
+constexpr int kMaxGroups = 32;   // < kMaxPlans: one call never evicts its own plans
+
+// Boundaries of consecutive groups: a matrix joins the current group unless
+// that would take it past `target` elements.
+std::vector<int> group_bounds(const std::vector<MatIn>& in, int64_t target) {
+  std::vector<int> bnd(1, 0);
+  int64_t acc = 0;
+  for (size_t i = 0; i < in.size(); ++i) {
+    const int64_t e = in[i].rows * in[i].cols;
+    if (acc > 0 && acc + e > target) {
+      bnd.push_back(static_cast<int>(i));
+      acc = 0;
+    }
+    acc += e;
+  }
+  bnd.push_back(static_cast<int>(in.size()));
+  return bnd;
+}
+
 int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, const StepOpts& o,
         cudaStream_t st) {
   const int steps = o.steps;
@@ -724,7 +750,27 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
   int dev = 0;
   int r = current_device(&dev);
   if (r != DMUON_OK) return r;
-  const size_t need = make_layout(in, steps).bytes;
+  // Clipping needs one global norm before any momentum update: one group.
+  std::vector<int> bnd;
+  if (o.max_norm > 0.0f) {
+    bnd = {0, static_cast<int>(in.size())};
+  } else {
+    int64_t total = 0;
+    for (const MatIn& x : in) total += x.rows * x.cols;
+    int64_t target = std::max<int64_t>(kGroupElems, (total + kMaxGroups - 1) / kMaxGroups);
+    bnd = group_bounds(in, target);
+    while (static_cast<int>(bnd.size()) - 1 > kMaxGroups) {   // ends: target >= total gives one group
+      target *= 2;
+      bnd = group_bounds(in, target);
+    }
+  }
+  const int ng = static_cast<int>(bnd.size()) - 1;
+  std::vector<std::vector<MatIn>> sub(ng);
+  size_t need = 0;
+  for (int gi = 0; gi < ng; ++gi) {
+    sub[gi].assign(in.begin() + bnd[gi], in.begin() + bnd[gi + 1]);
+    need = std::max(need, make_layout(sub[gi], steps).bytes);
+  }
   if (own_ws) {
     r = arena_get(dev, st, need, &ws);
     if (r != DMUON_OK) return r;
@@ -735,10 +781,17 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
                   ws_bytes, need);
     if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
-  Plan* plan = nullptr;
-  r = get_plan(in, steps, ws, dev, &plan);
-  if (r != DMUON_OK) return r;
-  return launch_plan(*plan, o, st);
+  // Every group's plan before anything is enqueued.
+  std::vector<Plan*> plans(ng, nullptr);
+  for (int gi = 0; gi < ng; ++gi) {
+    r = get_plan(sub[gi], steps, ws, dev, &plans[gi]);
+    if (r != DMUON_OK) return r;
+  }
+  for (int gi = 0; gi < ng; ++gi) {
+    r = launch_plan(*plans[gi], o, st);
+    if (r != DMUON_OK) return r;
+  }
+  return DMUON_OK;
 }
 
 int check_opts(const StepOpts& o) {
