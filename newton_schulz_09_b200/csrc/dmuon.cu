@@ -872,6 +872,37 @@ std::vector<int> chunk_bounds(const std::vector<size_t>& bytes, int chunks) {
 
 constexpr size_t kChunkTargetBytes = size_t(64) << 20;
 
+// Automatic groups of the host-buffer step, by gradient bytes: the first
+// group is small (its upload is exposed), each next one up to 1.5x the one
+// before (an upload must land before the kernels reach it; the copy engines
+// move ~55 GB/s, the update consumes gradients at ~35 GB/s), at most
+// `mid` bytes, and the groups shrink again towards the end (the last
+// group's download is exposed): a group may hold at most a third of the
+// bytes still to come including itself.  At most DMUON_MAX_CHUNKS groups.
+std::vector<int> ramp_bounds(const std::vector<size_t>& bytes) {
+  const int n = static_cast<int>(bytes.size());
+  size_t total = 0;
+  for (size_t b : bytes) total += b;
+  const size_t first = std::max(kChunkTargetBytes, total / 128);
+  const size_t mid = std::max(size_t(2) << 30, total / (DMUON_MAX_CHUNKS / 2));
+  std::vector<int> bnd(1, 0);
+  size_t acc = 0, done = 0;
+  double grow = static_cast<double>(first);
+  for (int i = 0; i + 1 < n; ++i) {
+    acc += bytes[i];
+    double target = std::min(static_cast<double>(mid), grow);
+    target = std::min(target, std::max(static_cast<double>(first), static_cast<double>(total - done) / 3.0));
+    if (static_cast<double>(acc) >= target && static_cast<int>(bnd.size()) < DMUON_MAX_CHUNKS) {
+      bnd.push_back(i + 1);
+      done += acc;
+      acc = 0;
+      grow *= 1.5;
+    }
+  }
+  bnd.push_back(n);
+  return bnd;
+}
+
 // in[k] are the matrices with a gradient; hg/hp/stage are parallel to in.
 int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
              const std::vector<void*>& hp, const std::vector<void*>& stage, int chunks, void* ws,
@@ -890,12 +921,13 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
     pb[k] = numel * elem_bytes(in[k].pdt);
     total += gb[k];
   }
-  if (chunks <= 0)
-    chunks = static_cast<int>(std::min<size_t>(DMUON_MAX_CHUNKS,
-                                               std::max<size_t>(1, (total + kChunkTargetBytes - 1) /
-                                                                       kChunkTargetBytes)));
-  chunks = std::min(chunks, n);
-  const std::vector<int> bnd = chunk_bounds(gb, chunks);
+  std::vector<int> bnd;
+  if (chunks <= 0) {
+    bnd = ramp_bounds(gb);
+  } else {
+    chunks = std::min(chunks, n);
+    bnd = chunk_bounds(gb, chunks);
+  }
   const int nc = static_cast<int>(bnd.size()) - 1;
   std::vector<std::vector<MatIn>> sub(nc);
   size_t need = 0;
