@@ -97,6 +97,23 @@ bool encode_2d(CUtensorMap* map, int dtype, void* base, uint64_t inner, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// bf16 matrix with `cols` a multiple of 256 seen as 3-D: {64 columns within a
+// block, rows, blocks of 64 columns}, box {64, 64, 4}, 128-byte swizzle.  One
+// box is the 64 x 256 MN-major operand tile that four 2-D boxes would bring,
+// in the same shared-memory layout (four 8 KB blocks).
+bool encode_mn3d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t pitch_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || cols % 256 != 0) return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {pitch_elems * 2, 128};
+  cuuint32_t box[3] = {64, 64, 4};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ inputs
 struct MatIn {
   void* W;
@@ -399,14 +416,19 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
         MatMaps& mm = maps[first + k];
         std::memset(&mm, 0, sizeof(mm));
         bool okm = true;
+        // 3-D MN-major maps when every buffer of the matrix allows them.
+        d.b3d = (dt == DMUON_BF16 && ml.n % 256 == 0) ? 1 : 0;
+        for (int b = 0; b < 2 && d.b3d; ++b)
+          if (d.Xop[b] && !encode_mn3d(&mm.xmn[b], d.Xop[b], ml.n, ml.m, ml.ldx)) d.b3d = 0;
         for (int b = 0; b < 2; ++b) {
           void* xb = d.Xop[b];
           if (!xb) { mm.xk[b] = mm.xk[0]; mm.xmn[b] = mm.xmn[0]; continue; }
           okm &= encode_2d(&mm.xk[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBM);
           // MN-major 32-bit operands need 32-byte swizzle units.
-          okm &= encode_2d(&mm.xmn[b], dt, xb, ml.n, ml.m, ml.ldx, BK, BK,
-                           dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
-                                           : CU_TENSOR_MAP_SWIZZLE_128B);
+          if (!d.b3d)
+            okm &= encode_2d(&mm.xmn[b], dt, xb, ml.n, ml.m, ml.ldx, BK, BK,
+                             dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                             : CU_TENSOR_MAP_SWIZZLE_128B);
         }
         if (d.A) okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
         if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed for matrix %d", i);

@@ -63,12 +63,13 @@ struct MatDesc {
   int g_bf16;          // gradient / input storage: 1 bf16, 0 fp32
   int vec4;            // parameter rows allow 4-element vector access
   int ptiles_c;        // transposed prologue tiles per parameter row band
-  int pad_;
+  int b3d;             // xmn maps are 3-D: one load brings a whole 256-column B operand
 };
 
 struct alignas(64) MatMaps {
   CUtensorMap xk[2];   // Xop as K-major operand, box (128 B of K) x 128 rows
-  CUtensorMap xmn[2];  // Xop as MN-major operand, box (128 B of N) x (BK rows of K)
+  CUtensorMap xmn[2];  // Xop as MN-major operand, box (128 B of N) x (BK rows of K); with b3d a
+                       // 3-D view {64 columns, rows, column blocks of 64} and a box of 4 blocks
   CUtensorMap a;       // A as K-major operand, box (128 B of K) x 128 rows
 };
 
@@ -565,11 +566,16 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           uint8_t* a_dst = sa + stage * kAStageBytes;
           uint8_t* b_dst = sb + stage * kBStageBytes;
           tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
-          for (int j = 0; j < nb; ++j) {
-            if (kMode == kSyrk)
-              tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
-            else
-              tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);
+          if (kMode == kGemm && md.b3d) {
+            // The four 64-column blocks of the tile in one load, same smem layout.
+            tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
+          } else {
+            for (int j = 0; j < nb; ++j) {
+              if (kMode == kSyrk)
+                tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
+              else
+                tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);
+            }
           }
         }
         __syncwarp();
