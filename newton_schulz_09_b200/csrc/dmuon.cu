@@ -422,8 +422,9 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
           if (d.Xop[b] && !encode_mn3d(&mm.xmn[b], d.Xop[b], ml.n, ml.m, ml.ldx)) d.b3d = 0;
         for (int b = 0; b < 2; ++b) {
           void* xb = d.Xop[b];
-          if (!xb) { mm.xk[b] = mm.xk[0]; mm.xmn[b] = mm.xmn[0]; continue; }
+          if (!xb) { mm.xk[b] = mm.xk[0]; mm.xkw[b] = mm.xkw[0]; mm.xmn[b] = mm.xmn[0]; continue; }
           okm &= encode_2d(&mm.xk[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBM);
+          okm &= encode_2d(&mm.xkw[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBN);
           // MN-major 32-bit operands need 32-byte swizzle units.
           if (!d.b3d)
             okm &= encode_2d(&mm.xmn[b], dt, xb, ml.n, ml.m, ml.ldx, BK, BK,
@@ -1464,8 +1465,12 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   bool okm = true;
   for (int b = 0; b < 2; ++b) {
     void* xb = d.X[b];
-    if (!xb) { sp.maps.xk[b] = sp.maps.xk[0]; sp.maps.xmn[b] = sp.maps.xmn[0]; continue; }
+    if (!xb) {
+      sp.maps.xk[b] = sp.maps.xk[0]; sp.maps.xkw[b] = sp.maps.xkw[0]; sp.maps.xmn[b] = sp.maps.xmn[0];
+      continue;
+    }
     okm &= encode_2d(&sp.maps.xk[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBM);
+    okm &= encode_2d(&sp.maps.xkw[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBN);
     okm &= encode_2d(&sp.maps.xmn[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, BK);
   }
   if (d.A) okm &= encode_2d(&sp.maps.a, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, kBM);

@@ -68,6 +68,7 @@ struct MatDesc {
 
 struct alignas(64) MatMaps {
   CUtensorMap xk[2];   // Xop as K-major operand, box (128 B of K) x 128 rows
+  CUtensorMap xkw[2];  // same, box (128 B of K) x 256 rows: a whole SYRK B operand in one load
   CUtensorMap xmn[2];  // Xop as MN-major operand, box (128 B of N) x (BK rows of K); with b3d a
                        // 3-D view {64 columns, rows, column blocks of 64} and a box of 4 blocks
   CUtensorMap a;       // A as K-major operand, box (128 B of K) x 128 rows
@@ -569,6 +570,9 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           if (kMode == kGemm && md.b3d) {
             // The four 64-column blocks of the tile in one load, same smem layout.
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
+          } else if (kMode == kSyrk && nb == 2) {
+            // Both 128-row halves of the B operand in one 256-row load.
+            tma_load_2d(b_dst, &mp.xkw[p.cur], &full[stage], kb * BK, b_row0);
           } else {
             for (int j = 0; j < nb; ++j) {
               if (kMode == kSyrk)
