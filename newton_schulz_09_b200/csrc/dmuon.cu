@@ -97,13 +97,14 @@ bool encode_2d(CUtensorMap* map, int dtype, void* base, uint64_t inner, uint64_t
   return r == CUDA_SUCCESS;
 }
 
-// bf16 matrix with `cols` a multiple of 256 seen as 3-D: {64 columns within a
+// bf16 matrix with `cols` a multiple of 64 seen as 3-D: {64 columns within a
 // block, rows, blocks of 64 columns}, box {64, 64, 4}, 128-byte swizzle.  One
 // box is the 64 x 256 MN-major operand tile that four 2-D boxes would bring,
-// in the same shared-memory layout (four 8 KB blocks).
+// in the same shared-memory layout (four 8 KB blocks); in the last column
+// tile, blocks past the last column are out of bounds and arrive as zeros.
 bool encode_mn3d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t pitch_elems) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || cols % 256 != 0) return false;
+  if (!fn || cols % 64 != 0) return false;
   cuuint64_t dims[3] = {64, rows, cols / 64};
   cuuint64_t strides[2] = {pitch_elems * 2, 128};
   cuuint32_t box[3] = {64, 64, 4};
@@ -417,7 +418,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
         std::memset(&mm, 0, sizeof(mm));
         bool okm = true;
         // 3-D MN-major maps when every buffer of the matrix allows them.
-        d.b3d = (dt == DMUON_BF16 && ml.n % 256 == 0) ? 1 : 0;
+        d.b3d = (dt == DMUON_BF16 && ml.n % 64 == 0) ? 1 : 0;
         for (int b = 0; b < 2 && d.b3d; ++b)
           if (d.Xop[b] && !encode_mn3d(&mm.xmn[b], d.Xop[b], ml.n, ml.m, ml.ldx)) d.b3d = 0;
         for (int b = 0; b < 2; ++b) {

@@ -63,7 +63,7 @@ struct MatDesc {
   int g_bf16;          // gradient / input storage: 1 bf16, 0 fp32
   int vec4;            // parameter rows allow 4-element vector access
   int ptiles_c;        // transposed prologue tiles per parameter row band
-  int b3d;             // xmn maps are 3-D: one load brings a whole 256-column B operand
+  int b3d;             // xmn maps are 3-D (bf16, n % 64 == 0): one load brings a whole B operand
 };
 
 struct alignas(64) MatMaps {
@@ -553,6 +553,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK B operand rows
       if (kMode == kSyrk) {
         nb = (ti.half || ti.tn * kBN + 128 >= md.m) ? 1 : 2;
+      } else if (md.b3d) {
+        nb = NBOX_B;   // the 3-D box is always whole: blocks past the last column arrive as zeros
       } else {
         const int left = md.n - ti.tn * kBN;
         nb = (left + BK - 1) / BK;

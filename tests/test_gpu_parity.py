@@ -27,6 +27,9 @@ def _rand(shape, dtype, seed, std=1.0):
 ORTHO_SHAPES = [
     (128, 256), (256, 512), (512, 256), (384, 384), (200, 328), (328, 200), (1, 1), (1, 9),
     (9, 1), (3, 5), (100, 1000), (1000, 100), (64, 2048), (130, 390), (520, 1040), (257, 513),
+    # long side a multiple of 64 but not of 256: the last column tile of the GEMM's
+    # B operand is partly past the matrix (3-D loads fill it with zeros)
+    (320, 640), (448, 192), (704, 2112),
 ]
 
 
