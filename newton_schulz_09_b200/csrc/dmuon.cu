@@ -742,11 +742,11 @@ int gather(void* const params[], const void* const grads[], float* const bufs[],
 
 // A large call runs as consecutive groups of matrices, one after the other on
 // the stream, sharing one scratch region.  Measured on the Llama-8B stack
-// (224 matrices, 7e9 elements): groups of ~2^30 elements (four layers) run
-// at a higher SM clock under the power cap than one launch per stage over
-// every matrix (413 ms against 440 ms per step); the arithmetic of each
-// matrix does not depend on the grouping.
-constexpr int64_t kGroupElems = int64_t(1) << 30;
+// (224 matrices, 7e9 elements): groups of one to four layers run at a higher
+// SM clock under the power cap than one launch per stage over every matrix
+// (413 ms against 440 ms per step), two-layer groups (~2^29 elements) best
+// by about 1 %; the arithmetic of each matrix does not depend on the grouping.
+constexpr int64_t kGroupElems = int64_t(1) << 29;
 constexpr int kMaxGroups = 32;   // < kMaxPlans: one call never evicts its own plans
 
 // Boundaries of consecutive groups: a matrix joins the current group unless
@@ -900,7 +900,8 @@ constexpr size_t kChunkTargetBytes = size_t(64) << 20;
 // group is small (its upload is exposed), each next one up to 1.5x the one
 // before (an upload must land before the kernels reach it; the copy engines
 // move ~55 GB/s, the update consumes gradients at ~35 GB/s), at most
-// `mid` bytes, and the groups shrink again towards the end (the last
+// `mid` bytes (about the compute grouping of bf16 gradients), and the groups
+// shrink again towards the end (the last
 // group's download is exposed): a group may hold at most a third of the
 // bytes still to come including itself.  At most DMUON_MAX_CHUNKS groups.
 std::vector<int> ramp_bounds(const std::vector<size_t>& bytes) {
@@ -908,7 +909,7 @@ std::vector<int> ramp_bounds(const std::vector<size_t>& bytes) {
   size_t total = 0;
   for (size_t b : bytes) total += b;
   const size_t first = std::max(kChunkTargetBytes, total / 128);
-  const size_t mid = std::max(size_t(2) << 30, total / (DMUON_MAX_CHUNKS / 2));
+  const size_t mid = std::max(size_t(1) << 30, total / (DMUON_MAX_CHUNKS / 2));
   std::vector<int> bnd(1, 0);
   size_t acc = 0, done = 0;
   double grow = static_cast<double>(first);
