@@ -307,6 +307,14 @@ int64_t dmuon_launch_count(void);
  * of memory (host-side fault injection; 0 disables). */
 void dmuon_debug_fail_allocations(int n);
 
+/* Test hook (host only, no CUDA call): the grouping the library uses for these
+ * shapes.  which = 0: the groups of a device call (dmuon_muon_step_batched
+ * and friends, without clipping); which = 1: the automatic groups of
+ * dmuon_muon_step_batched_host (by gradient bytes).  Writes the group
+ * boundaries (bounds[0] = 0, ..., bounds[groups] = count) and returns the
+ * number of groups, or DMUON_ERR_INVALID_ARG (bad shapes, cap < groups + 1). */
+int dmuon_debug_partition(const dmuon_shape shapes[], int count, int which, int* bounds, int cap);
+
 /* Test hook: launches one CTA that waits on a barrier nothing arrives at,
  * with a wait limit of `limit_us` microseconds, then records
  * DMUON_ERR_TIMEOUT in the device error word and returns.  Exercises the

@@ -111,6 +111,7 @@ def load_library() -> ctypes.CDLL:
                                                vp, sz, vp]),
         "dmuon_muon_step_batched_host": (i32, [pp, pp, pp, pp, pp, sp, i32,
                                                ctypes.POINTER(DmuonStepOptions), i32, vp, sz, vp]),
+        "dmuon_debug_partition": (i32, [sp, i32, i32, ctypes.POINTER(ctypes.c_int), i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -766,6 +766,21 @@ std::vector<int> group_bounds(const std::vector<MatIn>& in, int64_t target) {
   return bnd;
 }
 
+// The groups of one call.  Clipping needs one global norm before any
+// momentum update: one group.
+std::vector<int> step_groups(const std::vector<MatIn>& in, bool clipping) {
+  if (clipping) return {0, static_cast<int>(in.size())};
+  int64_t total = 0;
+  for (const MatIn& x : in) total += x.rows * x.cols;
+  int64_t target = std::max<int64_t>(kGroupElems, (total + kMaxGroups - 1) / kMaxGroups);
+  std::vector<int> bnd = group_bounds(in, target);
+  while (static_cast<int>(bnd.size()) - 1 > kMaxGroups) {   // ends: target >= total gives one group
+    target *= 2;
+    bnd = group_bounds(in, target);
+  }
+  return bnd;
+}
+
 int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, const StepOpts& o,
         cudaStream_t st) {
   const int steps = o.steps;
@@ -774,20 +789,7 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
   int dev = 0;
   int r = current_device(&dev);
   if (r != DMUON_OK) return r;
-  // Clipping needs one global norm before any momentum update: one group.
-  std::vector<int> bnd;
-  if (o.max_norm > 0.0f) {
-    bnd = {0, static_cast<int>(in.size())};
-  } else {
-    int64_t total = 0;
-    for (const MatIn& x : in) total += x.rows * x.cols;
-    int64_t target = std::max<int64_t>(kGroupElems, (total + kMaxGroups - 1) / kMaxGroups);
-    bnd = group_bounds(in, target);
-    while (static_cast<int>(bnd.size()) - 1 > kMaxGroups) {   // ends: target >= total gives one group
-      target *= 2;
-      bnd = group_bounds(in, target);
-    }
-  }
+  const std::vector<int> bnd = step_groups(in, o.max_norm > 0.0f);
   const int ng = static_cast<int>(bnd.size()) - 1;
   std::vector<std::vector<MatIn>> sub(ng);
   size_t need = 0;
@@ -1339,6 +1341,27 @@ int64_t dmuon_launch_count(void) {
 void dmuon_debug_fail_allocations(int n) {
   std::lock_guard<std::mutex> lk(g_mu);
   g_fail_allocs = n > 0 ? n : 0;
+}
+
+int dmuon_debug_partition(const dmuon_shape shapes[], int count, int which, int* bounds, int cap) {
+  t_last_error.clear();
+  if (!shapes || !bounds || count < 1 || cap < 2 || (which != 0 && which != 1))
+    return fail(DMUON_ERR_INVALID_ARG, "bad arguments");
+  std::vector<MatIn> in(count);
+  std::vector<size_t> gb(count);
+  for (int i = 0; i < count; ++i) {
+    in[i].rows = shapes[i].rows;
+    in[i].cols = shapes[i].cols;
+    in[i].pdt = shapes[i].param_dtype;
+    in[i].gdt = shapes[i].grad_dtype;
+    if (in[i].rows < 1 || in[i].cols < 1 || (in[i].gdt != DMUON_BF16 && in[i].gdt != DMUON_F32))
+      return fail(DMUON_ERR_INVALID_ARG, "bad shape %d", i);
+    gb[i] = static_cast<size_t>(in[i].rows) * static_cast<size_t>(in[i].cols) * elem_bytes(in[i].gdt);
+  }
+  const std::vector<int> bnd = which == 0 ? step_groups(in, false) : ramp_bounds(gb);
+  if (static_cast<int>(bnd.size()) > cap) return fail(DMUON_ERR_INVALID_ARG, "cap too small");
+  for (size_t k = 0; k < bnd.size(); ++k) bounds[k] = bnd[k];
+  return static_cast<int>(bnd.size()) - 1;
 }
 
 int dmuon_debug_wait_timeout(int limit_us, dmuon_stream_t stream) {

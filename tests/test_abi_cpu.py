@@ -156,3 +156,59 @@ def test_host_buffer_step_rejects_bad_arguments_on_the_host(lib):
     # pointers that are not page-locked host memory are refused
     assert call(ctypes.byref(o)) == -2
     assert "page-locked" in dm.dmuon_last_error()
+
+
+def _partition(lib, dims, which):
+    S = _shapes(*dims)
+    cap = len(dims) + 1
+    B = (ctypes.c_int * cap)()
+    n = lib.dmuon_debug_partition(S, len(dims), which, B, cap)
+    assert n > 0, dm.dmuon_last_error()
+    b = list(B[:n + 1])
+    assert b[0] == 0 and b[-1] == len(dims) and all(x < y for x, y in zip(b, b[1:]))
+    return b
+
+
+def _llama_dims():
+    from newton_schulz_09_b200 import synthetic
+    return [(s.rows, s.cols) for s in synthetic.workload("llama8b").specs]
+
+
+def test_device_call_groups(lib):
+    """Consecutive groups of at most 2^29 elements, each as full as the next
+    matrix allows, at most 32."""
+    dims = _llama_dims()
+    b = _partition(lib, dims, 0)
+    elems = [r * c for r, c in dims]
+    for lo, hi in zip(b, b[1:]):
+        assert sum(elems[lo:hi]) <= 2 ** 29 or hi - lo == 1
+        if hi < len(dims):
+            assert sum(elems[lo:hi + 1]) > 2 ** 29
+    assert len(b) - 1 == 14
+    assert _partition(lib, [(256, 512), (512, 256)], 0) == [0, 2]
+    big = [(16384, 16384)] * 64                       # 1.7e10 elements: the cap of 32 groups
+    assert len(_partition(lib, big, 0)) - 1 <= 32
+
+
+def test_host_step_groups_ramp(lib):
+    """The host-buffer step's automatic groups start and end small and grow
+    by at most 1.5x (plus one matrix) from one group to the next."""
+    dims = _llama_dims()
+    b = _partition(lib, dims, 1)
+    nbytes = [r * c * 2 for r, c in dims]
+    sizes = [sum(nbytes[lo:hi]) for lo, hi in zip(b, b[1:])]
+    total, biggest = sum(nbytes), max(nbytes)
+    assert 8 <= len(sizes) <= 32
+    assert sizes[0] <= total / 32 and sizes[-1] <= total / 32
+    assert max(sizes) <= (1 << 30) + biggest
+    first = max(64 << 20, total // 128)
+    for k, sz in enumerate(sizes[:-1]):
+        assert sz < first * 1.5 ** k + biggest
+    assert _partition(lib, [(256, 512)] * 3, 1) == [0, 3]     # small totals: one group
+
+
+def test_partition_rejects_bad_arguments(lib):
+    B = (ctypes.c_int * 4)()
+    assert lib.dmuon_debug_partition(_shapes((4, 4)), 1, 2, B, 4) == -1
+    assert lib.dmuon_debug_partition(_shapes((0, 4)), 1, 0, B, 4) == -1
+    assert lib.dmuon_debug_partition(_shapes((4, 4)), 1, 0, B, 1) == -1
