@@ -967,8 +967,11 @@ __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_consta
   extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
+  // A block's items only move forward through the matrices: one search,
+  // then a cursor.
+  int mi = blockIdx.x < p.ntiles ? find_slot64(p.ptile_prefix, p.nmat, blockIdx.x) : 0;
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
-    const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
+    while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
     const MatDesc& md = p.mats[mi];
     const int64_t item = t - __ldg(p.ptile_prefix + mi);
     float ss = md.T ? prologue_transposed<E>(p, md, item, pro_stage) : prologue_flat<E>(p, md, item, pro_stage);
@@ -993,8 +996,11 @@ template <typename E>
 __global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_constant__ ElemParams p) {
   __shared__ double red[kPThreads / 32];
   const int tid = threadIdx.x;
+  // A block's items only move forward through the matrices: one search,
+  // then a cursor.
+  int mi = blockIdx.x < p.ntiles ? find_slot64(p.ptile_prefix, p.nmat, blockIdx.x) : 0;
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
-    const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
+    while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
     const MatDesc& md = p.mats[mi];
     const int64_t item = t - __ldg(p.ptile_prefix + mi);
     double ss = 0.0;
@@ -1087,8 +1093,11 @@ __global__ void finalize_kernel(const __grid_constant__ ElemParams p) {
 // prologue.
 template <typename E>
 __global__ void __launch_bounds__(kPThreads) apply_kernel(const __grid_constant__ ElemParams p) {
+  // A block's items only move forward through the matrices: one search,
+  // then a cursor.
+  int mi = blockIdx.x < p.ntiles ? find_slot64(p.ptile_prefix, p.nmat, blockIdx.x) : 0;
   for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x) {
-    const int mi = find_slot64(p.ptile_prefix, p.nmat, t);
+    while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
     const MatDesc& md = p.mats[mi];
     const int64_t item = t - __ldg(p.ptile_prefix + mi);
     const float s = *md.scale;
