@@ -11,6 +11,10 @@
 //                         GEMM  X' = c (1.5 X - 0.5 A X), or on the last step
 //                               the weight update / output write.   [tensor]
 //   apply_kernel        the update for ns_steps == 0 (X = s M).
+//   grad_norm_kernel,   Muon-only global-norm gradient clipping: per-item
+//   clip_coef_kernel    sums of g^2 (fp64), then the clip coefficient.
+//   adamw_kernel        AdamW of the parameters Muon does not orthogonalise.
+//   wait_timeout_kernel test kernel of the bounded-wait path.
 //
 // Sources: DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销",
 // sections "Muon 核心：Newton-Schulz 迭代" (normalisation, cubic step,
