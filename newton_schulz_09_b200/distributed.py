@@ -7,15 +7,19 @@ LPT partition; the blog's "参数分片减少 N-S 计算量": each rank runs N-S
 on its share).  One step:
 
 1. the gradients are reduced to their owners (sum, then divided by the
-   number of ranks: the data-parallel mean), all reductions in flight at
-   once;
-2. every owner runs one batched Muon update over the matrices it owns (one
-   launch per stage on the GPU) -- only owners keep momentum buffers;
-3. every updated matrix is broadcast from its owner.
+   number of ranks: the data-parallel mean), every reduction issued at once;
+2. every owner updates the matrices it owns in a few chunks, one batched
+   call each (only owners keep momentum buffers); a chunk waits only for its
+   own reductions, so later reductions run while earlier chunks compute;
+3. every updated matrix is broadcast from its owner as soon as its chunk is
+   done, while later chunks compute.
 
-The collectives go through ``torch.distributed`` (NCCL on GPUs, gloo on
-CPUs); the update itself is ``dmuon_muon_step_batched`` unless a step
-function is given (the CPU tests pass one).
+All ranks issue the same collectives in the same order: every reduction,
+then the broadcasts chunk by chunk in one global schedule that interleaves
+the owners.  The collectives go through ``torch.distributed`` (NCCL on
+GPUs, gloo on CPUs), whose waits are stream-ordered on GPUs; the update
+itself is ``dmuon_muon_step_batched`` unless a step function is given (the
+CPU tests pass one).
 """
 from __future__ import annotations
 
@@ -65,6 +69,36 @@ def _default_step(params, grads, bufs, **kw) -> None:
     dmuon_muon_step_batched(params, grads, bufs, **kw)
 
 
+def owner_chunks(owner: Sequence[int], numel: Sequence[int], world: int,
+                 chunks_per_owner: int = 4) -> List[List[List[int]]]:
+    """Per owner rank, its matrices (in index order) cut into at most
+    ``chunks_per_owner`` consecutive chunks of about equal element count."""
+    out: List[List[List[int]]] = []
+    for r in range(world):
+        mine = [i for i, o in enumerate(owner) if o == r]
+        total = sum(numel[i] for i in mine)
+        target = total / max(1, chunks_per_owner)
+        chunks: List[List[int]] = []
+        cur: List[int] = []
+        acc = 0
+        for i in mine:
+            cur.append(i)
+            acc += numel[i]
+            if acc >= target and len(chunks) + 1 < chunks_per_owner:
+                chunks.append(cur)
+                cur, acc = [], 0
+        if cur:
+            chunks.append(cur)
+        out.append(chunks)
+    return out
+
+
+def global_schedule(chunks: Sequence[Sequence[Sequence[int]]]) -> List[tuple]:
+    """(owner, chunk index) pairs, chunk 0 of every owner first, then chunk 1, ..."""
+    depth = max((len(c) for c in chunks), default=0)
+    return [(r, c) for c in range(depth) for r in range(len(chunks)) if c < len(chunks[r])]
+
+
 class OwnerPartitionedMuon:
     """Muon over data-parallel ranks with one owner per matrix.
 
@@ -73,7 +107,7 @@ class OwnerPartitionedMuon:
     """
 
     def __init__(self, params: Sequence[torch.Tensor], group=None, ns_steps: int = 5,
-                 step_fn: Optional[StepFn] = None):
+                 step_fn: Optional[StepFn] = None, chunks_per_owner: int = 4):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -86,6 +120,9 @@ class OwnerPartitionedMuon:
                                     device=self.params[i].device) for i in self.owned}
         self.step_fn = step_fn or _default_step
         self.imbalance = imbalance(costs, self.owner, self.world)
+        self.chunks = owner_chunks(self.owner, [p.numel() for p in self.params], self.world,
+                                   chunks_per_owner)
+        self.schedule = global_schedule(self.chunks)
 
     def _global_rank(self, r: int) -> int:
         return r if self.group is None else dist.get_global_rank(self.group, r)
@@ -95,36 +132,38 @@ class OwnerPartitionedMuon:
              momentum: float = 0.95, nesterov: bool = True, weight_decay: float = 0.0) -> None:
         """One step.  ``grads`` are this rank's local gradients (None for a
         parameter without gradient on every rank); they are overwritten by
-        the reduction on the owner."""
-        # 1. reduce every gradient to its owner, all in flight at once
-        work = []
+        the reduction on the owner.  On GPUs the call only enqueues work (the
+        collectives' waits are stream-ordered); the parameters are final once
+        the current stream reaches the end of the step."""
+        # 1. every reduction to its owner, all in flight at once
+        red = {}
         for i, g in enumerate(grads):
-            if g is None:
+            if g is not None:
+                red[i] = dist.reduce(g, dst=self._global_rank(self.owner[i]), op=dist.ReduceOp.SUM,
+                                     group=self.group, async_op=True)
+        # 2.-3. chunk by chunk in the global schedule: the owner updates its
+        # chunk once that chunk's reductions are done, then every rank takes
+        # part in the chunk's broadcasts
+        bcast = []
+        for r, c in self.schedule:
+            idx = [i for i in self.chunks[r][c] if grads[i] is not None]
+            if not idx:
                 continue
-            work.append(dist.reduce(g, dst=self._global_rank(self.owner[i]), op=dist.ReduceOp.SUM,
-                                    group=self.group, async_op=True))
-        for w in work:
-            w.wait()
-        # 2. owners update their matrices in one batched call
-        ps, gs, bs = [], [], []
-        for i in self.owned:
-            if grads[i] is None:
-                continue
-            g = grads[i]
-            if self.world > 1:
-                g.div_(self.world)
-            ps.append(self.params[i])
-            gs.append(g)
-            bs.append(self.bufs[i])
-        if ps:
-            self.step_fn(ps, gs, bs, lr=lr, momentum=momentum, nesterov=nesterov,
-                         weight_decay=weight_decay, ns_steps=self.ns_steps)
-        # 3. broadcast every updated matrix from its owner
-        work = []
-        for i, g in enumerate(grads):
-            if g is None:
-                continue
-            work.append(dist.broadcast(self.params[i], src=self._global_rank(self.owner[i]),
-                                       group=self.group, async_op=True))
-        for w in work:
+            if r == self.rank:
+                for i in idx:
+                    red[i].wait()
+                gs = [grads[i] for i in idx]
+                if self.world > 1:
+                    for g in gs:
+                        g.div_(self.world)
+                self.step_fn([self.params[i] for i in idx], gs, [self.bufs[i] for i in idx], lr=lr,
+                             momentum=momentum, nesterov=nesterov, weight_decay=weight_decay,
+                             ns_steps=self.ns_steps)
+            for i in idx:
+                bcast.append(dist.broadcast(self.params[i], src=self._global_rank(r), group=self.group,
+                                            async_op=True))
+        for i, w in red.items():
+            if self.owner[i] != self.rank:
+                w.wait()
+        for w in bcast:
             w.wait()

@@ -37,8 +37,10 @@ def _params():
 
 
 def _grads(rank, step):
+    # small multiples of 2^-20: fp32 sums over ranks are exact in any order,
+    # so the mean is one rounding whatever order the reduction takes
     gen = torch.Generator().manual_seed(1000 * step + rank)
-    gs = [torch.randn(s, generator=gen) * 1e-3 for s in SHAPES]
+    gs = [torch.randint(-1000, 1001, s, generator=gen).float() * 2.0 ** -20 for s in SHAPES]
     gs[4] = None if step == 1 else gs[4]          # no gradient for one matrix on step 1
     return gs
 
@@ -82,25 +84,42 @@ def test_lpt_partition_is_deterministic_and_balanced():
         dmd.lpt_partition([1.0], 0)
 
 
-def test_two_ranks_match_one_step_on_averaged_gradients(tmp_path):
-    world = 2
+def test_owner_chunks_and_global_schedule():
+    owner = [0, 1, 0, 0, 1, 2, 0, 0]
+    numel = [10, 5, 10, 10, 5, 7, 10, 10]
+    ch = dmd.owner_chunks(owner, numel, 3, chunks_per_owner=2)
+    # each owner's matrices, in index order, cut into consecutive chunks
+    for r in range(3):
+        assert sum(ch[r], []) == [i for i, o in enumerate(owner) if o == r]
+        assert 1 <= len(ch[r]) <= 2
+    assert ch[0] == [[0, 2, 3], [6, 7]]
+    sched = dmd.global_schedule(ch)
+    # chunk 0 of every owner, then chunk 1 of those that have one
+    assert sched[:3] == [(0, 0), (1, 0), (2, 0)]
+    assert sorted(sched) == sorted((r, c) for r in range(3) for c in range(len(ch[r])))
+    assert dmd.global_schedule([[], [[1]]]) == [(1, 0)]
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ranks_match_one_step_on_averaged_gradients(tmp_path, world):
     mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
                        start_method="spawn", join=True)
     res = [torch.load(tmp_path / f"rank{r}.pt") for r in range(world)]
-    # both ranks hold identical weights after the broadcast
-    for a, b in zip(res[0]["params"], res[1]["params"]):
-        assert torch.equal(a, b)
+    # every rank holds identical weights after the broadcasts
+    for r in range(1, world):
+        for a, b in zip(res[0]["params"], res[r]["params"]):
+            assert torch.equal(a, b)
     # every matrix has exactly one owner, and only owners keep buffers
-    assert sorted(res[0]["owned"] + res[1]["owned"]) == list(range(len(SHAPES)))
-    # reference: two oracle steps on the mean gradient (sum in fp32, then / 2)
+    assert sorted(sum((res[r]["owned"] for r in range(world)), [])) == list(range(len(SHAPES)))
+    # reference: two oracle steps on the mean gradient (exact fp32 sum, then / world)
     W = [p.numpy().copy() for p in _params()]
     bufs = [np.zeros(s, np.float32) for s in SHAPES]
     for step in range(2):
-        g0, g1 = _grads(0, step), _grads(1, step)
+        gr = [_grads(r, step) for r in range(world)]
         for i in range(len(SHAPES)):
-            if g0[i] is None:
+            if gr[0][i] is None:
                 continue
-            gm = ((g0[i] + g1[i]) / 2).numpy()
+            gm = (sum(g[i] for g in gr) / world).numpy()
             bufs[i], _, Wn = oracle.muon_step(W[i], gm, bufs[i], ns_steps=3, **HP)
             W[i] = Wn.astype(np.float32)
     for i in range(len(SHAPES)):
