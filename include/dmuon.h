@@ -168,6 +168,29 @@ int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[]
                                  void* workspace, size_t ws_bytes, dmuon_stream_t stream);
 
 /*
+ * dmuon_muon_step_batched_reduce -- the owner's update of an owner-partitioned
+ * data-parallel step (the quick start's "刚才发生了什么": each projection has
+ * one owner that reduces its gradient and runs Newton-Schulz on it) with the
+ * gradient reduction fused into the update: matrix i's gradient is the mean
+ * of `world` buffers, grads[r * count + i] for r = 0 .. world-1, which the
+ * prologue reads directly.  In a multi-GPU job these are other GPUs' buffers
+ * mapped into this process (peer access, CUDA IPC or symmetric memory; the
+ * caller makes sure every rank's gradient is complete first); any device
+ * pointers work.  The mean is defined exactly: an fp32 sum in rank order,
+ * then one fp32 division by `world` (round to nearest), so the momentum
+ * buffers are reproducible bit for bit.  world == 1 is
+ * dmuon_muon_step_batched_opts.
+ *   grads      world * count device pointers, rank-major; for a matrix either
+ *              every rank's pointer is NULL (the matrix is skipped) or none.
+ *   world      1 .. 64.  Other arguments as dmuon_muon_step_batched_opts
+ *              (clipping, when on, uses the norm of the mean gradients).
+ */
+int dmuon_muon_step_batched_reduce(void* const params[], const void* const grads[], float* const bufs[],
+                                   const dmuon_shape shapes[], int count, int world,
+                                   const dmuon_step_options* opts, void* workspace, size_t ws_bytes,
+                                   dmuon_stream_t stream);
+
+/*
  * dmuon_muon_step_batched_host -- the same Muon update (the blog's Vanilla
  * Muon step, "代码实现" section) for a caller whose gradients arrive in, and
  * whose updated weights must return to, page-locked host memory.  The

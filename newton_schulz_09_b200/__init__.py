@@ -24,6 +24,7 @@ __all__ = [
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
     "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
     "dmuon_adamw_step_batched", "DmuonTensorDesc", "dmuon_muon_step_batched_host",
+    "dmuon_muon_step_batched_reduce",
     "DMUON_MAX_CHUNKS",
 ]
 
@@ -112,6 +113,8 @@ def load_library() -> ctypes.CDLL:
         "dmuon_muon_step_batched_host": (i32, [pp, pp, pp, pp, pp, sp, i32,
                                                ctypes.POINTER(DmuonStepOptions), i32, vp, sz, vp]),
         "dmuon_debug_partition": (i32, [sp, i32, i32, ctypes.POINTER(ctypes.c_int), i32]),
+        "dmuon_muon_step_batched_reduce": (i32, [pp, pp, pp, sp, i32, i32, ctypes.POINTER(DmuonStepOptions),
+                                                 vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -280,6 +283,54 @@ def dmuon_muon_step_batched_opts(params, grads, bufs, lr: float = 0.02, momentum
     with torch.cuda.device(b.device):
         _check(lib.dmuon_muon_step_batched_opts(*b.args(), ctypes.byref(o), ws_ptr, ws_bytes,
                                                 _stream(b.device)))
+
+
+def dmuon_muon_step_batched_reduce(params, rank_grads, bufs, lr: float = 0.02, momentum: float = 0.95,
+                                   nesterov: bool = True, weight_decay: float = 0.0, ns_steps: int = 5,
+                                   ns_coefficients=(1.5, -0.5), lr_scale: str = "plain",
+                                   max_grad_norm: float = 0.0,
+                                   workspace: Optional[torch.Tensor] = None) -> None:
+    """The owner's step with the data-parallel gradient reduction fused in:
+    ``rank_grads[r][i]`` is rank r's gradient of parameter i (a CUDA tensor
+    this device can read: local, or another GPU's memory mapped here); the
+    update uses their mean (fp32 sum in rank order, then one division).
+    ``rank_grads[r][i]`` must be None for every rank or for none."""
+    lib = load_library()
+    world = len(rank_grads)
+    n = len(params)
+    if world < 1 or any(len(g) != n for g in rank_grads):
+        raise ValueError("rank_grads must hold one list of len(params) gradients per rank")
+    for r in range(1, world):
+        for i in range(n):
+            g, g0 = rank_grads[r][i], rank_grads[0][i]
+            if (g is None) != (g0 is None):
+                raise ValueError(f"gradient {i}: given on some ranks only")
+            if g is not None:
+                if not g.is_cuda or g.dtype != g0.dtype or g.shape != g0.shape or not g.is_contiguous():
+                    raise ValueError(f"rank_grads[{r}][{i}] must match rank 0's gradient (CUDA, dtype, shape)")
+    b = _Batch(params, rank_grads[0], bufs)
+    if b.n == 0:
+        return
+    G = (ctypes.c_void_p * (world * n))()
+    for r in range(world):
+        for i in range(n):
+            g = rank_grads[r][i]
+            G[r * n + i] = g.data_ptr() if g is not None else None
+    o = DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
+    o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
+    o.ns_a, o.ns_b = ns_coefficients
+    o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
+    o.max_grad_norm = max_grad_norm
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    P, _, B, S, cnt = b.args()
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    with torch.cuda.device(b.device):
+        _check(lib.dmuon_muon_step_batched_reduce(P, ctypes.cast(G, pp), B, S, cnt, world, ctypes.byref(o),
+                                                  ws_ptr, ws_bytes, _stream(b.device)))
 
 
 def dmuon_muon_step_batched_host(params, grads, bufs, host_grads, host_params=None,

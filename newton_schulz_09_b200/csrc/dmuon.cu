@@ -124,6 +124,7 @@ struct MatIn {
   int pdt, gdt;
   int mode;
   float lr_mult = 1.0f;   // per-matrix factor on lr
+  std::vector<const void*> gr;   // with more than one: the ranks' gradient buffers to average
 };
 
 // Scalars and switches of one call.
@@ -347,6 +348,8 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     put(key, x.W); put(key, x.G); put(key, x.buf);
     put(key, x.rows); put(key, x.cols);
     put(key, x.pdt); put(key, x.gdt); put(key, x.mode); put(key, x.lr_mult);
+    put(key, static_cast<int64_t>(x.gr.size()));
+    for (const void* q : x.gr) put(key, q);
   }
   const uint64_t h = fnv1a(key.data(), key.size());
   for (auto it = g_plans.begin(); it != g_plans.end(); ++it) {
@@ -411,6 +414,9 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
       d.g_bf16 = x.gdt == DMUON_BF16 ? 1 : 0;
       d.vec4 = (x.cols % 4 == 0) && aligned(x.W, 16) && aligned(x.G, 16) &&
                (x.buf == nullptr || aligned(x.buf, 16));
+      for (const void* q : x.gr) d.vec4 = d.vec4 && aligned(q, 16);
+      d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
+      d.Gr = nullptr;   // set once the plan's device memory exists
       d.ptiles_c = static_cast<int>(ml.ptiles_c);
       A.pp.push_back(A.pp.back() + ml.ptiles);
       if (ws) {
@@ -480,7 +486,27 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     o_g[gi * 5 + 3] = off; off = align_up(off + sizeof(int) * ga[gi].go.size(), 128);
     o_g[gi * 5 + 4] = off; off = align_up(off + sizeof(int) * ga[gi].gp.size(), 128);
   }
+  // The ranks' gradient buffers of matrices that average several (rank order).
+  std::vector<const void*> gr_ptrs;
+  std::vector<int64_t> gr_at(nmat, -1);
+  for (int i = 0; i < nmat; ++i) {
+    if (in[i].gr.size() > 1) {
+      gr_at[desc_of[i]] = static_cast<int64_t>(gr_ptrs.size());
+      gr_ptrs.insert(gr_ptrs.end(), in[i].gr.begin(), in[i].gr.end());
+    }
+  }
+  const size_t o_gr = off; off = align_up(off + sizeof(void*) * gr_ptrs.size(), 128);
+  cudaError_t e = lib_malloc(&P->dmem, off);
+  if (e != cudaSuccess) {
+    P->dmem = nullptr;
+    return fail(DMUON_ERR_NO_WORKSPACE, "plan allocation of %zu bytes failed", off);
+  }
+  uint8_t* base = static_cast<uint8_t*>(P->dmem);
+  for (int k = 0; k < nmat; ++k)
+    if (gr_at[k] >= 0)
+      descs[k].Gr = reinterpret_cast<const void* const*>(base + o_gr + sizeof(void*) * gr_at[k]);
   std::vector<uint8_t> img(off, 0);
+  if (!gr_ptrs.empty()) std::memcpy(img.data() + o_gr, gr_ptrs.data(), sizeof(void*) * gr_ptrs.size());
   std::memcpy(img.data() + o_desc, descs.data(), sizeof(MatDesc) * nmat);
   std::memcpy(img.data() + o_maps, maps.data(), sizeof(MatMaps) * nmat);
   for (size_t gi = 0; gi < ga.size(); ++gi) {
@@ -490,14 +516,8 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     std::memcpy(img.data() + o_g[gi * 5 + 3], ga[gi].go.data(), sizeof(int) * ga[gi].go.size());
     std::memcpy(img.data() + o_g[gi * 5 + 4], ga[gi].gp.data(), sizeof(int) * ga[gi].gp.size());
   }
-  cudaError_t e = lib_malloc(&P->dmem, img.size());
-  if (e != cudaSuccess) {
-    P->dmem = nullptr;
-    return fail(DMUON_ERR_NO_WORKSPACE, "plan allocation of %zu bytes failed", img.size());
-  }
   e = cudaMemcpy(P->dmem, img.data(), img.size(), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "plan upload");
-  uint8_t* base = static_cast<uint8_t*>(P->dmem);
   for (size_t gi = 0; gi < P->groups.size(); ++gi) {
     GroupPlan& gp = P->groups[gi];
     gp.pprefix = reinterpret_cast<const int64_t*>(base + o_g[gi * 5 + 0]);
@@ -1082,6 +1102,50 @@ int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[]
   std::vector<MatIn> in;
   r = gather(params, grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
   if (r != DMUON_OK) return r;
+  return run(in, workspace, ws_bytes, workspace == nullptr, o, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dmuon_muon_step_batched_reduce(void* const params[], const void* const grads[], float* const bufs[],
+                                   const dmuon_shape shapes[], int count, int world,
+                                   const dmuon_step_options* opts, void* workspace, size_t ws_bytes,
+                                   dmuon_stream_t stream) {
+  t_last_error.clear();
+  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
+  if (opts->struct_size != sizeof(dmuon_step_options))
+    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
+                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
+  if (world < 1 || world > 64) return fail(DMUON_ERR_INVALID_ARG, "world must be in [1, 64]");
+  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
+  o.ca = opts->ns_a;
+  o.cb = opts->ns_b;
+  o.lr_scale = opts->lr_scale;
+  o.max_norm = opts->max_grad_norm;
+  o.norm_out = opts->grad_norm_out;
+  int r = check_opts(o);
+  if (r != DMUON_OK) return r;
+  if (o.norm_out && !aligned(o.norm_out, 4)) return fail(DMUON_ERR_INVALID_ARG, "grad_norm_out misaligned");
+  if (count > 0 && !grads) return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  // Rank 0's pointers stand for the gradients in the argument checks.
+  std::vector<MatIn> in;
+  r = gather(params, grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
+  if (r != DMUON_OK) return r;
+  size_t k = 0;
+  for (int i = 0; i < count; ++i) {
+    const bool has = grads[i] != nullptr;
+    const size_t eb = (shapes[i].grad_dtype == DMUON_BF16) ? 2 : 4;
+    for (int q = 1; q < world; ++q) {
+      const void* g = grads[static_cast<int64_t>(q) * count + i];
+      if ((g != nullptr) != has)
+        return fail(DMUON_ERR_INVALID_ARG, "matrix %d: rank %d's gradient is %s while rank 0's is %s", i, q,
+                    g ? "given" : "NULL", has ? "given" : "NULL");
+      if (g && !aligned(g, eb))
+        return fail(DMUON_ERR_INVALID_ARG, "matrix %d: rank %d's gradient is misaligned", i, q);
+    }
+    if (!has) continue;
+    if (world > 1)
+      for (int q = 0; q < world; ++q) in[k].gr.push_back(grads[static_cast<int64_t>(q) * count + i]);
+    ++k;
+  }
   return run(in, workspace, ws_bytes, workspace == nullptr, o, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -68,6 +68,8 @@ struct MatDesc {
   int vec4;            // parameter rows allow 4-element vector access
   int ptiles_c;        // transposed prologue tiles per parameter row band
   int b3d;             // xmn maps are 3-D (bf16, n % 64 == 0): one load brings a whole B operand
+  int world;           // > 1: the gradient is the mean of `world` buffers Gr[0..world)
+  const void* const* Gr;  // device array of the ranks' gradient buffers (rank order), or nullptr
 };
 
 struct alignas(64) MatMaps {
@@ -684,7 +686,9 @@ static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes, "transpose tile must fit the
 // memory with 16-byte asynchronous copies: the gradient at sg (2 or 4 bytes
 // an element), the momentum at sb.  Only whole, 16-byte aligned segments.
 __device__ __forceinline__ void stage8(const MatDesc& md, int64_t idx, bool has_buf, uint8_t* sg, float* sb) {
-  if (md.g_bf16) {
+  if (md.world > 1) {
+    // the mean over the ranks is read directly at use
+  } else if (md.g_bf16) {
     cp_async16(sg, reinterpret_cast<const __nv_bfloat16*>(md.G) + idx);
   } else {
     const float* g = reinterpret_cast<const float*>(md.G) + idx;
@@ -698,7 +702,9 @@ __device__ __forceinline__ void stage8(const MatDesc& md, int64_t idx, bool has_
 }
 __device__ __forceinline__ void unstage8(const MatDesc& md, bool has_buf, const uint8_t* sg, const float* sb,
                                          float (&g)[8], float (&b)[8]) {
-  if (md.g_bf16) {
+  if (md.world > 1) {
+    // not staged: the caller reads the mean over the ranks
+  } else if (md.g_bf16) {
     const uint4 u = *reinterpret_cast<const uint4*>(sg);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -721,10 +727,11 @@ __device__ __forceinline__ void unstage8(const MatDesc& md, bool has_buf, const 
   }
 }
 
-// 8 consecutive input elements (bf16 or fp32), 16-byte aligned when vec.
-__device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool vec, int valid, float (&g)[8]) {
-  if (md.g_bf16) {
-    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(md.G) + idx;
+// 8 consecutive elements (bf16 or fp32) of G, 16-byte aligned when vec.
+__device__ __forceinline__ void load8_from(const void* G, int g_bf16, int64_t idx, bool vec, int valid,
+                                           float (&g)[8]) {
+  if (g_bf16) {
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(G) + idx;
     if (vec) {
       const uint4 u = *reinterpret_cast<const uint4*>(src);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -739,7 +746,7 @@ __device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool ve
       for (int e = 0; e < 8; ++e) g[e] = (e < valid) ? __bfloat162float(src[e]) : 0.0f;
     }
   } else {
-    const float* src = reinterpret_cast<const float*>(md.G) + idx;
+    const float* src = reinterpret_cast<const float*>(G) + idx;
     if (vec) {
       const float4 a = *reinterpret_cast<const float4*>(src);
       const float4 b = *reinterpret_cast<const float4*>(src + 4);
@@ -750,6 +757,26 @@ __device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool ve
       for (int e = 0; e < 8; ++e) g[e] = (e < valid) ? src[e] : 0.0f;
     }
   }
+}
+// 8 consecutive gradient elements.  With world > 1 the gradient is the
+// data-parallel mean, read straight from every rank's buffer (in a multi-GPU
+// job, peer memory mapped into this process): an fp32 sum in rank order,
+// then one division by the number of ranks.
+__device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool vec, int valid, float (&g)[8]) {
+  if (md.world <= 1) {
+    load8_from(md.G, md.g_bf16, idx, vec, valid, g);
+    return;
+  }
+  load8_from(md.Gr[0], md.g_bf16, idx, vec, valid, g);
+  for (int r = 1; r < md.world; ++r) {
+    float h[8];
+    load8_from(md.Gr[r], md.g_bf16, idx, vec, valid, h);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g[e] = __fadd_rn(g[e], h[e]);
+  }
+  const float w = static_cast<float>(md.world);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) g[e] = __fdiv_rn(g[e], w);
 }
 __device__ __forceinline__ void load8_f32(const float* src, bool vec, int valid, float (&b)[8]) {
   if (vec) {
@@ -850,6 +877,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
     float g[8], b[8], M[8];
     if (vec) {
       unstage8(md, has_buf, stage + le * gb, sbuf + le, g, b);
+      if (md.world > 1) load8_in(md, e, true, 8, g);
     } else {
       load8_in(md, e, vec, valid, g);
       if (has_buf) load8_f32(md.buf + e, vec, valid, b);
@@ -920,6 +948,7 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
     if (vec) {
       const int slot = (i * kPThreads + tid) * 8;
       unstage8(md, has_buf, stage + slot * gb, sbuf + slot, g, b);
+      if (md.world > 1) load8_in(md, idx, true, 8, g);
     } else if (valid > 0) {
       load8_in(md, idx, vec, valid, g);
       if (has_buf) load8_f32(md.buf + idx, vec, valid, b);

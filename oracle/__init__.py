@@ -19,6 +19,7 @@ from .muon_oracle import (  # noqa: F401
     newton_schulz,
     ns_flops,
     ns_iteration,
+    rank_mean,
     orthogonality_error,
     relative_frobenius,
 )

@@ -197,6 +197,18 @@ def ns_flops(rows: int, cols: int, steps: int) -> float:
     return float(steps) * 3.0 * m * m * n
 
 
+def rank_mean(grads):
+    """Data-parallel mean of the ranks' gradients, as the owner computes it
+    when it reduces the gradient of a projection it owns (quick start,
+    "刚才发生了什么"; blog "参数分片减少 N-S 计算量"): a float32 sum in rank
+    order, then one float32 division by the number of ranks (the library's
+    fused owner step fixes this order so the buffers are reproducible)."""
+    acc = np.array(grads[0], dtype=np.float32, copy=True)
+    for g in grads[1:]:
+        acc = np.add(acc, np.asarray(g, dtype=np.float32), dtype=np.float32)
+    return np.divide(acc, np.float32(len(grads)), dtype=np.float32)
+
+
 def adamw_step(p, g, m, v, *, lr: float, beta1: float, beta2: float, eps: float,
                weight_decay: float, step: int):
     """AdamW of one tensor (training guide, "第 4 步：创建优化器": the second

@@ -382,7 +382,28 @@ def pin_adamw(o, seed: int = 20) -> None:
         assert m2[i] == want_m and v2[i] == want_v, i
 
 
+def pin_rank_mean(o) -> None:
+    """Mean of the ranks' gradients for the owner's fused reduction:
+    * one rank: the gradient itself, bit for bit;
+    * exactly summable values: the exact mean;
+    * the float32 sum runs in rank order: 1 + 2^-24 + 2^-24 rounds to 1 each
+      time (ties to even), while any other order or a wider sum keeps 2^-23;
+    * the division is one correctly rounded float32 division, checked
+      against exact rational rounding of S / 3 for S = 1 .. 200."""
+    g = np.array([0.1, -3.0, 7e-9], dtype=np.float32)
+    assert np.array_equal(o.rank_mean([g]).view(np.uint32), g.view(np.uint32))
+    ranks = [np.array([v], dtype=np.float32) for v in (1.0, 2.0, 3.0, 6.0)]
+    assert o.rank_mean(ranks)[0] == np.float32(3.0)
+    t = np.float32(2.0 ** -24)
+    got = o.rank_mean([np.array([1.0], np.float32), np.array([t]), np.array([t])])[0]
+    assert got == exact_f32_round(Fraction(1, 3)), got
+    S = np.arange(1, 201, dtype=np.float32)
+    got = o.rank_mean([S, np.zeros_like(S), np.zeros_like(S)])
+    for k in range(S.size):
+        assert got[k] == exact_f32_round(Fraction(int(S[k]), 3)), (k, got[k])
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
-            pin_lr_scale, pin_gradient_clipping, pin_adamw)
+            pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean)

@@ -164,6 +164,29 @@ MUTANTS["adamw_eps_inside_sqrt"] = dict(adamw_step=_adamw_variant("eps_inside_sq
 MUTANTS["clip_after_momentum"] = dict(muon_step=_clip_after_momentum)
 MUTANTS["lr_scale_min_side"] = dict(muon_step=_lr_scale_min_side)
 MUTANTS["custom_coefficients_ignored"] = dict(newton_schulz=_coeffs_ignored)
+
+
+def _rank_mean_variant(kind):
+    def f(grads):
+        gs = [np.asarray(g, np.float32) for g in grads]
+        w = np.float32(len(gs))
+        if kind == "wide_sum":
+            return (sum(g.astype(np.float64) for g in gs) / len(gs)).astype(np.float32)
+        if kind == "reverse_order":
+            acc = gs[-1].copy()
+            for g in reversed(gs[:-1]):
+                acc = np.add(acc, g, dtype=np.float32)
+            return np.divide(acc, w, dtype=np.float32)
+        acc = gs[0].copy()
+        for g in gs[1:]:
+            acc = np.add(acc, g, dtype=np.float32)
+        return np.multiply(acc, np.float32(1.0) / w, dtype=np.float32)   # reciprocal
+    return f
+
+
+MUTANTS["rank_mean_wide_sum"] = dict(rank_mean=_rank_mean_variant("wide_sum"))
+MUTANTS["rank_mean_reverse_order"] = dict(rank_mean=_rank_mean_variant("reverse_order"))
+MUTANTS["rank_mean_reciprocal"] = dict(rank_mean=_rank_mean_variant("reciprocal"))
 MUTANTS["clip_no_eps"] = dict(clip_coefficient=lambda grads, mx: (np.float32(min(1.0, float(np.float32(mx)) / np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))), float(np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))))
 
 
