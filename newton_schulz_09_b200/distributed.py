@@ -104,10 +104,19 @@ class OwnerPartitionedMuon:
 
     ``params`` are the full replicated weights (same on every rank).  Each
     rank allocates momentum buffers only for the matrices it owns.
+
+    ``grad_exchange``: "nccl" (default) reduces each gradient to its owner
+    with a collective.  "peer" keeps the gradients in symmetric memory
+    (``self.grads``, one view per parameter in the parameter's dtype, which
+    the caller fills): after a stream-ordered barrier each owner reads every
+    rank's gradient of the matrices it owns straight from peer memory inside
+    its update (``dmuon_muon_step_batched_reduce``), so no reduced copy is
+    written; the updated weights are then broadcast as in the NCCL mode.
     """
 
     def __init__(self, params: Sequence[torch.Tensor], group=None, ns_steps: int = 5,
-                 step_fn: Optional[StepFn] = None, chunks_per_owner: int = 4):
+                 step_fn: Optional[StepFn] = None, chunks_per_owner: int = 4,
+                 grad_exchange: str = "nccl"):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -123,9 +132,71 @@ class OwnerPartitionedMuon:
         self.chunks = owner_chunks(self.owner, [p.numel() for p in self.params], self.world,
                                    chunks_per_owner)
         self.schedule = global_schedule(self.chunks)
+        if grad_exchange not in ("nccl", "peer"):
+            raise ValueError("grad_exchange must be 'nccl' or 'peer'")
+        self.grad_exchange = grad_exchange
+        self.grads: Optional[List[torch.Tensor]] = None
+        if grad_exchange == "peer":
+            self._setup_peer()
+
+    def _setup_peer(self) -> None:
+        """One symmetric buffer per gradient dtype holding every parameter's
+        gradient (16-byte aligned offsets), and views of every rank's copy."""
+        import torch.distributed._symmetric_memory as symm
+        dev = self.params[0].device
+        if dev.type != "cuda":
+            raise ValueError("grad_exchange='peer' needs CUDA parameters")
+        group = self.group if self.group is not None else dist.group.WORLD
+        self.grads = [None] * len(self.params)
+        self._peer: dict = {}
+        self._handles = []
+        by_dtype: dict = {}
+        for i, p in enumerate(self.params):
+            by_dtype.setdefault(p.dtype, []).append(i)
+        for dt in sorted(by_dtype, key=str):            # the same order on every rank
+            idx = by_dtype[dt]
+            align = 16 // torch.empty((), dtype=dt).element_size()
+            offs, total = [], 0
+            for i in idx:
+                offs.append(total)
+                total += -(-self.params[i].numel() // align) * align
+            buf = symm.empty(total, dtype=dt, device=dev)
+            hdl = symm.rendezvous(buf, group)
+            self._handles.append((buf, hdl))
+            for i, off in zip(idx, offs):
+                n, shape = self.params[i].numel(), self.params[i].shape
+                self.grads[i] = buf[off:off + n].view(shape)
+                self._peer[i] = [hdl.get_buffer(r, (n,), dt, off).view(shape) for r in range(self.world)]
 
     def _global_rank(self, r: int) -> int:
         return r if self.group is None else dist.get_global_rank(self.group, r)
+
+    @torch.no_grad()
+    def step_peer(self, lr: float = 0.02, momentum: float = 0.95, nesterov: bool = True,
+                  weight_decay: float = 0.0) -> None:
+        """One step of the "peer" mode: every rank has written its gradients
+        into ``self.grads`` on its current stream.  Enqueues only."""
+        from . import dmuon_muon_step_batched_reduce
+        if self.grad_exchange != "peer":
+            raise RuntimeError("step_peer needs grad_exchange='peer'")
+        # Stream-ordered barrier: a collective completes only once every rank's
+        # stream has reached it, i.e. once every rank's gradients are written.
+        flag = torch.zeros(1, device=self.params[0].device)
+        dist.all_reduce(flag, group=self.group)
+        bcast = []
+        for r, c in self.schedule:
+            idx = self.chunks[r][c]
+            if r == self.rank:
+                dmuon_muon_step_batched_reduce(
+                    [self.params[i] for i in idx],
+                    [[self._peer[i][q] for i in idx] for q in range(self.world)],
+                    [self.bufs[i] for i in idx], lr=lr, momentum=momentum, nesterov=nesterov,
+                    weight_decay=weight_decay, ns_steps=self.ns_steps)
+            for i in idx:
+                bcast.append(dist.broadcast(self.params[i], src=self._global_rank(r), group=self.group,
+                                            async_op=True))
+        for w in bcast:
+            w.wait()
 
     @torch.no_grad()
     def step(self, grads: Sequence[Optional[torch.Tensor]], lr: float = 0.02,

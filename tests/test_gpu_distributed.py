@@ -42,3 +42,30 @@ def test_single_rank_nccl_matches_direct_step(cuda_lib):
             assert torch.equal(opt.bufs[i], bufs[i])
     finally:
         dist.destroy_process_group()
+
+
+def test_single_rank_peer_mode_matches_direct_step(cuda_lib):
+    """Gradients in symmetric memory, read by the owner's fused step: with one
+    rank the result equals a direct batched step bit for bit."""
+    dm = cuda_lib
+    dev = torch.device("cuda:0")
+    gen = torch.Generator(device=dev).manual_seed(4)
+    shapes = [(512, 1536), (1536, 512), (256, 256), (130, 72)]
+    pa = [(torch.randn(s, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for s in shapes]
+    pb = [p.clone() for p in pa]
+    grads = [(torch.randn(s, generator=gen, device=dev) * 1e-3).to(torch.bfloat16) for s in shapes]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        opt = dmd.OwnerPartitionedMuon(pa, grad_exchange="peer")
+        for g, view in zip(grads, opt.grads):
+            view.copy_(g)
+        opt.step_peer(lr=0.02, weight_decay=0.01)
+        bufs = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+        dm.dmuon_muon_step_batched(pb, grads, bufs, lr=0.02, weight_decay=0.01)
+        torch.cuda.synchronize()
+        for a, b in zip(pa, pb):
+            assert torch.equal(a, b)
+        for i in range(len(shapes)):
+            assert torch.equal(opt.bufs[i], bufs[i])
+    finally:
+        dist.destroy_process_group()
