@@ -768,7 +768,19 @@ __device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool ve
     return;
   }
   load8_from(md.Gr[0], md.g_bf16, idx, vec, valid, g);
-  for (int r = 1; r < md.world; ++r) {
+  int r = 1;
+  // Four ranks' loads in flight at once; the sum stays in rank order.
+  for (; r + 3 < md.world; r += 4) {
+    float h0[8], h1[8], h2[8], h3[8];
+    load8_from(md.Gr[r], md.g_bf16, idx, vec, valid, h0);
+    load8_from(md.Gr[r + 1], md.g_bf16, idx, vec, valid, h1);
+    load8_from(md.Gr[r + 2], md.g_bf16, idx, vec, valid, h2);
+    load8_from(md.Gr[r + 3], md.g_bf16, idx, vec, valid, h3);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      g[e] = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(g[e], h0[e]), h1[e]), h2[e]), h3[e]);
+  }
+  for (; r < md.world; ++r) {
     float h[8];
     load8_from(md.Gr[r], md.g_bf16, idx, vec, valid, h);
 #pragma unroll
