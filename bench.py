@@ -37,11 +37,11 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage per full
 # Llama-8B launch: the one-layer ncu capture (--workload llama8b_layer) scaled by 32 identical
 # layers; valid only for the kernel source it was measured on.
-# ncu capture of the GEMM stage on one Llama-8B layer (1.153 GB of DRAM traffic for
+# ncu capture of the GEMM stage on one Llama-8B layer (1.254 GB of DRAM traffic for
 # 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so
 # its traffic is this ratio times the useful FLOPs of that launch.
-PROFILED_TRAFFIC = {"kernels_sha256_prefix": "91573e6f083f6d4f", "workload": "llama8b",
-                    "gemm_bytes_per_useful_flop": 1.1529e9 / 1.735e12}
+PROFILED_TRAFFIC = {"kernels_sha256_prefix": "2f4971a39e1b5031", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 1.2537e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

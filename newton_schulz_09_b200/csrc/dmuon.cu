@@ -241,6 +241,7 @@ Layout make_layout(const std::vector<MatIn>& in, int steps) {
 // ------------------------------------------------------------------ plans
 struct GroupPlan {
   int dtype;
+  bool ranks = false;     // some matrix averages several ranks' gradients
   int nmat;
   int first;              // first MatDesc index of the group
   int64_t ptiles;
@@ -316,8 +317,10 @@ int device_setup(int dev) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
   }
-  const void* pk[] = {reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16>),
-                      reinterpret_cast<const void*>(&prologue_kernel<float>)};
+  const void* pk[] = {reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16, false>),
+                      reinterpret_cast<const void*>(&prologue_kernel<float, false>),
+                      reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16, true>),
+                      reinterpret_cast<const void*>(&prologue_kernel<float, true>)};
   for (const void* k : pk) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kProSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prologue smem)");
@@ -416,6 +419,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
                (x.buf == nullptr || aligned(x.buf, 16));
       for (const void* q : x.gr) d.vec4 = d.vec4 && aligned(q, 16);
       d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
+      if (d.world > 1) gp.ranks = true;
       d.Gr = nullptr;   // set once the plan's device memory exists
       d.ptiles_c = static_cast<int>(ml.ptiles_c);
       A.pp.push_back(A.pp.back() + ml.ptiles);
@@ -616,7 +620,8 @@ void launch_grad_norm(const Plan& P, const GroupPlan& g, const DeviceInfo& d, co
   const ElemParams ep = elem_params<E>(P, g, o);
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-  grad_norm_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+  if (g.ranks) grad_norm_kernel<E, true><<<pgrid, kPThreads, 0, st>>>(ep);
+  else grad_norm_kernel<E, false><<<pgrid, kPThreads, 0, st>>>(ep);
 }
 
 template <typename E>
@@ -628,7 +633,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-    prologue_kernel<E><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    else prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);

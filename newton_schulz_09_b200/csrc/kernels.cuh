@@ -685,8 +685,9 @@ static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes, "transpose tile must fit the
 // Stage 8 consecutive input elements (one thread's segment) into shared
 // memory with 16-byte asynchronous copies: the gradient at sg (2 or 4 bytes
 // an element), the momentum at sb.  Only whole, 16-byte aligned segments.
+template <bool kRanks>
 __device__ __forceinline__ void stage8(const MatDesc& md, int64_t idx, bool has_buf, uint8_t* sg, float* sb) {
-  if (md.world > 1) {
+  if (kRanks && md.world > 1) {
     // the mean over the ranks is read directly at use
   } else if (md.g_bf16) {
     cp_async16(sg, reinterpret_cast<const __nv_bfloat16*>(md.G) + idx);
@@ -700,9 +701,10 @@ __device__ __forceinline__ void stage8(const MatDesc& md, int64_t idx, bool has_
     cp_async16(sb + 4, md.buf + idx + 4);
   }
 }
+template <bool kRanks>
 __device__ __forceinline__ void unstage8(const MatDesc& md, bool has_buf, const uint8_t* sg, const float* sb,
                                          float (&g)[8], float (&b)[8]) {
-  if (md.world > 1) {
+  if (kRanks && md.world > 1) {
     // not staged: the caller reads the mean over the ranks
   } else if (md.g_bf16) {
     const uint4 u = *reinterpret_cast<const uint4*>(sg);
@@ -761,9 +763,12 @@ __device__ __forceinline__ void load8_from(const void* G, int g_bf16, int64_t id
 // 8 consecutive gradient elements.  With world > 1 the gradient is the
 // data-parallel mean, read straight from every rank's buffer (in a multi-GPU
 // job, peer memory mapped into this process): an fp32 sum in rank order,
-// then one division by the number of ranks.
+// then one division by the number of ranks.  Kernels instantiated with
+// kRanks = false (every launch without such matrices) compile this out and
+// keep their register budget.
+template <bool kRanks>
 __device__ __forceinline__ void load8_in(const MatDesc& md, int64_t idx, bool vec, int valid, float (&g)[8]) {
-  if (md.world <= 1) {
+  if (!kRanks || md.world <= 1) {
     load8_from(md.G, md.g_bf16, idx, vec, valid, g);
     return;
   }
@@ -854,7 +859,7 @@ __device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, flo
   }
 }
 
-template <typename E>
+template <typename E, bool kRanks>
 __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDesc& md, int64_t item,
                                                uint8_t* stage) {
   const int tid = threadIdx.x;
@@ -874,7 +879,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
   for (int j = 0; j < 4; ++j) {
     const int le = (j * kPThreads + tid) * 8;
     const int64_t e = e_begin + le;
-    if (md.vec4 && e + 8 <= numel) stage8(md, e, has_buf, stage + le * gb, sbuf + le);
+    if (md.vec4 && e + 8 <= numel) stage8<kRanks>(md, e, has_buf, stage + le * gb, sbuf + le);
   }
   cp_async_commit();
   cp_async_wait_all();
@@ -888,10 +893,10 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
     const bool vec = md.vec4 && valid == 8;
     float g[8], b[8], M[8];
     if (vec) {
-      unstage8(md, has_buf, stage + le * gb, sbuf + le, g, b);
-      if (md.world > 1) load8_in(md, e, true, 8, g);
+      unstage8<kRanks>(md, has_buf, stage + le * gb, sbuf + le, g, b);
+      if (kRanks && md.world > 1) load8_in<kRanks>(md, e, true, 8, g);
     } else {
-      load8_in(md, e, vec, valid, g);
+      load8_in<kRanks>(md, e, vec, valid, g);
       if (has_buf) load8_f32(md.buf + e, vec, valid, b);
     }
     momentum8(p, has_buf, g, b, M);
@@ -922,7 +927,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
   return ss;
 }
 
-template <typename E>
+template <typename E, bool kRanks>
 __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const MatDesc& md, int64_t item,
                                                      uint8_t* stage) {
   const int tid = threadIdx.x;
@@ -942,7 +947,7 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
     const int64_t idx = r * cols + c;
     const int slot = (i * kPThreads + tid) * 8;
     if (md.vec4 && r < rows && c + 8 <= cols && (idx & 7) == 0)
-      stage8(md, idx, has_buf, stage + slot * gb, sbuf + slot);
+      stage8<kRanks>(md, idx, has_buf, stage + slot * gb, sbuf + slot);
   }
   cp_async_commit();
   cp_async_wait_all();
@@ -959,10 +964,10 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
     const bool vec = md.vec4 && valid == 8 && ((idx & 7) == 0);
     if (vec) {
       const int slot = (i * kPThreads + tid) * 8;
-      unstage8(md, has_buf, stage + slot * gb, sbuf + slot, g, b);
-      if (md.world > 1) load8_in(md, idx, true, 8, g);
+      unstage8<kRanks>(md, has_buf, stage + slot * gb, sbuf + slot, g, b);
+      if (kRanks && md.world > 1) load8_in<kRanks>(md, idx, true, 8, g);
     } else if (valid > 0) {
-      load8_in(md, idx, vec, valid, g);
+      load8_in<kRanks>(md, idx, vec, valid, g);
       if (has_buf) load8_f32(md.buf + idx, vec, valid, b);
     }
     momentum8(p, has_buf, g, b, Mv[i]);
@@ -1007,7 +1012,7 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   return ss;
 }
 
-template <typename E>
+template <typename E, bool kRanks = false>
 __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
   extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
   __shared__ float red[kPThreads / 32];
@@ -1019,7 +1024,8 @@ __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_consta
     while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
     const MatDesc& md = p.mats[mi];
     const int64_t item = t - __ldg(p.ptile_prefix + mi);
-    float ss = md.T ? prologue_transposed<E>(p, md, item, pro_stage) : prologue_flat<E>(p, md, item, pro_stage);
+    float ss = md.T ? prologue_transposed<E, kRanks>(p, md, item, pro_stage)
+                    : prologue_flat<E, kRanks>(p, md, item, pro_stage);
     // Fixed-order block reduction of the item's sum of squares.
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -1037,7 +1043,7 @@ __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_consta
 
 // Sum of squares of the gradients (fp64 accumulation), one partial per
 // prologue work item (the items cover every gradient element exactly once).
-template <typename E>
+template <typename E, bool kRanks = false>
 __global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_constant__ ElemParams p) {
   __shared__ double red[kPThreads / 32];
   const int tid = threadIdx.x;
@@ -1058,7 +1064,7 @@ __global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_const
         if (e >= numel) break;
         const int valid = static_cast<int>(numel - e < 8 ? numel - e : 8);
         float g[8];
-        load8_in(md, e, md.vec4 && valid == 8, valid, g);
+        load8_in<kRanks>(md, e, md.vec4 && valid == 8, valid, g);
 #pragma unroll
         for (int k = 0; k < 8; ++k) ss += static_cast<double>(g[k]) * g[k];
       }
@@ -1072,7 +1078,7 @@ __global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_const
         const int valid = static_cast<int>(cols - c < 8 ? cols - c : 8);
         const int64_t idx = r * cols + c;
         float g[8];
-        load8_in(md, idx, md.vec4 && valid == 8 && ((idx & 7) == 0), valid, g);
+        load8_in<kRanks>(md, idx, md.vec4 && valid == 8 && ((idx & 7) == 0), valid, g);
 #pragma unroll
         for (int k = 0; k < 8; ++k) ss += static_cast<double>(g[k]) * g[k];
       }
