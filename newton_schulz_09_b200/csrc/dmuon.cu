@@ -2,11 +2,13 @@
 // scratch layout, TMA descriptors and the C ABI declared in include/dmuon.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <list>
 #include <map>
@@ -282,6 +284,15 @@ struct Arena {
 };
 std::map<std::pair<int, cudaStream_t>, Arena> g_arenas;
 
+// DMUON_LOG set to anything but "0": one stderr line per launch plan built.
+bool log_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("DMUON_LOG");
+    return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+  }();
+  return on;
+}
+
 uint64_t fnv1a(const uint8_t* p, size_t n) {
   uint64_t h = 1469598103934665603ull;
   for (size_t i = 0; i < n; ++i) { h ^= p[i]; h *= 1099511628211ull; }
@@ -533,6 +544,14 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   P->clip = reinterpret_cast<float*>(wsb + L.clip);
   P->d_mats = reinterpret_cast<const MatDesc*>(base + o_desc);
   P->d_maps = reinterpret_cast<const MatMaps*>(base + o_maps);
+  if (log_enabled()) {
+    int64_t syrk = 0, gemm = 0, items = 0;
+    for (const GroupPlan& gp : P->groups) { syrk += gp.syrk_tiles; gemm += gp.gemm_tiles; items += gp.ptiles; }
+    std::fprintf(stderr, "dmuon: plan on device %d: %d matrices in %zu dtype groups, %lld prologue items, "
+                 "%lld SYRK and %lld GEMM tiles per stage, scratch %zu bytes, plan %zu bytes\n", dev, nmat,
+                 P->groups.size(), static_cast<long long>(items), static_cast<long long>(syrk),
+                 static_cast<long long>(gemm), L.bytes, img.size());
+  }
   g_plans.emplace_front(std::move(P));
   Plan* plan = g_plans.front().get();
   while (g_plans.size() > kMaxPlans) {
@@ -570,12 +589,18 @@ cudaEvent_t pool_event() {
   return e;
 }
 
+// NVTX range names of the kernel kinds (a timeline tool shows every launch;
+// without one attached the calls cost next to nothing).
+const char* const kKindNames[DMUON_KERNEL_KINDS] = {"dmuon prologue", "dmuon finalize", "dmuon syrk",
+                                                    "dmuon gemm", "dmuon apply", "dmuon adamw"};
+
 struct LaunchScope {
   cudaStream_t st;
   int kind;
   cudaEvent_t a = nullptr;
   LaunchScope(cudaStream_t s, int k) : st(s), kind(k) {
     ++g_launches;
+    nvtxRangePushA(kKindNames[k]);
     if (g_timing) {
       a = pool_event();
       cudaEventRecord(a, st);
@@ -587,6 +612,7 @@ struct LaunchScope {
       cudaEventRecord(b, st);
       g_brackets.push_back(Bracket{a, b, kind});
     }
+    nvtxRangePop();
   }
 };
 
