@@ -168,6 +168,23 @@ class OwnerPartitionedMuon:
                 self.grads[i] = buf[off:off + n].view(shape)
                 self._peer[i] = [hdl.get_buffer(r, (n,), dt, off).view(shape) for r in range(self.world)]
 
+    def state_dict(self) -> dict:
+        """This rank's optimizer state: the momentum buffers of the matrices
+        it owns (by parameter index) and the partition they belong to."""
+        return {"owner": list(self.owner), "ns_steps": self.ns_steps,
+                "bufs": {i: b.detach().clone() for i, b in self.bufs.items()}}
+
+    def load_state_dict(self, state: dict) -> None:
+        """Restores buffers saved by ``state_dict`` on the same rank of a job
+        with the same parameters and number of ranks (so the same partition)."""
+        if list(state["owner"]) != self.owner:
+            raise ValueError("the saved state belongs to another partition of the parameters")
+        if set(state["bufs"]) != set(self.bufs):
+            raise ValueError("the saved buffers are not this rank's")
+        for i, b in state["bufs"].items():
+            self.bufs[i].copy_(b)
+        self.ns_steps = int(state["ns_steps"])
+
     def _global_rank(self, r: int) -> int:
         return r if self.group is None else dist.get_global_rank(self.group, r)
 

@@ -60,6 +60,30 @@ def _worker(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
+def _resume_worker(rank, world, port, out_dir):
+    """Two steps in one go, or one step, a checkpoint, a fresh optimizer
+    restored from it, and the second step: the results must be identical."""
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        straight = _params()
+        opt = dmd.OwnerPartitionedMuon(straight, ns_steps=3, step_fn=oracle_step_fn)
+        for step in range(2):
+            opt.step(_grads(rank, step), **HP)
+        resumed = _params()
+        opt1 = dmd.OwnerPartitionedMuon(resumed, ns_steps=3, step_fn=oracle_step_fn)
+        opt1.step(_grads(rank, 0), **HP)
+        saved = opt1.state_dict()
+        opt2 = dmd.OwnerPartitionedMuon(resumed, ns_steps=3, step_fn=oracle_step_fn)
+        opt2.load_state_dict(saved)
+        opt2.step(_grads(rank, 1), **HP)
+        same = all(torch.equal(a, b) for a, b in zip(straight, resumed))
+        same = same and all(torch.equal(opt.bufs[i], opt2.bufs[i]) for i in opt.bufs)
+        torch.save({"same": same}, os.path.join(out_dir, f"resume{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -127,3 +151,24 @@ def test_ranks_match_one_step_on_averaged_gradients(tmp_path, world):
         assert np.array_equal(got, W[i]), i
         owner = res[0]["owner"][i]
         assert np.array_equal(res[owner]["bufs"][i].numpy(), bufs[i])
+
+
+def test_checkpoint_and_resume(tmp_path):
+    world = 2
+    mp.start_processes(_resume_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    for r in range(world):
+        assert torch.load(tmp_path / f"resume{r}.pt")["same"]
+
+
+def test_load_state_dict_checks_the_partition():
+    opt = dmd.OwnerPartitionedMuon.__new__(dmd.OwnerPartitionedMuon)
+    opt.owner = [0, 1, 0]
+    opt.bufs = {0: torch.zeros(2), 2: torch.zeros(3)}
+    opt.ns_steps = 5
+    with pytest.raises(ValueError):
+        opt.load_state_dict({"owner": [1, 0, 0], "ns_steps": 5, "bufs": {}})
+    with pytest.raises(ValueError):
+        opt.load_state_dict({"owner": [0, 1, 0], "ns_steps": 5, "bufs": {0: torch.ones(2)}})
+    opt.load_state_dict({"owner": [0, 1, 0], "ns_steps": 3, "bufs": {0: torch.ones(2), 2: torch.ones(3)}})
+    assert torch.equal(opt.bufs[2], torch.ones(3)) and opt.ns_steps == 3
