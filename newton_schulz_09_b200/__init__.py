@@ -505,3 +505,8 @@ def dmuon_adamw_step_batched(params, grads, exp_avgs, exp_avg_sqs, lr: float = 1
         _check(lib.dmuon_adamw_step_batched(ctypes.cast(P, pp), ctypes.cast(G, pp), ctypes.cast(M, pp),
                                             ctypes.cast(V, pp), D, n, lr, betas[0], betas[1], eps,
                                             weight_decay, step, _stream(dev)))
+
+
+from .optim import Muon  # noqa: E402  (the optimizer wraps the functions above)
+
+__all__.append("Muon")
