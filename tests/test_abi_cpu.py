@@ -212,3 +212,20 @@ def test_partition_rejects_bad_arguments(lib):
     assert lib.dmuon_debug_partition(_shapes((4, 4)), 1, 2, B, 4) == -1
     assert lib.dmuon_debug_partition(_shapes((0, 4)), 1, 0, B, 4) == -1
     assert lib.dmuon_debug_partition(_shapes((4, 4)), 1, 0, B, 1) == -1
+
+
+def test_reduce_step_rejects_bad_arguments_on_the_host(lib):
+    o = dm.DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    P, B = _ptrs(0x10000), _ptrs(0x30000)
+    S = _shapes((4, 4))
+    call = lambda grads, world, n=1, opts=ctypes.byref(o): lib.dmuon_muon_step_batched_reduce(
+        P, grads, B, S, n, world, opts, None, 0, None)
+    assert call(_ptrs(0x20000), 1, n=0) == 0                       # nothing to do
+    assert call(_ptrs(0x20000), 0) == -1 and "world" in dm.dmuon_last_error()
+    assert call(_ptrs(*([0x20000] * 65)), 65) == -1
+    assert call(_ptrs(0x20000), 1, opts=None) == -1
+    assert call(_ptrs(0x20000, None), 2) == -1 and "rank 1" in dm.dmuon_last_error()
+    assert call(_ptrs(None, 0x20000), 2) == -1
+    assert call(_ptrs(0x20000, 0x20001), 2) == -1 and "misaligned" in dm.dmuon_last_error()
+    assert call(_ptrs(None, None), 2) == 0                         # no gradient on any rank: skipped
