@@ -20,7 +20,7 @@ Sources (page title, section):
   input is ``grad + momentum * buf``; ``weight_decay`` is a Muon parameter
   (section "第 4 步：创建优化器") without a stated formula.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * Nesterov uses the buffer *after* its update (the update is the first
   statement of the step on the blog's Vanilla Muon).
