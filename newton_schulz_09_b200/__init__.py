@@ -150,6 +150,18 @@ def _cuda_matrix(t: torch.Tensor, what: str) -> None:
         raise ValueError(f"{what} must be contiguous (row-major)")
 
 
+def _workspace(workspace: Optional[torch.Tensor], device: torch.device):
+    """(address, bytes) of a caller's scratch tensor, (None, 0) without one.
+    The scratch must be contiguous device memory on the matrices' device: a
+    host tensor's address would be written by the kernels."""
+    if workspace is None:
+        return None, 0
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+            or workspace.device != device or not workspace.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous CUDA tensor on {device}")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
 # ---------------------------------------------------------------- orthogonalise
 def dmuon_ns_workspace_bytes(m: int, n: int, dtype: torch.dtype = torch.bfloat16) -> int:
     return int(load_library().dmuon_ns_workspace_bytes(m, n, _dtype_code(dtype)))
@@ -177,10 +189,10 @@ def dmuon_ns_orthogonalize_ex(X: torch.Tensor, steps: int = 5,
     need = int(lib.dmuon_ns_workspace_bytes(X.shape[0], X.shape[1], dt))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_ptr, ws_bytes = _workspace(workspace, X.device)
     with torch.cuda.device(X.device):
         _check(lib.dmuon_ns_orthogonalize_ex(X.data_ptr(), X.shape[0], X.shape[1], steps, dt,
-                                             workspace.data_ptr(), workspace.numel(),
-                                             _stream(X.device)))
+                                             ws_ptr, ws_bytes, _stream(X.device)))
     return X
 
 
@@ -274,12 +286,10 @@ def dmuon_muon_step_batched_opts(params, grads, bufs, lr: float = 0.02, momentum
     o.max_grad_norm = max_grad_norm
     if grad_norm_out is not None:
         if (grad_norm_out.dtype != torch.float32 or not grad_norm_out.is_cuda
-                or grad_norm_out.numel() < 1):
+                or grad_norm_out.device != b.device or grad_norm_out.numel() < 1):
             raise ValueError("grad_norm_out must be a CUDA fp32 tensor with one element")
         o.grad_norm_out = grad_norm_out.data_ptr()
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    ws_ptr, ws_bytes = _workspace(workspace, b.device)
     with torch.cuda.device(b.device):
         _check(lib.dmuon_muon_step_batched_opts(*b.args(), ctypes.byref(o), ws_ptr, ws_bytes,
                                                 _stream(b.device)))
@@ -323,9 +333,7 @@ def dmuon_muon_step_batched_reduce(params, rank_grads, bufs, lr: float = 0.02, m
     o.ns_a, o.ns_b = ns_coefficients
     o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
     o.max_grad_norm = max_grad_norm
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    ws_ptr, ws_bytes = _workspace(workspace, b.device)
     P, _, B, S, cnt = b.args()
     pp = ctypes.POINTER(ctypes.c_void_p)
     with torch.cuda.device(b.device):
@@ -374,9 +382,7 @@ def dmuon_muon_step_batched_host(params, grads, bufs, host_grads, host_params=No
     o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
     o.ns_a, o.ns_b = ns_coefficients
     o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    ws_ptr, ws_bytes = _workspace(workspace, b.device)
     P, G, B, S, cnt = b.args()
     pp = ctypes.POINTER(ctypes.c_void_p)
     with torch.cuda.device(b.device):
@@ -398,10 +404,11 @@ def dmuon_muon_step_batched_ex(params, grads, bufs, lr: float = 0.02, momentum: 
     need = dmuon_workspace_bytes(params, ns_steps, grads)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=b.device)
+    ws_ptr, ws_bytes = _workspace(workspace, b.device)
     with torch.cuda.device(b.device):
         _check(lib.dmuon_muon_step_batched_ex(*b.args(), lr, momentum, 1 if nesterov else 0,
-                                              weight_decay, ns_steps, workspace.data_ptr(),
-                                              workspace.numel(), _stream(b.device)))
+                                              weight_decay, ns_steps, ws_ptr, ws_bytes,
+                                              _stream(b.device)))
 
 
 # ---------------------------------------------------------------- misc

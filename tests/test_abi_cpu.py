@@ -229,3 +229,15 @@ def test_reduce_step_rejects_bad_arguments_on_the_host(lib):
     assert call(_ptrs(None, 0x20000), 2) == -1
     assert call(_ptrs(0x20000, 0x20001), 2) == -1 and "misaligned" in dm.dmuon_last_error()
     assert call(_ptrs(None, None), 2) == 0                         # no gradient on any rank: skipped
+
+
+def test_caller_workspace_must_be_device_memory_of_the_matrices_device():
+    """A host tensor as scratch would hand the kernels a host address: the
+    binding refuses it, and counts a workspace's size in bytes, not elements."""
+    import torch
+    cuda0 = torch.device("cuda", 0)
+    assert dm._workspace(None, cuda0) == (None, 0)
+    with pytest.raises(ValueError, match="workspace"):
+        dm._workspace(torch.empty(4096, dtype=torch.uint8), cuda0)
+    with pytest.raises(ValueError, match="workspace"):
+        dm._workspace("not a tensor", cuda0)

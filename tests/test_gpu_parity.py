@@ -204,7 +204,8 @@ def test_ex_entry_with_torch_workspace_matches_arena(cuda_lib):
     bs = [torch.zeros(s, dtype=torch.float32, device=DEV) for s in shapes]
     p2, b2 = [p.clone() for p in ps], [b.clone() for b in bs]
     dm.dmuon_muon_step_batched(ps, gs, bs)
-    ws = torch.empty(dm.dmuon_workspace_bytes(p2), dtype=torch.uint8, device=DEV)
+    # any dtype serves as scratch: its size counts in bytes
+    ws = torch.empty((dm.dmuon_workspace_bytes(p2) + 3) // 4, dtype=torch.float32, device=DEV)
     dm.dmuon_muon_step_batched_ex(p2, gs, b2, workspace=ws)
     torch.cuda.synchronize()
     for a, b in zip(ps, p2):
