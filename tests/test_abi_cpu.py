@@ -241,3 +241,24 @@ def test_caller_workspace_must_be_device_memory_of_the_matrices_device():
         dm._workspace(torch.empty(4096, dtype=torch.uint8), cuda0)
     with pytest.raises(ValueError, match="workspace"):
         dm._workspace("not a tensor", cuda0)
+
+
+def test_header_serves_a_plain_c99_program(lib):
+    """include/dmuon.h is plain C: a C99 program compiled with -pedantic
+    -Werror against it links to the library and gets the documented host-side
+    answers (tests/c_consumer.c)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "_build", "c_consumer")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "c_consumer")
+    libdir = os.path.dirname(dm.library_path())
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_consumer.c"),
+                    "-o", exe, "-L", libdir, "-ldmuon", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "ok"
