@@ -56,6 +56,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-adamw", action="store_true")
+    ap.add_argument("--adamw-only", type=int, default=0, metavar="ROWS",
+                    help="time only the AdamW leg, with embedding and head of ROWS x 4096 "
+                         "(128256 for Llama-8B; smaller for a profiler capture)")
     return ap.parse_args()
 
 
@@ -250,13 +253,13 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- ours
-def measure_adamw(dm, dev, stream, world, peaks, steps):
+def measure_adamw(dm, dev, stream, world, peaks, steps, rows=128256):
     """AdamW over the Llama-8B parameters that are not 2-D projections: token
-    embedding and LM head (128256 x 4096 each) and 65 norm weights (4096),
-    bf16 parameters and gradients, fp32 moments; 22 algorithmic bytes per
-    element (p read+write 4, g 2, m and v read+write 16)."""
+    embedding and LM head (``rows`` = 128256 x 4096 each) and 65 norm weights
+    (4096), bf16 parameters and gradients, fp32 moments; 22 algorithmic bytes
+    per element (p read+write 4, g 2, m and v read+write 16)."""
     import torch
-    shapes = [(128256 * 4096,), (128256 * 4096,)] + [(4096,)] * 65
+    shapes = [(rows * 4096,), (rows * 4096,)] + [(4096,)] * 65
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
     ps = [(torch.randn(s, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for s in shapes]
@@ -538,8 +541,36 @@ def run_torch(args):
     return 0
 
 
+def run_adamw_only(args):
+    """The AdamW leg alone (one GPU): its own JSON line, GB/s of algorithmic
+    traffic against the measured copy bandwidth."""
+    import torch
+    import newton_schulz_09_b200 as dm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dm.load_library()
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    a = measure_adamw(dm, dev, torch.cuda.current_stream(dev), 1, peaks, args.steps, rows=args.adamw_only)
+    clocks = sampler.stop()
+    print(json.dumps({
+        "metric": "AdamW step GB/s (Llama-8B embedding, head and norms)", "value": a["achieved"],
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": 3, "ms_per_step": a["ms_per_step"],
+        "higher_is_better": True, "dtype": "f32", "data": "synthetic", "clocks": clocks,
+        "config": {"workload": f"adamw {args.adamw_only}x4096 x2 + 65x4096", "elements": a["elements"],
+                   "bytes_per_element": 22, "l2": "inputs larger than L2" if 22 * a["elements"] > 126e6
+                   else "inputs within L2"},
+        "roofline": {"bound": "hbm", "achieved": a["achieved"], "peak": a["peak"], "unit": "GB/s",
+                     "frac": a["frac"], "peak_source": f"{peak_src} hbm_gbs"}}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.adamw_only > 0:
+        return run_adamw_only(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.impl == "torch":

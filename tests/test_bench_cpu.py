@@ -42,3 +42,9 @@ def test_product_arm_refuses_to_run_without_a_gpu():
     r = _bench(["--steps", "1", "--warmup", "3", "--workload", "tinymlp"], timeout=300)
     assert r.returncode != 0
     assert "{" not in r.stdout          # no JSON line: no CPU fallback number
+
+
+def test_adamw_only_mode_refuses_to_run_without_a_gpu():
+    r = _bench(["--adamw-only", "16", "--steps", "1"], timeout=300)
+    assert r.returncode != 0
+    assert "{" not in r.stdout
