@@ -1,4 +1,7 @@
 import os
+import pathlib
+import re
+import shutil
 import sys
 
 import pytest
@@ -22,3 +25,15 @@ def cuda_lib():
     import newton_schulz_09_b200 as dm
     dm.load_library()
     return dm
+
+
+@pytest.fixture
+def scratch_dir(request) -> pathlib.Path:
+    """An empty per-test folder inside the repository's git-ignored build
+    folder (tests keep their files inside the working tree)."""
+    name = re.sub(r"[^A-Za-z0-9_.-]+", "_", request.node.nodeid)[-120:]
+    path = pathlib.Path(ROOT) / "_build" / "test_scratch" / name
+    if path.exists():
+        shutil.rmtree(path)
+    path.mkdir(parents=True)
+    return path

@@ -125,10 +125,10 @@ def test_owner_chunks_and_global_schedule():
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_ranks_match_one_step_on_averaged_gradients(tmp_path, world):
-    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+def test_ranks_match_one_step_on_averaged_gradients(scratch_dir, world):
+    mp.start_processes(_worker, args=(world, _free_port(), str(scratch_dir)), nprocs=world,
                        start_method="spawn", join=True)
-    res = [torch.load(tmp_path / f"rank{r}.pt") for r in range(world)]
+    res = [torch.load(scratch_dir / f"rank{r}.pt") for r in range(world)]
     # every rank holds identical weights after the broadcasts
     for r in range(1, world):
         for a, b in zip(res[0]["params"], res[r]["params"]):
@@ -153,12 +153,12 @@ def test_ranks_match_one_step_on_averaged_gradients(tmp_path, world):
         assert np.array_equal(res[owner]["bufs"][i].numpy(), bufs[i])
 
 
-def test_checkpoint_and_resume(tmp_path):
+def test_checkpoint_and_resume(scratch_dir):
     world = 2
-    mp.start_processes(_resume_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+    mp.start_processes(_resume_worker, args=(world, _free_port(), str(scratch_dir)), nprocs=world,
                        start_method="spawn", join=True)
     for r in range(world):
-        assert torch.load(tmp_path / f"resume{r}.pt")["same"]
+        assert torch.load(scratch_dir / f"resume{r}.pt")["same"]
 
 
 def test_load_state_dict_checks_the_partition():
