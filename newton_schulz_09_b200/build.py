@@ -53,7 +53,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    # the compiler's intermediate files stay in the working tree too
+    tmp = os.path.join(ROOT, "_build", "nvcc_tmp")
+    os.makedirs(tmp, exist_ok=True)
+    subprocess.run(cmd, check=True, env=dict(os.environ, TMPDIR=tmp))
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -258,7 +258,8 @@ def test_header_serves_a_plain_c99_program(lib):
     libdir = os.path.dirname(dm.library_path())
     subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
                     "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_consumer.c"),
-                    "-o", exe, "-L", libdir, "-ldmuon", f"-Wl,-rpath,{libdir}"], check=True)
+                    "-o", exe, "-L", libdir, "-ldmuon", f"-Wl,-rpath,{libdir}"], check=True,
+                   env=dict(os.environ, TMPDIR=out_dir))
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "ok"
