@@ -263,3 +263,19 @@ def test_header_serves_a_plain_c99_program(lib):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "ok"
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without the built library every entry point raises: there is no
+    Python or CPU path to fall back to."""
+    import torch
+    monkeypatch.setattr(dm, "_lib", None)
+    monkeypatch.setattr(dm, "_LIB_PATH", os.path.join(ROOT, "_build", "no_such_library.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        dm.load_library()
+    with pytest.raises(RuntimeError, match="missing"):
+        dm.dmuon_backend_string()
+    with pytest.raises(RuntimeError, match="missing"):
+        dm.dmuon_muon_step_batched([], [], [])
+    with pytest.raises(RuntimeError, match="missing"):
+        dm.dmuon_ns_orthogonalize(torch.zeros(4, 4, dtype=torch.bfloat16))
