@@ -403,7 +403,55 @@ def pin_rank_mean(o) -> None:
         assert got[k] == exact_f32_round(Fraction(int(S[k]), 3)), (k, got[k])
 
 
+def pin_relative_frobenius(o) -> None:
+    """||a - b||_F / ||b||_F against values worked out by hand:
+    * b = [[3, 4]] (norm 5), a = b + 0.5 e_11: 0.5 / 5 = 0.1 (the
+      denominator is b's norm, not a's, which is sqrt(28.25));
+    * b = [[1, 2], [2, 4]] (norm 5), a - b = diag(0.3, 0.4): the difference
+      norm adds every element, sqrt(0.09 + 0.16) = 0.5, so again 0.1 (the
+      largest element alone would give 0.08);
+    * both zero gives 0, a nonzero a against a zero b gives inf, a == b gives 0;
+    * scaling both arguments by the same c > 0 leaves the value unchanged."""
+    b = np.array([[3.0, 4.0]])
+    a = b + np.array([[0.5, 0.0]])
+    assert abs(o.relative_frobenius(a, b) - 0.1) <= 1e-16, o.relative_frobenius(a, b)
+    b2 = np.array([[1.0, 2.0], [2.0, 4.0]])
+    a2 = b2 + np.diag([0.3, 0.4])
+    assert abs(o.relative_frobenius(a2, b2) - 0.1) <= 1e-15, o.relative_frobenius(a2, b2)
+    assert abs(o.relative_frobenius(7.0 * a2, 7.0 * b2) - 0.1) <= 1e-15
+    assert o.relative_frobenius(np.zeros((2, 3)), np.zeros((2, 3))) == 0.0
+    assert o.relative_frobenius(np.ones((2, 3)), np.zeros((2, 3))) == float("inf")
+    assert o.relative_frobenius(b2, b2) == 0.0
+
+
+def pin_orthogonality_error(o, seed: int = 21) -> None:
+    """||X X^T - I||_F on the short side of X, against closed forms:
+    * hand-worked: [[1, 1]] gives |2 - 1| = 1; diag(2, 1) gives 3;
+      [[1, 1], [0, 1]] gives ||[[1, 1], [1, 0]]||_F = sqrt(3);
+    * c Q with orthonormal rows (m x n, m < n) and its transpose (tall) both
+      give sqrt(m) |c^2 - 1|: the tall one must use the m x m column Gram, the
+      n x n row Gram would add n - m to the squared value;
+    * a tall 96 x 40 random matrix gives sqrt(sum_i (sigma_i^2 - 1)^2) over
+      its 40 singular values from the hand-written Jacobi SVD."""
+    assert abs(o.orthogonality_error(np.array([[1.0, 1.0]])) - 1.0) <= 1e-15
+    assert abs(o.orthogonality_error(np.diag([2.0, 1.0])) - 3.0) <= 1e-15
+    assert abs(o.orthogonality_error(np.array([[1.0, 1.0], [0.0, 1.0]])) - math.sqrt(3.0)) <= 1e-15
+    rng = np.random.default_rng(seed)
+    for (m, n) in ((16, 40), (5, 64)):
+        Q = _semi_orthogonal(rng, m, n)
+        for c in (0.5, 1.0, 1.7):
+            want = math.sqrt(m) * abs(c * c - 1.0)
+            assert abs(o.orthogonality_error(c * Q) - want) <= 1e-12, (m, n, c)
+            assert abs(o.orthogonality_error((c * Q).T) - want) <= 1e-12, (m, n, c, "tall")
+    G = rng.standard_normal((96, 40))
+    _, sig, _ = jacobi_svd(G)
+    want = math.sqrt(float(np.sum((sig * sig - 1.0) ** 2)))
+    got = o.orthogonality_error(G)
+    assert abs(got - want) <= 1e-10 * want, (got, want)
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
-            pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean)
+            pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean,
+            pin_relative_frobenius, pin_orthogonality_error)

@@ -190,6 +190,41 @@ MUTANTS["rank_mean_reciprocal"] = dict(rank_mean=_rank_mean_variant("reciprocal"
 MUTANTS["clip_no_eps"] = dict(clip_coefficient=lambda grads, mx: (np.float32(min(1.0, float(np.float32(mx)) / np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))), float(np.sqrt(sum(float(np.sum(np.asarray(x, np.float64) ** 2)) for x in grads)))))
 
 
+def _ortho_variant(kind):
+    def f(X):
+        X = np.asarray(X, dtype=np.float64)
+        if kind != "row_gram_on_tall" and X.shape[0] > X.shape[1]:
+            X = X.T
+        R = X @ X.T
+        if kind != "no_identity":
+            R[np.diag_indices_from(R)] -= 1.0
+        sq = float(np.sum(R * R))
+        return sq if kind == "missing_sqrt" else float(np.sqrt(sq))
+    return f
+
+
+def _relfro_variant(kind):
+    def f(a, b):
+        a = np.asarray(a, dtype=np.float64)
+        b = np.asarray(b, dtype=np.float64)
+        d = a - b
+        num = float(np.max(np.abs(d))) if kind == "max_element" else float(np.sqrt(np.sum(d * d)))
+        den = float(np.sqrt(np.sum((a if kind == "denominator_a" else b) ** 2)))
+        if den == 0.0:
+            return 0.0 if num == 0.0 else float("inf")
+        r = num / den
+        return r * r if kind == "squared_ratio" else r
+    return f
+
+
+MUTANTS["orthogonality_row_gram_on_tall"] = dict(orthogonality_error=_ortho_variant("row_gram_on_tall"))
+MUTANTS["orthogonality_missing_sqrt"] = dict(orthogonality_error=_ortho_variant("missing_sqrt"))
+MUTANTS["orthogonality_without_identity"] = dict(orthogonality_error=_ortho_variant("no_identity"))
+MUTANTS["relative_frobenius_squared_ratio"] = dict(relative_frobenius=_relfro_variant("squared_ratio"))
+MUTANTS["relative_frobenius_denominator_a"] = dict(relative_frobenius=_relfro_variant("denominator_a"))
+MUTANTS["relative_frobenius_max_element"] = dict(relative_frobenius=_relfro_variant("max_element"))
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(name):
     m = _mutant(**MUTANTS[name])
