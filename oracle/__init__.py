@@ -10,6 +10,7 @@ from .muon_oracle import (  # noqa: F401
     NS_B,
     adamw_step,
     clip_coefficient,
+    clip_grad_norm_buckets,
     frobenius_normalize,
     lr_scale_factor,
     momentum_update,
@@ -22,4 +23,5 @@ from .muon_oracle import (  # noqa: F401
     rank_mean,
     orthogonality_error,
     relative_frobenius,
+    round_to_bf16,
 )

@@ -141,6 +141,49 @@ def clip_coefficient(grads, max_norm: float):
     return np.float32(c), norm
 
 
+def round_to_bf16(x32: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (8 significant bits, round to nearest,
+    ties to even), returned as the float32 values they widen to exactly.
+    bfloat16 is the upper half of the float32 bit pattern, so the rounding is
+    done on the integer bits; NaN stays NaN, values past the largest bfloat16
+    round to infinity."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    u = x32.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    r = ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)) << np.uint64(16)
+    out = r.astype(np.uint32).view(np.float32).copy()
+    nan = np.isnan(x32)
+    out[nan] = x32[nan]
+    return out
+
+
+def clip_grad_norm_buckets(segments, max_norms):
+    """Clipping of several gradient groups ("segments"), each with its own
+    norm and coefficient (training guide, "梯度裁剪", the fused
+    regular / Muon / AdamW clipping that keeps per-segment semantics).
+
+    ``segments[s]`` is a list of (values, is_bf16) pairs: the gradient values
+    as float32 (bfloat16 values widen exactly) and their storage type.  For
+    each segment, as for the Muon-only clip: ||g||_s is the 2-norm over all
+    of its gradients (fp64), c_s = fl32(min(1, max_norm_s / (||g||_s + 1e-6)))
+    with min(1, NaN) = 1, and every gradient becomes fl32(g * c_s), rounded to
+    bfloat16 for bfloat16 storage.  Returns (new segments as float32 arrays,
+    norms, coefficients)."""
+    if len(max_norms) != len(segments):
+        raise ValueError("one max_norm per segment")
+    out, norms, coefs = [], [], []
+    for seg, mx in zip(segments, max_norms):
+        c32, nrm = clip_coefficient([v for v, _ in seg], mx)
+        new = []
+        for v, is_bf16 in seg:
+            y = np.multiply(np.asarray(v, np.float32), c32, dtype=np.float32)
+            new.append(round_to_bf16(y) if is_bf16 else y)
+        out.append(new)
+        norms.append(nrm)
+        coefs.append(c32)
+    return out, norms, coefs
+
+
 def muon_step(W, g, buf, *, lr: float, momentum: float, nesterov: bool,
               weight_decay: float, ns_steps: int, ns_coeffs=(NS_A, NS_B),
               lr_scale: bool = False, grad_scale=None):

@@ -104,6 +104,27 @@ def exact_f32_round(x: Fraction) -> np.float32:
     return np.float32(best[1])
 
 
+def exact_bf16_round(x: Fraction) -> float:
+    """Round an exact rational in the normal range to the nearest bfloat16
+    (8 significant bits), ties to even, worked out on the rational itself."""
+    if x == 0:
+        return 0.0
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = math.floor(math.log2(a))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 7)
+    q = a / ulp                      # in [128, 256)
+    lo = math.floor(q)
+    rem = q - lo
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return float(sign * lo * ulp)
+
+
 # -------------------------------------------------------------------- pins
 def pin_scalar_closed_form(o) -> None:
     """A 1x1 input reduces to s0 = x / (|x| + 1e-7), s <- 1.5 s - 0.5 s^3."""
@@ -450,8 +471,82 @@ def pin_orthogonality_error(o, seed: int = 21) -> None:
     assert abs(got - want) <= 1e-10 * want, (got, want)
 
 
+def pin_round_to_bf16(o, seed: int = 22) -> None:
+    """float32 -> bfloat16 rounding against exact rational rounding to 8
+    significant bits: random values over many binades, the exact halfway
+    points between neighbours (ties to even, both parities), values that are
+    already bfloat16, signs, and overflow past the largest bfloat16."""
+    rng = np.random.default_rng(seed)
+    vals = (rng.standard_normal(400) * 10.0 ** rng.integers(-30, 30, 400)).astype(np.float32)
+    ties = []
+    for k in range(128, 140):
+        for e in (-3, 0, 5):
+            ties.append(np.float32((k + 0.5) * 2.0 ** (e - 7)))     # halfway, both parities of k
+            ties.append(np.float32(k * 2.0 ** (e - 7)))             # already bfloat16
+    vals = np.concatenate([vals, np.array(ties, np.float32), -np.array(ties, np.float32)])
+    got = o.round_to_bf16(vals)
+    for v, r in zip(vals, got):
+        want = exact_bf16_round(Fraction(float(v)))
+        assert float(r) == want, (float(v), float(r), want)
+    big = o.round_to_bf16(np.array([3.4e38, -3.4e38, 3.38e38], np.float32))
+    assert big[0] == np.inf and big[1] == -np.inf and np.isfinite(big[2])
+    assert np.isnan(o.round_to_bf16(np.array([np.nan], np.float32))[0])
+
+
+def pin_clip_buckets(o) -> None:
+    """Per-segment clipping: three segments of +-1/4 Hadamard rows with
+    exactly known norms, sqrt(4) = 2, sqrt(16) = 4 and sqrt(1) = 1, and
+    max_norm 1.5 for each.  Segment 0 is scaled by
+    c0 = fl32(1.5 / (2 + 1e-6)), segment 1 by c1 = fl32(1.5 / (4 + 1e-6)),
+    segment 2 is below its bound and stays bit for bit (c2 = 1).  One global
+    norm (sqrt(21)) would give every segment the same coefficient.  Every
+    element must equal the exact product g * c rounded once to float32 and,
+    for bfloat16 storage, once more to bfloat16."""
+    H = _hadamard(16) / 4.0
+    seg0 = [(H[:4].astype(np.float32), True)]                      # norm 2 (bf16)
+    seg1 = [(H[:10].astype(np.float32), False), (H[10:].astype(np.float32), True)]   # norm 4
+    seg2 = [(H[:1].astype(np.float32), True)]                      # norm 1: no clipping
+    out, norms, coefs = o.clip_grad_norm_buckets([seg0, seg1, seg2], [1.5, 1.5, 1.5])
+    assert [abs(n - w) <= 1e-15 for n, w in zip(norms, (2.0, 4.0, 1.0))] == [True] * 3, norms
+    for c, nrm in zip(coefs[:2], (2.0, 4.0)):
+        assert c == exact_f32_round(Fraction(1.5) / (Fraction(nrm) + Fraction(1e-6))), (c, nrm)
+    assert coefs[2] == np.float32(1.0)
+    for seg, new, c in zip((seg0, seg1, seg2), out, coefs):
+        for (v, is_bf16), y in zip(seg, new):
+            assert y.dtype == np.float32 and y.shape == v.shape
+            for a, b in zip(v.ravel(), y.ravel()):
+                prod = exact_f32_round(Fraction(float(a)) * Fraction(float(c)))
+                want = exact_bf16_round(Fraction(float(prod))) if is_bf16 else float(prod)
+                assert float(b) == want, (float(a), float(c), float(b), want)
+    # random values: bfloat16 ones built from integer significands, float32
+    # ones from a generator; the norm comes from the exact sum of squares and
+    # an integer square root with 100 fractional bits
+    rng = np.random.default_rng(23)
+    vb = (rng.integers(128, 256, (8, 8)) * 2.0 ** rng.integers(-12, -6, (8, 8))
+          * rng.choice([-1.0, 1.0], (8, 8))).astype(np.float32)
+    vf = (rng.standard_normal((5, 3)) * 0.01).astype(np.float32)
+    S = sum(Fraction(float(x)) ** 2 for x in np.concatenate([vb.ravel(), vf.ravel()]))
+    root = Fraction(math.isqrt(int(S * 2 ** 200)), 2 ** 100)
+    mx = 0.3 * float(root)
+    out3, norms3, coefs3 = o.clip_grad_norm_buckets([[(vb, True), (vf, False)]], [mx])
+    assert abs(norms3[0] - float(root)) <= 1e-15 * float(root)
+    c = coefs3[0]
+    assert c == exact_f32_round(Fraction(float(np.float32(mx))) / (root + Fraction(1e-6))), c
+    for (v, is_bf16), y in zip(((vb, True), (vf, False)), out3[0]):
+        for a, b in zip(v.ravel(), y.ravel()):
+            prod = exact_f32_round(Fraction(float(a)) * Fraction(float(c)))
+            want = exact_bf16_round(Fraction(float(prod))) if is_bf16 else float(prod)
+            assert float(b) == want, (float(a), float(c), float(b), want)
+    # a NaN norm leaves its segment unchanged; an empty segment has norm 0
+    nan_seg = [(np.array([1.0, np.nan], np.float32), False)]
+    out2, norms2, coefs2 = o.clip_grad_norm_buckets([nan_seg, []], [1.0, 1.0])
+    assert np.isnan(norms2[0]) and coefs2[0] == np.float32(1.0) and out2[0][0][0] == 1.0
+    assert norms2[1] == 0.0 and coefs2[1] == np.float32(1.0) and out2[1] == []
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
             pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean,
-            pin_relative_frobenius, pin_orthogonality_error)
+            pin_relative_frobenius, pin_orthogonality_error, pin_round_to_bf16,
+            pin_clip_buckets)

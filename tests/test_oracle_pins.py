@@ -225,6 +225,49 @@ MUTANTS["relative_frobenius_denominator_a"] = dict(relative_frobenius=_relfro_va
 MUTANTS["relative_frobenius_max_element"] = dict(relative_frobenius=_relfro_variant("max_element"))
 
 
+def _bf16_truncate(x32):
+    x32 = np.asarray(x32, dtype=np.float32)
+    u = x32.view(np.uint32) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).copy()
+
+
+def _clip_buckets_variant(kind):
+    def f(segments, max_norms):
+        if kind == "global_norm":
+            allv = [v for seg in segments for v, _ in seg]
+            c_all, n_all = muon_oracle.clip_coefficient(allv, max_norms[0])
+        out, norms, coefs = [], [], []
+        for seg, mx in zip(segments, max_norms):
+            if kind == "global_norm":
+                c32, nrm = c_all, n_all
+            else:
+                c32, nrm = muon_oracle.clip_coefficient([v for v, _ in seg], mx)
+            if kind == "no_clamp":
+                c32 = np.float32(float(np.float32(mx)) / (nrm + 1e-6))
+            new = []
+            for v, is_bf16 in seg:
+                if kind == "scale_in_bf16" and is_bf16:
+                    cb = muon_oracle.round_to_bf16(np.array([c32], np.float32))[0]
+                    y = muon_oracle.round_to_bf16(np.multiply(v, cb, dtype=np.float32))
+                else:
+                    y = np.multiply(np.asarray(v, np.float32), c32, dtype=np.float32)
+                    if is_bf16:
+                        y = _bf16_truncate(y) if kind == "bf16_truncate" else muon_oracle.round_to_bf16(y)
+                new.append(y)
+            out.append(new)
+            norms.append(nrm)
+            coefs.append(c32)
+        return out, norms, coefs
+    return f
+
+
+MUTANTS["clip_buckets_global_norm"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("global_norm"))
+MUTANTS["clip_buckets_no_clamp"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("no_clamp"))
+MUTANTS["clip_buckets_scale_in_bf16"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("scale_in_bf16"))
+MUTANTS["clip_buckets_bf16_truncate"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("bf16_truncate"))
+MUTANTS["round_to_bf16_truncates"] = dict(round_to_bf16=_bf16_truncate)
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(name):
     m = _mutant(**MUTANTS[name])
