@@ -83,12 +83,17 @@ def frobenius_normalize(G: np.ndarray) -> np.ndarray:
     return G / (norm + NORM_EPS)
 
 
-def ns_iteration(X: np.ndarray, a: float = NS_A, b: float = NS_B) -> np.ndarray:
-    """One cubic step X <- a X + b (X X^T) X; the blog's step ("Muon 核心")
-    is a = 1.5, b = -0.5, other (a, b) are the training guide's custom
-    coefficients ("超参数指南", ns_backend row)."""
+def ns_iteration(X: np.ndarray, a: float = NS_A, b: float = NS_B, c=None) -> np.ndarray:
+    """One Newton-Schulz step.  Cubic: X <- a X + b (X X^T) X; the blog's
+    step ("Muon 核心") is a = 1.5, b = -0.5, other (a, b) are the training
+    guide's custom coefficients ("超参数指南", ns_backend row).  With a third
+    coefficient c the step is the quintic odd polynomial
+    X <- a X + b A X + c A^2 X with A = X X^T (the guide's custom
+    coefficients read as a degree-5 form)."""
     A = X @ X.T
-    return a * X + b * (A @ X)
+    if c is None:
+        return a * X + b * (A @ X)
+    return a * X + b * (A @ X) + c * (A @ (A @ X))
 
 
 def newton_schulz(G: np.ndarray, steps: int, coeffs=(NS_A, NS_B)) -> np.ndarray:
@@ -96,19 +101,22 @@ def newton_schulz(G: np.ndarray, steps: int, coeffs=(NS_A, NS_B)) -> np.ndarray:
 
     Blog, "Muon 核心" listing: transpose when rows > cols, normalise, iterate,
     transpose back.  Returns fp64 with the input's shape.  ``coeffs`` are the
-    float32 values (a, b) the caller passes through the C ABI.
+    float32 values (a, b), or (a, b, c) for the quintic form, that the caller
+    passes through the C ABI.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
         raise ValueError("newton_schulz needs a 2-D matrix")
     if steps < 0:
         raise ValueError("steps must be >= 0")
+    if len(coeffs) not in (2, 3):
+        raise ValueError("coeffs must be (a, b) or (a, b, c)")
     transposed = G.shape[0] > G.shape[1]
     X = G.T.copy() if transposed else G.copy()
     X = frobenius_normalize(X)
-    a, b = (float(np.float32(c)) for c in coeffs)
+    cf = [float(np.float32(c)) for c in coeffs]
     for _ in range(steps):
-        X = ns_iteration(X, a, b)
+        X = ns_iteration(X, *cf)
     return X.T.copy() if transposed else X
 
 
@@ -233,11 +241,13 @@ def relative_frobenius(a: np.ndarray, b: np.ndarray) -> float:
     return float(num / den)
 
 
-def ns_flops(rows: int, cols: int, steps: int) -> float:
+def ns_flops(rows: int, cols: int, steps: int, quintic: bool = False) -> float:
     """Useful Newton-Schulz FLOPs of one matrix: per step m^2 n for the
-    symmetric product X X^T and 2 m^2 n for (X X^T) X, m = min, n = max."""
+    symmetric product X X^T and 2 m^2 n for (X X^T) X, m = min, n = max;
+    the quintic form adds m^3 for the symmetric square A A."""
     m, n = min(rows, cols), max(rows, cols)
-    return float(steps) * 3.0 * m * m * n
+    per = 3.0 * m * m * n + (float(m) ** 3 if quintic else 0.0)
+    return float(steps) * per
 
 
 def rank_mean(grads):

@@ -544,9 +544,47 @@ def pin_clip_buckets(o) -> None:
     assert norms2[1] == 0.0 and coefs2[1] == np.float32(1.0) and out2[1] == []
 
 
+def pin_quintic_coefficients(o, seed: int = 24) -> None:
+    """Quintic custom coefficients (a, b, c): X <- a X + b A X + c A^2 X,
+    A = X X^T, acts on each singular value as f(s) = a s + b s^3 + c s^5
+    (float32 a, b, c):
+    * a 1x1 input follows that scalar recurrence;
+    * random wide and tall inputs match U diag(f^k(sigma / (||G|| + 1e-7))) V^T
+      from the hand-written Jacobi SVD;
+    * the textbook quintic Newton-Schulz polynomial (15 s - 10 s^3 + 3 s^5) / 8
+      has f(1) = 1, so orthonormal rows are a fixed point of its inner step;
+    * c = 0 gives the cubic step with the same (a, b)."""
+    rng = np.random.default_rng(seed)
+    for coeffs in ((3.4445, -4.7750, 2.0315), (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0)):
+        a, b, c = (float(np.float32(x)) for x in coeffs)
+        f = lambda t: a * t + b * t ** 3 + c * t ** 5
+        for x in (0.8, -3.0, 1e-6):
+            t = x / (abs(x) + EPS)
+            for _ in range(4):
+                t = f(t)
+            got = o.newton_schulz(np.array([[x]]), 4, coeffs)[0, 0]
+            assert abs(got - t) <= 1e-13 * max(1.0, abs(t)), (coeffs, x, got, t)
+        G = rng.standard_normal((9, 21))
+        U, sig, V = jacobi_svd(G)
+        nrm = math.sqrt(float(np.sum(G * G)))
+        fs = []
+        for sv in sig:
+            t = sv / (nrm + EPS)
+            for _ in range(3):
+                t = f(t)
+            fs.append(t)
+        want = (U * np.array(fs)) @ V.T
+        assert _rel(o.newton_schulz(G, 3, coeffs), want) <= 1e-12
+        assert _rel(o.newton_schulz(G.T, 3, coeffs), want.T) <= 1e-12
+    Q = _semi_orthogonal(rng, 12, 30)
+    assert _rel(o.ns_iteration(Q, 15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0), Q) <= 1e-14
+    G = rng.standard_normal((7, 16))
+    assert _rel(o.newton_schulz(G, 4, (1.875, -0.875, 0.0)), o.newton_schulz(G, 4, (1.875, -0.875))) <= 1e-15
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
             pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean,
             pin_relative_frobenius, pin_orthogonality_error, pin_round_to_bf16,
-            pin_clip_buckets)
+            pin_clip_buckets, pin_quintic_coefficients)

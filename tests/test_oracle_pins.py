@@ -50,9 +50,9 @@ def _mutant(**overrides):
         transposed = G.shape[0] > G.shape[1]
         X = G.T.copy() if transposed else G.copy()
         X = m.frobenius_normalize(X)
-        a, b = (float(np.float32(c)) for c in coeffs)
+        cf = [float(np.float32(c)) for c in coeffs]
         for _ in range(steps):
-            X = m.ns_iteration(X, a, b)
+            X = m.ns_iteration(X, *cf)
         return X.T.copy() if transposed else X
 
     def muon_step(W, g, buf, *, lr, momentum, nesterov, weight_decay, ns_steps,
@@ -82,12 +82,12 @@ def _no_eps(G):
 
 
 MUTANTS = {
-    "sign_of_cubic_term": dict(ns_iteration=lambda X, a=1.5, b=-0.5: a * X - b * (X @ X.T) @ X),
-    "coefficient_3_not_1.5": dict(ns_iteration=lambda X, a=1.5, b=-0.5: 2 * a * X + b * (X @ X.T) @ X),
+    "sign_of_cubic_term": dict(ns_iteration=lambda X, a=1.5, b=-0.5, c=None: a * X - b * (X @ X.T) @ X + (0 if c is None else c * (X @ X.T) @ ((X @ X.T) @ X))),
+    "coefficient_3_not_1.5": dict(ns_iteration=lambda X, a=1.5, b=-0.5, c=None: 2 * a * X + b * (X @ X.T) @ X + (0 if c is None else c * (X @ X.T) @ ((X @ X.T) @ X))),
     # X^T X in place of X X^T: only expressible for square X (otherwise the
     # shapes do not conform), where it differs unless X is normal.
-    "gram_of_columns": dict(ns_iteration=lambda X, a=1.5, b=-0.5: a * X + b * ((X.T @ X) @ X if X.shape[0] == X.shape[1] else (X @ X.T) @ X)),
-    "one_step_short": dict(ns_iteration=lambda X, a=1.5, b=-0.5: X),
+    "gram_of_columns": dict(ns_iteration=lambda X, a=1.5, b=-0.5, c=None: a * X + b * ((X.T @ X) @ X if X.shape[0] == X.shape[1] else (X @ X.T) @ X)),
+    "one_step_short": dict(ns_iteration=lambda X, a=1.5, b=-0.5, c=None: X),
     "dropped_norm_eps": dict(frobenius_normalize=_no_eps),
     "eps_on_squared_norm": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64) / np.sqrt(np.sum(np.asarray(G, np.float64) ** 2) + 1e-7)),
     "no_normalisation": dict(frobenius_normalize=lambda G: np.asarray(G, np.float64)),
@@ -266,6 +266,25 @@ MUTANTS["clip_buckets_no_clamp"] = dict(clip_grad_norm_buckets=_clip_buckets_var
 MUTANTS["clip_buckets_scale_in_bf16"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("scale_in_bf16"))
 MUTANTS["clip_buckets_bf16_truncate"] = dict(clip_grad_norm_buckets=_clip_buckets_variant("bf16_truncate"))
 MUTANTS["round_to_bf16_truncates"] = dict(round_to_bf16=_bf16_truncate)
+
+
+
+def _quintic_variant(kind):
+    def f(X, a=1.5, b=-0.5, c=None):
+        A = X @ X.T
+        if c is None:
+            return a * X + b * (A @ X)
+        if kind == "c_on_AX":
+            return a * X + b * (A @ X) + c * (A @ X)
+        if kind == "b_c_swapped":
+            return a * X + c * (A @ X) + b * (A @ (A @ X))
+        return a * X + b * (A @ X)            # c ignored
+    return f
+
+
+MUTANTS["quintic_c_on_AX"] = dict(ns_iteration=_quintic_variant("c_on_AX"))
+MUTANTS["quintic_b_c_swapped"] = dict(ns_iteration=_quintic_variant("b_c_swapped"))
+MUTANTS["quintic_c_ignored"] = dict(ns_iteration=_quintic_variant("c_ignored"))
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
