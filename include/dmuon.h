@@ -28,14 +28,23 @@
  *     during the call only, and the page-locked host buffers named host_* of
  *     dmuon_muon_step_batched_host.  Updated tensors are written in place.
  *   - Calls are asynchronous: they only enqueue work on `stream` (a
- *     cudaStream_t; NULL is the legacy default stream).  Device pointers must
- *     stay valid until the stream reaches that work.
+ *     cudaStream_t; NULL is the legacy default stream) and never wait for the
+ *     device.  Device pointers must stay valid until the stream reaches that
+ *     work.  Tensor addresses are checked to be device memory (host memory,
+ *     page-locked or not, is refused with DMUON_ERR_INVALID_ARG).
  *   - Errors are returned before anything is enqueued; the message is in
  *     dmuon_last_error() (per host thread).  NaN/Inf in the data propagate and
  *     are not reported.
- *   - The first call with a new set of shapes / pointers builds a launch plan
- *     (host work plus one small synchronous upload); later identical calls
- *     reuse it.  Make that first call before capturing a CUDA graph.
+ *   - Launch plans (descriptors, TMA tensor maps, tile tables) depend on the
+ *     shapes, types, options and scratch address of a call, not on the tensor
+ *     addresses: a call with new shapes builds one on the host and uploads it
+ *     with small kernels on `stream`; later calls with the same shapes reuse
+ *     it, and new tensor addresses are written into it by one small kernel
+ *     per group, in stream order.  Library memory (plans, the per-stream
+ *     scratch arena) comes from a library memory pool in stream order
+ *     (cudaMallocFromPoolAsync / cudaFreeAsync); a plan evicted from the cache
+ *     (more than 64) is freed after the latest work that used it.  The first
+ *     call on a device also sets the device up (kernel attributes, the pool).
  */
 #ifndef DMUON_H_
 #define DMUON_H_
@@ -85,7 +94,8 @@ typedef struct {
  *   m, n    rows and cols, >= 1.
  *   steps   number of cubic steps, >= 0 (0 returns the normalised input).
  * Scratch memory comes from a library-owned per-stream arena (grown on
- * demand with cudaMalloc, kept until dmuon_release_cache()).
+ * demand in stream order from the library's memory pool, kept until
+ * dmuon_release_cache()).
  */
 int dmuon_ns_orthogonalize(void* X, int64_t m, int64_t n, int steps, dmuon_stream_t stream);
 
@@ -135,6 +145,13 @@ int dmuon_muon_step_batched_ex(void* const params[], const void* const grads[], 
  *   ns_a, ns_b      coefficients of the cubic step X <- a X + b (X X^T) X
  *                   (the training guide's custom NewtonSchulz coefficients,
  *                   "超参数指南"; the blog's step is a = 1.5, b = -0.5).
+ *   ns_c            != 0: the quintic step X <- a X + b A X + c A^2 X with
+ *                   A = X X^T (the same custom coefficients read as a degree-5
+ *                   odd polynomial; the pages print none).  A^2 is formed as a
+ *                   symmetric product (upper tiles): one more launch and
+ *                   m^3 more useful FLOPs per step, and one more m x m matrix
+ *                   of scratch.  struct_size may also be the size without
+ *                   this last field (then the step is cubic).
  *   lr_scale        DMUON_LR_PLAIN: lr as given.  DMUON_LR_SQRT_MAX: each
  *                   matrix uses lr * 0.2 * sqrt(max(rows, cols)) in place of lr
  *                   everywhere in its update (the guide's "internally scaled
@@ -157,15 +174,20 @@ typedef struct {
   int lr_scale;
   float max_grad_norm;
   float* grad_norm_out;
+  float ns_c; /* quintic coefficient (0: the cubic step); see above */
 } dmuon_step_options;
 void dmuon_step_options_default(dmuon_step_options* opts);
 
 /* One Muon update of `count` matrices with options (arguments otherwise as
  * dmuon_muon_step_batched).  workspace may be NULL (library arena) or a
- * caller buffer of ws_bytes >= dmuon_workspace_bytes(). */
+ * caller buffer of ws_bytes >= dmuon_workspace_bytes_opts() (which equals
+ * dmuon_workspace_bytes() for the cubic step). */
 int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[], float* const bufs[],
                                  const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
                                  void* workspace, size_t ws_bytes, dmuon_stream_t stream);
+/* Scratch bytes for dmuon_muon_step_batched_opts with these options (the
+ * quintic step needs one more m x m matrix per matrix); 0 for invalid input. */
+size_t dmuon_workspace_bytes_opts(const dmuon_shape shapes[], int count, const dmuon_step_options* opts);
 
 /*
  * dmuon_muon_step_batched_reduce -- the owner's update of an owner-partitioned
@@ -257,6 +279,43 @@ int dmuon_adamw_step_batched(void* const params[], const void* const grads[], fl
                              float lr, float beta1, float beta2, float eps, float weight_decay,
                              int64_t step, dmuon_stream_t stream);
 
+/*
+ * dmuon_clip_grad_norm_buckets -- gradient clipping of several gradient
+ * groups at once, each group ("segment") with its own norm and coefficient:
+ * the training guide's fused clipping of the regular / Muon / AdamW
+ * gradients ("梯度裁剪", "regular / Muon / AdamW 的融合 CUDA 裁剪"), which
+ * computes every segment's norm, clip coefficient and in-place scaling in
+ * one pass over the gradients while keeping per-segment semantics.  For each
+ * segment s, as for the Muon-only clip of dmuon_step_options:
+ *   ||g||_s = sqrt(sum of g^2 over every tensor of segment s)   (fp64 sums)
+ *   c_s     = fl32(min(1, max_norms[s] / (||g||_s + 1e-6)))     (a NaN norm gives 1)
+ *   g      <- fl32(g * c_s), rounded to nearest for bf16 storage, in place
+ * Segments with c_s == 1 are not rewritten (the scaling is the identity).
+ * The sums have a fixed order: results are identical run to run.
+ *   grads[i]    device pointer of descs[i].numel elements (flat, any shape),
+ *               updated in place; NULL skips tensor i.
+ *   descs[i]    numel >= 1, dtype DMUON_BF16 or DMUON_F32, segment in [0, nseg).
+ *   max_norms   HOST array of nseg values > 0; +inf measures a segment
+ *               without scaling it.
+ *   nseg        1 .. DMUON_MAX_SEGMENTS.  A segment without tensors has norm 0.
+ *   norms_out   optional DEVICE pointer to nseg floats: ||g||_s before clipping.
+ *   coefs_out   optional DEVICE pointer to nseg floats: c_s.
+ *   workspace   NULL (library arena of the stream) or device scratch of
+ *               ws_bytes >= dmuon_clip_workspace_bytes(), 256-byte aligned.
+ * Launches: one norm pass, one block per segment for the coefficients, one
+ * scale pass (more launches only past 512 tensors).  Errors as for the other
+ * entry points; nothing is enqueued after an argument error.
+ */
+#define DMUON_MAX_SEGMENTS 64
+typedef struct {
+  int64_t numel;
+  int32_t dtype, segment;
+} dmuon_grad_desc;
+size_t dmuon_clip_workspace_bytes(const dmuon_grad_desc descs[], int count, int nseg);
+int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc descs[], int count,
+                                 const float max_norms[], int nseg, float* norms_out, float* coefs_out,
+                                 void* workspace, size_t ws_bytes, dmuon_stream_t stream);
+
 /* Scratch bytes that suffice for dmuon_muon_step_batched_ex on these shapes
  * (matrices with a NULL gradient may be left out or counted; counting them
  * over-estimates): the need of the whole set as one group, which covers any
@@ -276,9 +335,20 @@ const char* dmuon_backend_string(void);
  * clear != 0 resets the word to 0. */
 int dmuon_device_status(int clear);
 
-/* Frees the library's cached plans and scratch arenas (synchronises the
- * device).  Safe to call at any time from the host. */
+/* Frees the library's cached plans and scratch arenas and returns the pool's
+ * memory (synchronises the device: the one call that does).  Safe to call at
+ * any time from the host. */
 void dmuon_release_cache(void);
+
+/* Number of launch plans built in this process (a call with shapes seen
+ * before builds none, whatever its tensor addresses). */
+int64_t dmuon_plan_builds(void);
+
+/* Test hook (host only, launches nothing): the device-memory check the entry
+ * points apply to every tensor address.  DMUON_OK for device or managed
+ * memory, DMUON_ERR_INVALID_ARG for host memory (page-locked or not) and
+ * NULL. */
+int dmuon_debug_check_pointer(const void* p);
 
 /*
  * dmuon_ns_orthogonalize_noalloc -- same result as dmuon_ns_orthogonalize
@@ -289,16 +359,20 @@ void dmuon_release_cache(void);
  * block or synchronise the device.  It calls no allocation routine.  (The
  * pages have no counterpart of this entry point; it is a property of this
  * library.)
- *   Scratch: a fixed 32 MiB device array inside the library, reserved on
- *   every device that loads the library and held until the process exits.
- *   Matrices whose scratch (dmuon_ns_workspace_bytes(m, n, DMUON_BF16) for
- *   steps >= 2) exceeds 32 MiB - 16 KiB are rejected with
- *   DMUON_ERR_UNSUPPORTED; e.g. 2048 x 2048 and 1024 x 4096 fit, 4096 x 4096
- *   does not.
+ *   Scratch: a fixed 32 MiB device array inside the library.  The driver
+ *   allocates it when the library's module is loaded on a device, i.e. at the
+ *   first call of any entry point there, and it is held until the process
+ *   exits; a caller that pre-reserves the device's memory should make one
+ *   library call first.  Matrices whose scratch
+ *   (dmuon_ns_workspace_bytes(m, n, DMUON_BF16) for steps >= 2) exceeds
+ *   32 MiB - 16 KiB are rejected with DMUON_ERR_UNSUPPORTED; e.g. 2048 x 2048
+ *   and 1024 x 4096 fit, 4096 x 4096 does not.
  *   Sharing: every call uses the same array, and nothing carries over from
- *   one call to the next.  Calls that may overlap on the GPU (different
- *   streams without ordering between them) race on it; calls on one stream
- *   are ordered.
+ *   one call to the next: each call writes its own launch description
+ *   (descriptor and tensor maps, passed as kernel parameters of a small
+ *   upload kernel on `stream`) at the front of the array.  Calls that may
+ *   overlap on the GPU (different streams without ordering between them) race
+ *   on it; calls on one stream are ordered.
  *   Set-up: the first call on a device looks up the array's device address
  *   (once per device); make that first call before any stream capture.
  */
@@ -312,7 +386,9 @@ enum {
   DMUON_KERNEL_GEMM = 3,     /* X <- 1.5 X - 0.5 A X, last step fused with the update */
   DMUON_KERNEL_APPLY = 4,    /* update for ns_steps == 0 */
   DMUON_KERNEL_ADAMW = 5,    /* AdamW of the non-orthogonalised parameters */
-  DMUON_KERNEL_KINDS = 6
+  DMUON_KERNEL_CLIP = 6,     /* per-segment gradient clipping (norms, coefficients, scaling) */
+  DMUON_KERNEL_SQUARE = 7,   /* quintic coefficients: P = b A + c A A (upper tiles) */
+  DMUON_KERNEL_KINDS = 8
 };
 
 /* Per-kernel timing: while enabled, every launch is bracketed by CUDA events

@@ -22,14 +22,15 @@ __all__ = [
     "dmuon_last_error", "dmuon_backend_string", "dmuon_device_status", "dmuon_release_cache",
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
+    "dmuon_plan_builds", "dmuon_debug_check_pointer",
     "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
     "dmuon_adamw_step_batched", "DmuonTensorDesc", "dmuon_muon_step_batched_host",
-    "dmuon_muon_step_batched_reduce",
-    "DMUON_MAX_CHUNKS",
+    "dmuon_muon_step_batched_reduce", "dmuon_clip_grad_norm_buckets", "dmuon_clip_workspace_bytes",
+    "DmuonGradDesc", "DMUON_MAX_CHUNKS", "DMUON_MAX_SEGMENTS",
 ]
 
 #: Kernel kinds of dmuon_stage_times(), in order.
-KERNEL_KINDS = ("prologue", "finalize", "syrk", "gemm", "apply", "adamw")
+KERNEL_KINDS = ("prologue", "finalize", "syrk", "gemm", "apply", "adamw", "clip", "square")
 
 DMUON_F32 = 0
 DMUON_BF16 = 1
@@ -55,6 +56,11 @@ class DmuonShape(ctypes.Structure):
 DMUON_LR_PLAIN = 0
 DMUON_LR_SQRT_MAX = 1
 DMUON_MAX_CHUNKS = 32
+DMUON_MAX_SEGMENTS = 64
+
+
+class DmuonGradDesc(ctypes.Structure):
+    _fields_ = [("numel", ctypes.c_int64), ("dtype", ctypes.c_int32), ("segment", ctypes.c_int32)]
 
 
 class DmuonTensorDesc(ctypes.Structure):
@@ -67,7 +73,19 @@ class DmuonStepOptions(ctypes.Structure):
                 ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("nesterov", ctypes.c_int), ("ns_steps", ctypes.c_int),
                 ("ns_a", ctypes.c_float), ("ns_b", ctypes.c_float), ("lr_scale", ctypes.c_int),
-                ("max_grad_norm", ctypes.c_float), ("grad_norm_out", ctypes.c_void_p)]
+                ("max_grad_norm", ctypes.c_float), ("grad_norm_out", ctypes.c_void_p),
+                ("ns_c", ctypes.c_float)]
+
+
+def _set_coefficients(o: "DmuonStepOptions", coeffs) -> None:
+    """(a, b): the cubic step; (a, b, c): the quintic step."""
+    if len(coeffs) == 2:
+        o.ns_a, o.ns_b = coeffs
+        o.ns_c = 0.0
+    elif len(coeffs) == 3:
+        o.ns_a, o.ns_b, o.ns_c = coeffs
+    else:
+        raise ValueError("ns_coefficients must be (a, b) or (a, b, c)")
 
 
 def library_path() -> str:
@@ -115,6 +133,12 @@ def load_library() -> ctypes.CDLL:
         "dmuon_debug_partition": (i32, [sp, i32, i32, ctypes.POINTER(ctypes.c_int), i32]),
         "dmuon_muon_step_batched_reduce": (i32, [pp, pp, pp, sp, i32, i32, ctypes.POINTER(DmuonStepOptions),
                                                  vp, sz, vp]),
+        "dmuon_clip_workspace_bytes": (sz, [ctypes.POINTER(DmuonGradDesc), i32, i32]),
+        "dmuon_workspace_bytes_opts": (sz, [sp, i32, ctypes.POINTER(DmuonStepOptions)]),
+        "dmuon_plan_builds": (ctypes.c_int64, []),
+        "dmuon_debug_check_pointer": (i32, [vp]),
+        "dmuon_clip_grad_norm_buckets": (i32, [pp, ctypes.POINTER(DmuonGradDesc), i32,
+                                               ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -281,7 +305,7 @@ def dmuon_muon_step_batched_opts(params, grads, bufs, lr: float = 0.02, momentum
     lib.dmuon_step_options_default(ctypes.byref(o))
     o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
     o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
-    o.ns_a, o.ns_b = ns_coefficients
+    _set_coefficients(o, ns_coefficients)
     o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
     o.max_grad_norm = max_grad_norm
     if grad_norm_out is not None:
@@ -330,7 +354,7 @@ def dmuon_muon_step_batched_reduce(params, rank_grads, bufs, lr: float = 0.02, m
     lib.dmuon_step_options_default(ctypes.byref(o))
     o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
     o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
-    o.ns_a, o.ns_b = ns_coefficients
+    _set_coefficients(o, ns_coefficients)
     o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
     o.max_grad_norm = max_grad_norm
     ws_ptr, ws_bytes = _workspace(workspace, b.device)
@@ -380,7 +404,7 @@ def dmuon_muon_step_batched_host(params, grads, bufs, host_grads, host_params=No
     lib.dmuon_step_options_default(ctypes.byref(o))
     o.lr, o.momentum, o.weight_decay = lr, momentum, weight_decay
     o.nesterov, o.ns_steps = (1 if nesterov else 0), ns_steps
-    o.ns_a, o.ns_b = ns_coefficients
+    _set_coefficients(o, ns_coefficients)
     o.lr_scale = {"plain": DMUON_LR_PLAIN, "sqrt_max": DMUON_LR_SQRT_MAX}[lr_scale]
     ws_ptr, ws_bytes = _workspace(workspace, b.device)
     P, G, B, S, cnt = b.args()
@@ -455,6 +479,17 @@ def dmuon_launch_count() -> int:
     return int(load_library().dmuon_launch_count())
 
 
+def dmuon_plan_builds() -> int:
+    """Launch plans built so far (shapes seen before build none)."""
+    return int(load_library().dmuon_plan_builds())
+
+
+def dmuon_debug_check_pointer(address: int) -> int:
+    """The entry points' device-memory check of one address (launches
+    nothing): 0 for device memory, DMUON_ERR_INVALID_ARG (-1) otherwise."""
+    return int(load_library().dmuon_debug_check_pointer(address))
+
+
 def dmuon_ns_orthogonalize_noalloc(X: torch.Tensor, steps: int = 5) -> torch.Tensor:
     """In-place cubic Newton-Schulz of one bf16 matrix without allocating
     any device memory: the scratch is a fixed 32 MiB array inside the
@@ -471,6 +506,57 @@ def dmuon_ns_orthogonalize_noalloc(X: torch.Tensor, steps: int = 5) -> torch.Ten
                                                   _stream(X.device)))
     return X
 
+
+
+def _clip_descs(segments):
+    flat, descs = [], []
+    dev = None
+    for si, seg in enumerate(segments):
+        for g in seg:
+            if g is None:
+                continue
+            if not isinstance(g, torch.Tensor) or not g.is_cuda or not g.is_contiguous():
+                raise ValueError(f"segment {si}: gradients must be contiguous CUDA tensors")
+            dev = dev or g.device
+            if g.device != dev:
+                raise ValueError("all gradients must be on one device")
+            flat.append(g)
+            descs.append(DmuonGradDesc(g.numel(), _dtype_code(g.dtype), si))
+    D = (DmuonGradDesc * max(len(descs), 1))(*descs)
+    return flat, D, dev
+
+
+def dmuon_clip_workspace_bytes(segments) -> int:
+    flat, D, _ = _clip_descs(segments)
+    return int(load_library().dmuon_clip_workspace_bytes(D, len(flat), max(len(segments), 1)))
+
+
+def dmuon_clip_grad_norm_buckets(segments, max_norms, workspace: Optional[torch.Tensor] = None,
+                                 device: Optional[torch.device] = None):
+    """Clip several gradient groups in place, each with its own norm and
+    coefficient: ``segments[s]`` is a list of gradient tensors (bf16 or fp32,
+    any shape; None entries are skipped), ``max_norms`` one bound per segment
+    (or one for all; ``math.inf`` measures without clipping).  Returns the
+    per-segment norms before clipping and the coefficients, as fp32 CUDA
+    tensors (asynchronous on the current stream)."""
+    lib = load_library()
+    nseg = len(segments)
+    if isinstance(max_norms, (int, float)):
+        max_norms = [float(max_norms)] * nseg
+    if len(max_norms) != nseg or nseg < 1:
+        raise ValueError("one max_norm per segment, at least one segment")
+    flat, D, dev = _clip_descs(segments)
+    dev = dev or device or torch.device("cuda", torch.cuda.current_device())
+    norms = torch.empty(nseg, dtype=torch.float32, device=dev)
+    coefs = torch.empty(nseg, dtype=torch.float32, device=dev)
+    G = (ctypes.c_void_p * max(len(flat), 1))(*[g.data_ptr() for g in flat])
+    M = (ctypes.c_float * nseg)(*max_norms)
+    ws_ptr, ws_bytes = _workspace(workspace, dev)
+    with torch.cuda.device(dev):
+        _check(lib.dmuon_clip_grad_norm_buckets(ctypes.cast(G, ctypes.POINTER(ctypes.c_void_p)), D,
+                                                len(flat), M, nseg, norms.data_ptr(), coefs.data_ptr(),
+                                                ws_ptr, ws_bytes, _stream(dev)))
+    return norms, coefs
 
 
 def dmuon_adamw_step_batched(params, grads, exp_avgs, exp_avg_sqs, lr: float = 1e-3,

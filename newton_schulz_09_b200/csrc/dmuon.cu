@@ -15,6 +15,7 @@
 #include <memory>
 #include <mutex>
 #include <string>
+#include <unordered_set>
 #include <utility>
 #include <vector>
 
@@ -46,8 +47,13 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 std::mutex g_mu;
 int g_fail_allocs = 0;
+int64_t g_launches = 0;   // kernels this library has launched
 
-cudaError_t lib_malloc(void** p, size_t bytes) {
+// Device memory of the library (launch plans, scratch arenas) comes from one
+// memory pool per device, allocated and freed in stream order: no call
+// blocks on, or synchronises, the device.  The pool keeps freed memory for
+// reuse (release threshold: unlimited) until dmuon_release_cache().
+cudaError_t lib_malloc_async(void** p, size_t bytes, cudaMemPool_t pool, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_fail_allocs > 0) {
@@ -56,7 +62,7 @@ cudaError_t lib_malloc(void** p, size_t bytes) {
       return cudaErrorMemoryAllocation;
     }
   }
-  return cudaMalloc(p, bytes);
+  return cudaMallocFromPoolAsync(p, bytes, pool, st);
 }
 
 // ------------------------------------------------------------------ driver
@@ -134,6 +140,7 @@ struct StepOpts {
   float lr = 0.0f, mu = 0.0f, wd = 0.0f;
   int nesterov = 0, steps = 0;
   float ca = 1.5f, cb = -0.5f;      // cubic coefficients
+  float cc = 0.0f;                  // != 0: quintic X <- ca X + cb A X + cc A A X
   int lr_scale = DMUON_LR_PLAIN;
   float max_norm = 0.0f;            // > 0: global-norm gradient clipping
   float* norm_out = nullptr;        // device pointer for the pre-clip norm
@@ -173,6 +180,7 @@ int check_matrix(const MatIn& x, int i) {
 struct MatLayout {
   int64_t m, n, ldx, lda;
   size_t x0, x1, a;        // byte offsets in the workspace (x1/a = SIZE_MAX if unused)
+  size_t p;                // quintic: P = b A + c A A (SIZE_MAX if unused)
   size_t o0, o1;           // tf32 operand copies of X0/X1 (fp32 only; else == x0/x1)
   int64_t ptiles, ptiles_c;
 };
@@ -190,7 +198,7 @@ struct Layout {
   size_t bytes = 0;
 };
 
-Layout make_layout(const std::vector<MatIn>& in, int steps) {
+Layout make_layout(const std::vector<MatIn>& in, int steps, bool quintic = false) {
   Layout L;
   L.mats.resize(in.size());
   size_t off = 0;
@@ -220,6 +228,8 @@ Layout make_layout(const std::vector<MatIn>& in, int steps) {
         if (steps >= 2) { ml.o1 = off; off = align_up(off + xb, 1024); }
       }
       if (steps >= 1) { ml.a = off; off = align_up(off + ab, 1024); }
+      ml.p = SIZE_MAX;
+      if (steps >= 1 && quintic) { ml.p = off; off = align_up(off + ab, 1024); }
       // Prologue work items: flat chunks, or kTR x kTC tiles when transposed.
       if (in[i].rows > in[i].cols) {
         ml.ptiles_c = cdiv(in[i].cols, kTC);
@@ -247,25 +257,45 @@ struct GroupPlan {
   int nmat;
   int first;              // first MatDesc index of the group
   int64_t ptiles;
-  int syrk_tiles, gemm_tiles;
+  int syrk_tiles, gemm_tiles, square_tiles;
   const int* syrk_order; const int* syrk_prefix;
   const int* gemm_order; const int* gemm_prefix;
+  const int* square_prefix;   // SQUARE tiles along gemm_order (quintic plans)
   const int64_t* pprefix;
   float* partials;
   double* gpartials;
 };
 
+// The caller's addresses of one matrix, as a plan's device descriptors hold them.
+struct PtrSet {
+  void* W = nullptr;
+  const void* G = nullptr;
+  float* buf = nullptr;
+  int vec4 = 0;
+  bool operator==(const PtrSet& o) const { return W == o.W && G == o.G && buf == o.buf && vec4 == o.vec4; }
+};
+
+// A launch plan depends on the shapes, types, options class and scratch
+// address of a call, not on the caller's tensor addresses: those are written
+// into the plan's descriptors by a small patch kernel, in stream order, when
+// they differ from the ones the descriptors hold.
 struct Plan {
   std::vector<uint8_t> key;
   uint64_t hash = 0;
   int device = 0;
-  void* dmem = nullptr;
+  void* dmem = nullptr;           // pool memory (freed in stream order on eviction)
   const MatDesc* d_mats = nullptr;
   const MatMaps* d_maps = nullptr;
   float* clip = nullptr;          // workspace: {clip coefficient, gradient norm}
+  bool quintic = false;
   std::vector<GroupPlan> groups;
+  std::vector<int> desc_of;       // input matrix -> descriptor index
+  std::vector<PtrSet> cur;        // per descriptor: the addresses its device copy holds
+  cudaEvent_t last = nullptr;     // recorded after the latest work that used the plan
+  cudaStream_t last_st = nullptr; // ... on this stream
   ~Plan() {
     if (dmem) cudaFree(dmem);
+    if (last) cudaEventDestroy(last);
   }
 };
 
@@ -273,6 +303,7 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int* err = nullptr;
+  cudaMemPool_t pool = nullptr;
 };
 DeviceInfo g_dev[64];
 std::list<std::unique_ptr<Plan>> g_plans;   // most recently used first
@@ -323,7 +354,9 @@ int device_setup(int dev) {
       reinterpret_cast<const void*>(&ns_stage_kernel<kSyrk, __nv_bfloat16>),
       reinterpret_cast<const void*>(&ns_stage_kernel<kGemm, __nv_bfloat16>),
       reinterpret_cast<const void*>(&ns_stage_kernel<kSyrk, float>),
-      reinterpret_cast<const void*>(&ns_stage_kernel<kGemm, float>)};
+      reinterpret_cast<const void*>(&ns_stage_kernel<kGemm, float>),
+      reinterpret_cast<const void*>(&ns_stage_kernel<kSquare, __nv_bfloat16>),
+      reinterpret_cast<const void*>(&ns_stage_kernel<kSquare, float>)};
   for (const void* k : ks) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
@@ -337,7 +370,63 @@ int device_setup(int dev) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prologue smem)");
   }
   if (!encode_fn()) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  e = cudaMemPoolCreate(&d.pool, &props);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+  uint64_t keep = UINT64_MAX;
+  e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolSetAttribute");
   d.ready = true;
+  return DMUON_OK;
+}
+
+int64_t g_plan_builds = 0;   // launch plans built in this process
+
+// Writes `bytes` (a multiple of 16) of host data to device memory with
+// upload kernels on `st`: stream ordered, no host staging, no synchronous copy.
+void enqueue_upload(void* dst, const uint8_t* src, size_t bytes, cudaStream_t st) {
+  std::unique_ptr<UploadParams> up(new UploadParams());
+  const size_t words = bytes / 16;
+  for (size_t w0 = 0; w0 < words; w0 += kUploadWords) {
+    const int n = static_cast<int>(std::min<size_t>(kUploadWords, words - w0));
+    up->dst = reinterpret_cast<uint4*>(dst) + w0;
+    up->nwords = n;
+    std::memcpy(up->w, src + w0 * 16, static_cast<size_t>(n) * 16);
+    ++g_launches;
+    upload_kernel<<<1, 256, 0, st>>>(*up);
+  }
+}
+
+// Device pointers already checked (per device).  A checked address stays
+// device memory: under unified addressing, host and device allocations never
+// share virtual addresses.
+std::unordered_set<const void*> g_checked[64];
+
+// 0 when `p` is device (or managed) memory; DMUON_ERR_INVALID_ARG for host
+// memory (page-locked or not); nothing is launched either way.
+int classify_pointer(const void* p) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return DMUON_ERR_INVALID_ARG;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) ? DMUON_OK : DMUON_ERR_INVALID_ARG;
+}
+
+int check_device_ptr(int dev, const void* p, int i, const char* what) {
+  if (p == nullptr) return DMUON_OK;
+  std::unordered_set<const void*>& seen = g_checked[dev];
+  if (seen.count(p)) return DMUON_OK;
+  if (classify_pointer(p) != DMUON_OK)
+    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: %s is not device memory (host memory cannot be "
+                "passed to the kernels)", i, what);
+  if (seen.size() >= 65536) seen.clear();
+  seen.insert(p);
   return DMUON_OK;
 }
 
@@ -351,15 +440,34 @@ int64_t syrk_tiles_of(int64_t m) {
 int64_t gemm_tiles_of(int64_t m, int64_t n) { return cdiv(m, kBM) * cdiv(n, kBN); }
 
 // Builds (or finds) the plan for these matrices and this workspace.
-int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** out) {
+// 16-byte vector access of a matrix's parameter, gradient and buffer rows.
+int vec4_of(const MatIn& x) {
+  bool v = (x.cols % 4 == 0) && aligned(x.W, 16) && aligned(x.G, 16) && (x.buf == nullptr || aligned(x.buf, 16));
+  for (const void* q : x.gr) v = v && aligned(q, 16);
+  return v ? 1 : 0;
+}
+
+PtrSet ptrs_of(const MatIn& x) {
+  PtrSet p;
+  p.W = x.W;
+  p.G = x.G;
+  p.buf = x.buf;
+  p.vec4 = vec4_of(x);
+  return p;
+}
+
+// Builds (or finds) the plan for these shapes and this workspace; a new
+// plan's device memory is allocated from the pool and uploaded on `st`.
+int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, int dev, cudaStream_t st,
+             Plan** out) {
   std::vector<uint8_t> key;
-  key.reserve(64 + in.size() * 56);
+  key.reserve(64 + in.size() * 48);
   put(key, dev);
   put(key, steps > 1 ? 2 : steps);
+  put(key, quintic);
   put(key, ws);
   put(key, static_cast<int64_t>(in.size()));
   for (const MatIn& x : in) {
-    put(key, x.W); put(key, x.G); put(key, x.buf);
     put(key, x.rows); put(key, x.cols);
     put(key, x.pdt); put(key, x.gdt); put(key, x.mode); put(key, x.lr_mult);
     put(key, static_cast<int64_t>(x.gr.size()));
@@ -374,7 +482,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     }
   }
 
-  const Layout L = make_layout(in, steps);
+  const Layout L = make_layout(in, steps, quintic);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const int nmat = static_cast<int>(in.size());
 
@@ -382,7 +490,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   std::vector<MatDesc> descs(nmat);
   std::vector<MatMaps> maps(nmat);
   struct GroupArrays {
-    std::vector<int> so, sp, go, gp;
+    std::vector<int> so, sp, go, gp, qp;
     std::vector<int64_t> pp;
   };
   std::vector<GroupArrays> ga(L.groups.size());
@@ -390,6 +498,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   P->key = std::move(key);
   P->hash = h;
   P->device = dev;
+  P->quintic = quintic;
 
   int first = 0;
   std::vector<int> desc_of(nmat, -1);
@@ -420,15 +529,14 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
       d.Xop[0] = wsb + ml.o0;
       d.Xop[1] = (ml.o1 != SIZE_MAX) ? wsb + ml.o1 : nullptr;
       d.A = (ml.a != SIZE_MAX) ? wsb + ml.a : nullptr;
+      d.P = (ml.p != SIZE_MAX) ? wsb + ml.p : nullptr;
       d.scale = reinterpret_cast<float*>(wsb + g.scales) + k;
       d.lr_mult = x.lr_mult;
       d.m = static_cast<int>(ml.m); d.n = static_cast<int>(ml.n);
       d.T = x.rows > x.cols ? 1 : 0;
       d.mode = x.mode;
       d.g_bf16 = x.gdt == DMUON_BF16 ? 1 : 0;
-      d.vec4 = (x.cols % 4 == 0) && aligned(x.W, 16) && aligned(x.G, 16) &&
-               (x.buf == nullptr || aligned(x.buf, 16));
-      for (const void* q : x.gr) d.vec4 = d.vec4 && aligned(q, 16);
+      d.vec4 = vec4_of(x);
       d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
       if (d.world > 1) gp.ranks = true;
       d.Gr = nullptr;   // set once the plan's device memory exists
@@ -454,6 +562,10 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
                                              : CU_TENSOR_MAP_SWIZZLE_128B);
         }
         if (d.A) okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+        if (d.P) {
+          okm &= encode_2d(&mm.aw, dt, d.A, ml.m, ml.m, ml.lda, BK, kBN);
+          okm &= encode_2d(&mm.p, dt, d.P, ml.m, ml.m, ml.lda, BK, kBM);
+        }
         if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed for matrix %d", i);
       }
     }
@@ -469,20 +581,24 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
       const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
       return x.m != y.m ? x.m > y.m : x.n > y.n;
     });
-    int64_t st = 0, gt = 0;
+    int64_t st = 0, gt = 0, qt = 0;
     A.sp.push_back(0);
     A.gp.push_back(0);
+    A.qp.push_back(0);
     for (int k = 0; k < gp.nmat; ++k) {
       st += syrk_tiles_of(descs[first + so[k]].m);
       gt += gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
+      qt += syrk_tiles_of(descs[first + go[k]].m);   // SQUARE contracts over m: the GEMM's order
       A.sp.push_back(static_cast<int>(st));
       A.gp.push_back(static_cast<int>(gt));
+      A.qp.push_back(static_cast<int>(qt));
     }
     if (st > INT32_MAX || gt > INT32_MAX)
       return fail(DMUON_ERR_UNSUPPORTED, "too many tiles in one launch");
     A.so = so; A.go = go;
     gp.syrk_tiles = static_cast<int>(st);
     gp.gemm_tiles = static_cast<int>(gt);
+    gp.square_tiles = static_cast<int>(qt);
     gp.partials = reinterpret_cast<float*>(wsb + g.partials);
     gp.gpartials = reinterpret_cast<double*>(wsb + g.gpartials);
     P->groups.push_back(gp);
@@ -493,13 +609,15 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   size_t off = 0;
   const size_t o_desc = off; off = align_up(off + sizeof(MatDesc) * nmat, 128);
   const size_t o_maps = off; off = align_up(off + sizeof(MatMaps) * nmat, 128);
-  std::vector<size_t> o_g(ga.size() * 5);
+  constexpr int kArr = 6;
+  std::vector<size_t> o_g(ga.size() * kArr);
   for (size_t gi = 0; gi < ga.size(); ++gi) {
-    o_g[gi * 5 + 0] = off; off = align_up(off + sizeof(int64_t) * ga[gi].pp.size(), 128);
-    o_g[gi * 5 + 1] = off; off = align_up(off + sizeof(int) * ga[gi].so.size(), 128);
-    o_g[gi * 5 + 2] = off; off = align_up(off + sizeof(int) * ga[gi].sp.size(), 128);
-    o_g[gi * 5 + 3] = off; off = align_up(off + sizeof(int) * ga[gi].go.size(), 128);
-    o_g[gi * 5 + 4] = off; off = align_up(off + sizeof(int) * ga[gi].gp.size(), 128);
+    o_g[gi * kArr + 0] = off; off = align_up(off + sizeof(int64_t) * ga[gi].pp.size(), 128);
+    o_g[gi * kArr + 1] = off; off = align_up(off + sizeof(int) * ga[gi].so.size(), 128);
+    o_g[gi * kArr + 2] = off; off = align_up(off + sizeof(int) * ga[gi].sp.size(), 128);
+    o_g[gi * kArr + 3] = off; off = align_up(off + sizeof(int) * ga[gi].go.size(), 128);
+    o_g[gi * kArr + 4] = off; off = align_up(off + sizeof(int) * ga[gi].gp.size(), 128);
+    o_g[gi * kArr + 5] = off; off = align_up(off + sizeof(int) * ga[gi].qp.size(), 128);
   }
   // The ranks' gradient buffers of matrices that average several (rank order).
   std::vector<const void*> gr_ptrs;
@@ -511,9 +629,15 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
     }
   }
   const size_t o_gr = off; off = align_up(off + sizeof(void*) * gr_ptrs.size(), 128);
-  cudaError_t e = lib_malloc(&P->dmem, off);
+  cudaError_t e = cudaEventCreateWithFlags(&P->last, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    P->last = nullptr;
+    return cuda_fail(e, "cudaEventCreate");
+  }
+  e = lib_malloc_async(&P->dmem, off, g_dev[dev].pool, st);
   if (e != cudaSuccess) {
     P->dmem = nullptr;
+    cudaGetLastError();
     return fail(DMUON_ERR_NO_WORKSPACE, "plan allocation of %zu bytes failed", off);
   }
   uint8_t* base = static_cast<uint8_t*>(P->dmem);
@@ -525,21 +649,29 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   std::memcpy(img.data() + o_desc, descs.data(), sizeof(MatDesc) * nmat);
   std::memcpy(img.data() + o_maps, maps.data(), sizeof(MatMaps) * nmat);
   for (size_t gi = 0; gi < ga.size(); ++gi) {
-    std::memcpy(img.data() + o_g[gi * 5 + 0], ga[gi].pp.data(), sizeof(int64_t) * ga[gi].pp.size());
-    std::memcpy(img.data() + o_g[gi * 5 + 1], ga[gi].so.data(), sizeof(int) * ga[gi].so.size());
-    std::memcpy(img.data() + o_g[gi * 5 + 2], ga[gi].sp.data(), sizeof(int) * ga[gi].sp.size());
-    std::memcpy(img.data() + o_g[gi * 5 + 3], ga[gi].go.data(), sizeof(int) * ga[gi].go.size());
-    std::memcpy(img.data() + o_g[gi * 5 + 4], ga[gi].gp.data(), sizeof(int) * ga[gi].gp.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 0], ga[gi].pp.data(), sizeof(int64_t) * ga[gi].pp.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 1], ga[gi].so.data(), sizeof(int) * ga[gi].so.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 2], ga[gi].sp.data(), sizeof(int) * ga[gi].sp.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 3], ga[gi].go.data(), sizeof(int) * ga[gi].go.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 4], ga[gi].gp.data(), sizeof(int) * ga[gi].gp.size());
+    std::memcpy(img.data() + o_g[gi * kArr + 5], ga[gi].qp.data(), sizeof(int) * ga[gi].qp.size());
   }
-  e = cudaMemcpy(P->dmem, img.data(), img.size(), cudaMemcpyHostToDevice);
+  enqueue_upload(P->dmem, img.data(), img.size(), st);
+  e = cudaEventRecord(P->last, st);
   if (e != cudaSuccess) return cuda_fail(e, "plan upload");
+  P->last_st = st;
+  ++g_plan_builds;
+  P->desc_of = desc_of;
+  P->cur.resize(nmat);
+  for (int i = 0; i < nmat; ++i) P->cur[desc_of[i]] = ptrs_of(in[i]);
   for (size_t gi = 0; gi < P->groups.size(); ++gi) {
     GroupPlan& gp = P->groups[gi];
-    gp.pprefix = reinterpret_cast<const int64_t*>(base + o_g[gi * 5 + 0]);
-    gp.syrk_order = reinterpret_cast<const int*>(base + o_g[gi * 5 + 1]);
-    gp.syrk_prefix = reinterpret_cast<const int*>(base + o_g[gi * 5 + 2]);
-    gp.gemm_order = reinterpret_cast<const int*>(base + o_g[gi * 5 + 3]);
-    gp.gemm_prefix = reinterpret_cast<const int*>(base + o_g[gi * 5 + 4]);
+    gp.pprefix = reinterpret_cast<const int64_t*>(base + o_g[gi * kArr + 0]);
+    gp.syrk_order = reinterpret_cast<const int*>(base + o_g[gi * kArr + 1]);
+    gp.syrk_prefix = reinterpret_cast<const int*>(base + o_g[gi * kArr + 2]);
+    gp.gemm_order = reinterpret_cast<const int*>(base + o_g[gi * kArr + 3]);
+    gp.gemm_prefix = reinterpret_cast<const int*>(base + o_g[gi * kArr + 4]);
+    gp.square_prefix = reinterpret_cast<const int*>(base + o_g[gi * kArr + 5]);
   }
   P->clip = reinterpret_cast<float*>(wsb + L.clip);
   P->d_mats = reinterpret_cast<const MatDesc*>(base + o_desc);
@@ -555,19 +687,69 @@ int get_plan(const std::vector<MatIn>& in, int steps, void* ws, int dev, Plan** 
   g_plans.emplace_front(std::move(P));
   Plan* plan = g_plans.front().get();
   while (g_plans.size() > kMaxPlans) {
-    cudaDeviceSynchronize();   // an evicted plan may still be read by queued kernels
+    // An evicted plan may still be read by queued kernels: its memory is
+    // freed in stream order after the latest work that used it.
+    Plan& old = *g_plans.back();
+    if (old.dmem) {
+      cudaStreamWaitEvent(st, old.last, 0);
+      cudaFreeAsync(old.dmem, st);
+      old.dmem = nullptr;
+    }
     g_plans.pop_back();
   }
   *out = plan;
   return DMUON_OK;
 }
 
+// Before a plan's kernels run on `st`: order after the plan's latest use on
+// another stream, then write the caller's addresses where they differ from
+// the ones the descriptors hold.
+int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  if (P.last_st != st) e = cudaStreamWaitEvent(st, P.last, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  std::unique_ptr<PatchParams> pp;
+  auto flush = [&]() {
+    if (!pp || pp->n == 0) return;
+    ++g_launches;
+    patch_kernel<<<1, 256, 0, st>>>(*pp);
+    pp->n = 0;
+  };
+  for (size_t i = 0; i < in.size(); ++i) {
+    const int d = P.desc_of[i];
+    const PtrSet now = ptrs_of(in[i]);
+    if (now == P.cur[d]) continue;
+    if (!pp) {
+      pp.reset(new PatchParams());
+      pp->mats = const_cast<MatDesc*>(P.d_mats);
+      pp->n = 0;
+    }
+    PatchEntry& en = pp->e[pp->n++];
+    en.W = now.W;
+    en.G = now.G;
+    en.buf = now.buf;
+    en.index = d;
+    en.vec4 = now.vec4;
+    P.cur[d] = now;
+    if (pp->n == kPatchMax) flush();
+  }
+  flush();
+  return DMUON_OK;
+}
+
+// After a plan's kernels were enqueued on `st`.
+int finish_plan(Plan& P, cudaStream_t st) {
+  cudaError_t e = cudaEventRecord(P.last, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  P.last_st = st;
+  return DMUON_OK;
+}
+
 // ------------------------------------------------------------------ launch
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per bounded device wait
 
-// Launch bookkeeping: a process-wide launch counter and, when enabled,
-// CUDA-event brackets around each launch for per-kernel device time.
-int64_t g_launches = 0;
+// Launch bookkeeping: a process-wide launch counter (g_launches, above) and,
+// when enabled, CUDA-event brackets around each launch for per-kernel device time.
 bool g_timing = false;
 struct Bracket {
   cudaEvent_t a, b;
@@ -592,7 +774,8 @@ cudaEvent_t pool_event() {
 // NVTX range names of the kernel kinds (a timeline tool shows every launch;
 // without one attached the calls cost next to nothing).
 const char* const kKindNames[DMUON_KERNEL_KINDS] = {"dmuon prologue", "dmuon finalize", "dmuon syrk",
-                                                    "dmuon gemm", "dmuon apply", "dmuon adamw"};
+                                                    "dmuon gemm",     "dmuon apply",    "dmuon adamw",
+                                                    "dmuon clip",     "dmuon square"};
 
 struct LaunchScope {
   cudaStream_t st;
@@ -677,8 +860,10 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   np.nmat = g.nmat;
   np.lr = lr;
   np.wd = wd;
+  np.quintic = P.quintic ? 1 : 0;
   np.ca = o.ca;
-  np.cb = o.cb;
+  np.cb = P.quintic ? 1.0f : o.cb;   // quintic: X <- a X + P X with P = b A + c A A
+  np.cc = 0.0f;
   np.err = d.err;
   np.wait_limit_ns = kWaitLimitNs;
   for (int s = 0; s < steps; ++s) {
@@ -691,6 +876,16 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     {
       LaunchScope ls(st, DMUON_KERNEL_SYRK);
       launch_ns_stage<kSyrk, E>(np, d, st);
+    }
+    if (P.quintic) {
+      NsParams sq = np;
+      sq.cb = o.cb;
+      sq.cc = o.cc;
+      sq.order = g.gemm_order;
+      sq.tile_prefix = g.square_prefix;
+      sq.ntiles = g.square_tiles;
+      LaunchScope ls(st, DMUON_KERNEL_SQUARE);
+      launch_ns_stage<kSquare, E>(sq, d, st);
     }
     np.order = g.gemm_order;
     np.tile_prefix = g.gemm_prefix;
@@ -740,16 +935,17 @@ int current_device(int* dev) {
   return device_setup(*dev);
 }
 
+// The library's scratch for calls on `st` that bring none: grown in stream
+// order (the old region is freed after the work queued on `st` before it).
 int arena_get(int dev, cudaStream_t st, size_t bytes, void** out) {
   Arena& a = g_arenas[std::make_pair(dev, st)];
   if (a.bytes < bytes) {
     if (a.ptr) {
-      cudaStreamSynchronize(st);
-      cudaFree(a.ptr);
+      cudaFreeAsync(a.ptr, st);
       a.ptr = nullptr;
       a.bytes = 0;
     }
-    cudaError_t e = lib_malloc(&a.ptr, bytes);
+    cudaError_t e = lib_malloc_async(&a.ptr, bytes, g_dev[dev].pool, st);
     if (e != cudaSuccess) {
       a.ptr = nullptr;
       cudaGetLastError();
@@ -833,6 +1029,21 @@ std::vector<int> step_groups(const std::vector<MatIn>& in, bool clipping) {
   return bnd;
 }
 
+// Every tensor address of a call must be device memory: checked on the host
+// before anything is enqueued (a kernel given host memory would fault).
+int check_call_pointers(int dev, const std::vector<MatIn>& in) {
+  for (size_t i = 0; i < in.size(); ++i) {
+    const MatIn& x = in[i];
+    int r = check_device_ptr(dev, x.W, static_cast<int>(i), x.mode == kModeMuon ? "the parameter" : "X");
+    if (r == DMUON_OK && x.G != x.W) r = check_device_ptr(dev, x.G, static_cast<int>(i), "the gradient");
+    if (r == DMUON_OK) r = check_device_ptr(dev, x.buf, static_cast<int>(i), "the momentum buffer");
+    for (size_t q = 0; q < x.gr.size() && r == DMUON_OK; ++q)
+      r = check_device_ptr(dev, x.gr[q], static_cast<int>(i), "a rank's gradient");
+    if (r != DMUON_OK) return r;
+  }
+  return DMUON_OK;
+}
+
 int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, const StepOpts& o,
         cudaStream_t st) {
   const int steps = o.steps;
@@ -841,13 +1052,15 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
   int dev = 0;
   int r = current_device(&dev);
   if (r != DMUON_OK) return r;
+  r = check_call_pointers(dev, in);
+  if (r != DMUON_OK) return r;
   const std::vector<int> bnd = step_groups(in, o.max_norm > 0.0f);
   const int ng = static_cast<int>(bnd.size()) - 1;
   std::vector<std::vector<MatIn>> sub(ng);
   size_t need = 0;
   for (int gi = 0; gi < ng; ++gi) {
     sub[gi].assign(in.begin() + bnd[gi], in.begin() + bnd[gi + 1]);
-    need = std::max(need, make_layout(sub[gi], steps).bytes);
+    need = std::max(need, make_layout(sub[gi], steps, o.cc != 0.0f).bytes);
   }
   if (own_ws) {
     r = arena_get(dev, st, need, &ws);
@@ -859,14 +1072,19 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
                   ws_bytes, need);
     if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
-  // Every group's plan before anything is enqueued.
+  // Every group's plan before any kernel of the call is enqueued (a new
+  // plan's upload writes library memory only).  Groups with the same shapes
+  // share one plan; its descriptors are patched with each group's addresses
+  // in stream order.
   std::vector<Plan*> plans(ng, nullptr);
   for (int gi = 0; gi < ng; ++gi) {
-    r = get_plan(sub[gi], steps, ws, dev, &plans[gi]);
+    r = get_plan(sub[gi], steps, o.cc != 0.0f, ws, dev, st, &plans[gi]);
     if (r != DMUON_OK) return r;
   }
   for (int gi = 0; gi < ng; ++gi) {
-    r = launch_plan(*plans[gi], o, st);
+    r = prepare_plan(*plans[gi], sub[gi], st);
+    if (r == DMUON_OK) r = launch_plan(*plans[gi], o, st);
+    if (r == DMUON_OK) r = finish_plan(*plans[gi], st);
     if (r != DMUON_OK) return r;
   }
   return DMUON_OK;
@@ -874,7 +1092,7 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
 
 int check_opts(const StepOpts& o) {
   if (!std::isfinite(o.lr) || !std::isfinite(o.mu) || !std::isfinite(o.wd) || !std::isfinite(o.ca) ||
-      !std::isfinite(o.cb))
+      !std::isfinite(o.cb) || !std::isfinite(o.cc))
     return fail(DMUON_ERR_INVALID_ARG, "lr, momentum, weight_decay and the NS coefficients must be finite");
   if (!(o.max_norm >= 0.0f) || !std::isfinite(o.max_norm))
     return fail(DMUON_ERR_INVALID_ARG, "max_grad_norm must be finite and >= 0");
@@ -991,6 +1209,8 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
   int dev = 0;
   int r = current_device(&dev);
   if (r != DMUON_OK) return r;
+  r = check_call_pointers(dev, in);
+  if (r != DMUON_OK) return r;
   const int n = static_cast<int>(in.size());
   std::vector<size_t> gb(n), pb(n);
   size_t total = 0;
@@ -1012,7 +1232,7 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
   size_t need = 0;
   for (int c = 0; c < nc; ++c) {
     sub[c].assign(in.begin() + bnd[c], in.begin() + bnd[c + 1]);
-    need = std::max(need, make_layout(sub[c], o.steps).bytes);
+    need = std::max(need, make_layout(sub[c], o.steps, o.cc != 0.0f).bytes);
   }
   if (own_ws) {
     r = arena_get(dev, st, need, &ws);
@@ -1024,11 +1244,12 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
                   ws_bytes, need);
     if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
-  // Every group's plan before anything is enqueued.  The cache holds more
-  // plans than DMUON_MAX_CHUNKS, so none of these is evicted by the others.
+  // Every group's plan before any copy is enqueued (a new plan's upload
+  // writes library memory only).  The cache holds more plans than
+  // DMUON_MAX_CHUNKS, so none of these is evicted by the others.
   std::vector<Plan*> plans(nc, nullptr);
   for (int c = 0; c < nc; ++c) {
-    r = get_plan(sub[c], o.steps, ws, dev, &plans[c]);
+    r = get_plan(sub[c], o.steps, o.cc != 0.0f, ws, dev, st, &plans[c]);
     if (r != DMUON_OK) return r;
   }
   CopyLanes* L = nullptr;
@@ -1049,7 +1270,9 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
   for (int c = 0; c < nc; ++c) {
     e = cudaStreamWaitEvent(st, L->ev[c], 0);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
-    r = launch_plan(*plans[c], o, st);
+    r = prepare_plan(*plans[c], sub[c], st);
+    if (r == DMUON_OK) r = launch_plan(*plans[c], o, st);
+    if (r == DMUON_OK) r = finish_plan(*plans[c], st);
     if (r != DMUON_OK) return r;
     e = cudaEventRecord(L->ev[DMUON_MAX_CHUNKS + c], st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(L->down, L->ev[DMUON_MAX_CHUNKS + c], 0);
@@ -1098,6 +1321,37 @@ int dmuon_muon_step_batched(void* const params[], const void* const grads[], flo
   return run(in, nullptr, 0, true, o, reinterpret_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace dmuon {
+namespace {
+// Options as the caller passed them.  The struct grew by ns_c at its end; a
+// caller built against the earlier layout passes the shorter size and gets
+// the cubic step.
+constexpr size_t kOptsSizeNoQuintic = offsetof(dmuon_step_options, ns_c);
+
+int read_opts(const dmuon_step_options* opts, StepOpts* o) {
+  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
+  if (opts->struct_size != sizeof(dmuon_step_options) && opts->struct_size != kOptsSizeNoQuintic)
+    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
+                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
+  *o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
+  o->ca = opts->ns_a;
+  o->cb = opts->ns_b;
+  o->cc = opts->struct_size == sizeof(dmuon_step_options) ? opts->ns_c : 0.0f;
+  o->lr_scale = opts->lr_scale;
+  o->max_norm = opts->max_grad_norm;
+  o->norm_out = opts->grad_norm_out;
+  int r = check_opts(*o);
+  if (r != DMUON_OK) return r;
+  if (o->norm_out && !aligned(o->norm_out, 4)) return fail(DMUON_ERR_INVALID_ARG, "grad_norm_out misaligned");
+  return DMUON_OK;
+}
+}  // namespace
+}  // namespace dmuon
+
+extern "C" {
+
 void dmuon_step_options_default(dmuon_step_options* o) {
   if (!o) return;
   std::memset(o, 0, sizeof(*o));
@@ -1112,25 +1366,16 @@ void dmuon_step_options_default(dmuon_step_options* o) {
   o->lr_scale = DMUON_LR_PLAIN;
   o->max_grad_norm = 0.0f;
   o->grad_norm_out = nullptr;
+  o->ns_c = 0.0f;
 }
 
 int dmuon_muon_step_batched_opts(void* const params[], const void* const grads[], float* const bufs[],
                                  const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
                                  void* workspace, size_t ws_bytes, dmuon_stream_t stream) {
   t_last_error.clear();
-  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
-  if (opts->struct_size != sizeof(dmuon_step_options))
-    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
-                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
-  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
-  o.ca = opts->ns_a;
-  o.cb = opts->ns_b;
-  o.lr_scale = opts->lr_scale;
-  o.max_norm = opts->max_grad_norm;
-  o.norm_out = opts->grad_norm_out;
-  int r = check_opts(o);
+  StepOpts o;
+  int r = read_opts(opts, &o);
   if (r != DMUON_OK) return r;
-  if (o.norm_out && !aligned(o.norm_out, 4)) return fail(DMUON_ERR_INVALID_ARG, "grad_norm_out misaligned");
   std::vector<MatIn> in;
   r = gather(params, grads, bufs, shapes, count, opts->ns_steps, o.lr_scale, &in);
   if (r != DMUON_OK) return r;
@@ -1142,20 +1387,10 @@ int dmuon_muon_step_batched_reduce(void* const params[], const void* const grads
                                    const dmuon_step_options* opts, void* workspace, size_t ws_bytes,
                                    dmuon_stream_t stream) {
   t_last_error.clear();
-  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
-  if (opts->struct_size != sizeof(dmuon_step_options))
-    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
-                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
-  if (world < 1 || world > 64) return fail(DMUON_ERR_INVALID_ARG, "world must be in [1, 64]");
-  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
-  o.ca = opts->ns_a;
-  o.cb = opts->ns_b;
-  o.lr_scale = opts->lr_scale;
-  o.max_norm = opts->max_grad_norm;
-  o.norm_out = opts->grad_norm_out;
-  int r = check_opts(o);
+  StepOpts o;
+  int r = read_opts(opts, &o);
   if (r != DMUON_OK) return r;
-  if (o.norm_out && !aligned(o.norm_out, 4)) return fail(DMUON_ERR_INVALID_ARG, "grad_norm_out misaligned");
+  if (world < 1 || world > 64) return fail(DMUON_ERR_INVALID_ARG, "world must be in [1, 64]");
   if (count > 0 && !grads) return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
   // Rank 0's pointers stand for the gradients in the argument checks.
   std::vector<MatIn> in;
@@ -1186,17 +1421,10 @@ int dmuon_muon_step_batched_host(void* const params[], void* const grads[], floa
                                  const dmuon_shape shapes[], int count, const dmuon_step_options* opts,
                                  int chunks, void* workspace, size_t ws_bytes, dmuon_stream_t stream) {
   t_last_error.clear();
-  if (!opts) return fail(DMUON_ERR_INVALID_ARG, "NULL options");
-  if (opts->struct_size != sizeof(dmuon_step_options))
-    return fail(DMUON_ERR_INVALID_ARG, "options.struct_size is %zu, this library expects %zu (use "
-                "dmuon_step_options_default)", opts->struct_size, sizeof(dmuon_step_options));
-  StepOpts o = plain_opts(opts->lr, opts->momentum, opts->nesterov, opts->weight_decay, opts->ns_steps);
-  o.ca = opts->ns_a;
-  o.cb = opts->ns_b;
-  o.lr_scale = opts->lr_scale;
-  int r = check_opts(o);
+  StepOpts o;
+  int r = read_opts(opts, &o);
   if (r != DMUON_OK) return r;
-  if (opts->max_grad_norm != 0.0f)
+  if (o.max_norm != 0.0f)
     return fail(DMUON_ERR_UNSUPPORTED, "gradient clipping needs every gradient before the first "
                 "update; use dmuon_muon_step_batched_opts");
   if (chunks > DMUON_MAX_CHUNKS)
@@ -1245,6 +1473,25 @@ size_t dmuon_workspace_bytes(const dmuon_shape shapes[], int count, int ns_steps
     if (x.rows < 1 || x.cols < 1 || (x.pdt != DMUON_BF16 && x.pdt != DMUON_F32)) return 0;
   }
   return make_layout(in, ns_steps).bytes;
+}
+
+size_t dmuon_workspace_bytes_opts(const dmuon_shape shapes[], int count, const dmuon_step_options* opts) {
+  if (!opts || (opts->struct_size != sizeof(dmuon_step_options) && opts->struct_size != kOptsSizeNoQuintic))
+    return 0;
+  const int steps = opts->ns_steps;
+  if (count <= 0 || !shapes || steps < 0 || steps > DMUON_MAX_STEPS) return 0;
+  const bool quintic = opts->struct_size == sizeof(dmuon_step_options) && opts->ns_c != 0.0f;
+  std::vector<MatIn> in(count);
+  for (int i = 0; i < count; ++i) {
+    MatIn& x = in[i];
+    x.rows = shapes[i].rows;
+    x.cols = shapes[i].cols;
+    x.pdt = shapes[i].param_dtype;
+    x.gdt = shapes[i].grad_dtype;
+    x.mode = kModeMuon;
+    if (x.rows < 1 || x.cols < 1 || (x.pdt != DMUON_BF16 && x.pdt != DMUON_F32)) return 0;
+  }
+  return make_layout(in, steps, quintic).bytes;
 }
 
 static int ortho_input(void* X, int64_t m, int64_t n, int steps, int dtype, std::vector<MatIn>* in) {
@@ -1323,6 +1570,21 @@ void dmuon_release_cache(void) {
   for (auto& kv : g_arenas)
     if (kv.second.ptr) cudaFree(kv.second.ptr);
   g_arenas.clear();
+  for (DeviceInfo& d : g_dev)
+    if (d.pool) cudaMemPoolTrimTo(d.pool, 0);
+}
+
+int64_t dmuon_plan_builds(void) {
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  return g_plan_builds;
+}
+
+int dmuon_debug_check_pointer(const void* p) {
+  t_last_error.clear();
+  if (p == nullptr) return fail(DMUON_ERR_INVALID_ARG, "NULL pointer");
+  const int r = classify_pointer(p);
+  if (r != DMUON_OK) return fail(r, "not device memory");
+  return DMUON_OK;
 }
 
 int dmuon_adamw_step_batched(void* const params[], const void* const grads[], float* const exp_avgs[],
@@ -1394,6 +1656,132 @@ int dmuon_adamw_step_batched(void* const params[], const void* const grads[], fl
     LaunchScope ls(st, DMUON_KERNEL_ADAMW);
     adamw_kernel<<<grid, kPThreads, 0, st>>>(*ap);
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return DMUON_OK;
+}
+
+static int clip_check(const dmuon_grad_desc descs[], int count, int nseg) {
+  if (count < 0) return fail(DMUON_ERR_INVALID_ARG, "count must be >= 0");
+  if (nseg < 1 || nseg > DMUON_MAX_SEGMENTS)
+    return fail(DMUON_ERR_INVALID_ARG, "nseg must be in [1, %d]", DMUON_MAX_SEGMENTS);
+  if (count > 0 && !descs) return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  for (int i = 0; i < count; ++i) {
+    const dmuon_grad_desc& d = descs[i];
+    if (d.numel < 1) return fail(DMUON_ERR_INVALID_ARG, "tensor %d: numel must be >= 1", i);
+    if (d.dtype != DMUON_BF16 && d.dtype != DMUON_F32)
+      return fail(DMUON_ERR_UNSUPPORTED, "tensor %d: dtype must be DMUON_BF16 or DMUON_F32", i);
+    if (d.segment < 0 || d.segment >= nseg)
+      return fail(DMUON_ERR_INVALID_ARG, "tensor %d: segment %d is outside [0, %d)", i, d.segment, nseg);
+  }
+  return DMUON_OK;
+}
+
+// Scratch of one clip call: one fp64 partial per 8192-element item, then the
+// per-segment coefficients.
+static size_t clip_scratch_bytes(const dmuon_grad_desc descs[], int count, int nseg, size_t* coef_off) {
+  int64_t items = 0;
+  for (int i = 0; i < count; ++i) items += cdiv(descs[i].numel, kClipChunk);
+  const size_t off = align_up(sizeof(double) * static_cast<size_t>(std::max<int64_t>(items, 1)), 256);
+  if (coef_off) *coef_off = off;
+  return off + align_up(sizeof(float) * nseg, 256);
+}
+
+size_t dmuon_clip_workspace_bytes(const dmuon_grad_desc descs[], int count, int nseg) {
+  if (clip_check(descs, count, nseg) != DMUON_OK) return 0;
+  return clip_scratch_bytes(descs, count, nseg, nullptr);
+}
+
+int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc descs[], int count,
+                                 const float max_norms[], int nseg, float* norms_out, float* coefs_out,
+                                 void* workspace, size_t ws_bytes, dmuon_stream_t stream) {
+  t_last_error.clear();
+  int r = clip_check(descs, count, nseg);
+  if (r != DMUON_OK) return r;
+  if (count > 0 && !grads) return fail(DMUON_ERR_INVALID_ARG, "NULL array argument");
+  if (!max_norms) return fail(DMUON_ERR_INVALID_ARG, "NULL max_norms");
+  for (int s = 0; s < nseg; ++s)
+    if (!(max_norms[s] > 0.0f))
+      return fail(DMUON_ERR_INVALID_ARG, "max_norms[%d] must be > 0 (+inf measures without clipping)", s);
+  if ((norms_out && !aligned(norms_out, 4)) || (coefs_out && !aligned(coefs_out, 4)))
+    return fail(DMUON_ERR_INVALID_ARG, "norms_out / coefs_out misaligned");
+  // Tensors with a gradient, sorted by segment (stable): each segment's work
+  // items form one contiguous range.
+  std::vector<int> idx;
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i]) continue;
+    if (!aligned(grads[i], elem_bytes(descs[i].dtype)))
+      return fail(DMUON_ERR_INVALID_ARG, "tensor %d: pointer not aligned to its element size", i);
+    idx.push_back(i);
+  }
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return descs[a].segment < descs[b].segment; });
+  std::vector<ClipTensor> ts(idx.size());
+  std::unique_ptr<ClipFinalizeParams> fp(new ClipFinalizeParams());
+  int64_t items = 0;
+  int seg = 0;
+  fp->seg_item0[0] = 0;
+  for (size_t k = 0; k < idx.size(); ++k) {
+    const dmuon_grad_desc& d = descs[idx[k]];
+    while (seg < d.segment) fp->seg_item0[++seg] = items;
+    ts[k].g = grads[idx[k]];
+    ts[k].numel = d.numel;
+    ts[k].item0 = items;
+    ts[k].seg = d.segment;
+    ts[k].bf16 = d.dtype == DMUON_BF16;
+    items += cdiv(d.numel, kClipChunk);
+  }
+  while (seg < nseg) fp->seg_item0[++seg] = items;
+  for (int s = 0; s < nseg; ++s) fp->max_norm[s] = max_norms[s];
+  size_t coef_off = 0;
+  const size_t need = clip_scratch_bytes(descs, count, nseg, &coef_off);
+
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  int dev = 0;
+  r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws) {
+    r = arena_get(dev, st, need, &ws);
+    if (r != DMUON_OK) return r;
+  } else {
+    if (ws_bytes < need)
+      return fail(DMUON_ERR_NO_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+    if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  double* partials = static_cast<double*>(ws);
+  float* coef = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + coef_off);
+  fp->partials = partials;
+  fp->coef = coef;
+  fp->norms_out = norms_out;
+  fp->coefs_out = coefs_out;
+  const int sms = g_dev[dev].sms;
+  std::unique_ptr<ClipBucketParams> cp(new ClipBucketParams());
+  cp->partials = partials;
+  cp->coef = coef;
+  // The tensors in launches of at most kClipMaxTensors, for the norm pass and
+  // then (after the coefficients) for the scale pass.
+  auto launch_all = [&](bool scale) {
+    for (size_t first = 0; first < ts.size(); first += kClipMaxTensors) {
+      const int n = static_cast<int>(std::min<size_t>(kClipMaxTensors, ts.size() - first));
+      for (int k = 0; k < n; ++k) cp->t[k] = ts[first + k];
+      cp->count = n;
+      cp->item_begin = ts[first].item0;
+      cp->item_end = (first + n < ts.size()) ? ts[first + n].item0 : items;
+      const int64_t ni = cp->item_end - cp->item_begin;
+      if (ni <= 0) continue;
+      const int grid = static_cast<int>(std::min<int64_t>(ni, static_cast<int64_t>(sms) * 8));
+      LaunchScope ls(st, DMUON_KERNEL_CLIP);
+      if (scale) clip_scale_kernel<<<grid, kPThreads, 0, st>>>(*cp);
+      else clip_norm_kernel<<<grid, kPThreads, 0, st>>>(*cp);
+    }
+  };
+  launch_all(false);
+  {
+    LaunchScope ls(st, DMUON_KERNEL_CLIP);
+    clip_finalize_kernel<<<nseg, 256, 0, st>>>(*fp);
+  }
+  launch_all(true);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return DMUON_OK;
@@ -1584,6 +1972,10 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   sp.pprefix[1] = ml.ptiles;
   const int BK = 64;   // bf16: 128-byte K slices
   bool okm = true;
+  // As in the regular plans: the GEMM's B operand in one 3-D load when n % 64 == 0.
+  d.b3d = (ml.n % 64 == 0) ? 1 : 0;
+  for (int b = 0; b < 2 && d.b3d; ++b)
+    if (d.X[b] && !encode_mn3d(&sp.maps.xmn[b], d.X[b], ml.n, ml.m, ml.ldx)) d.b3d = 0;
   for (int b = 0; b < 2; ++b) {
     void* xb = d.X[b];
     if (!xb) {
@@ -1592,14 +1984,15 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     }
     okm &= encode_2d(&sp.maps.xk[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBM);
     okm &= encode_2d(&sp.maps.xkw[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBN);
-    okm &= encode_2d(&sp.maps.xmn[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, BK);
+    if (!d.b3d) okm &= encode_2d(&sp.maps.xmn[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, BK);
   }
   if (d.A) okm &= encode_2d(&sp.maps.a, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, kBM);
   if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
-  // Upload on the caller's stream: ordered after any earlier call on it.
-  cudaError_t e = cudaMemcpyAsync(base, &sp, sizeof(sp), cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return cuda_fail(e, "uploading the launch description");
+  // The launch description travels as kernel parameters of an upload kernel
+  // on the caller's stream: ordered after any earlier call on it, no host
+  // staging memory.  The stage kernels acquire the tensor maps before use.
+  enqueue_upload(base, reinterpret_cast<const uint8_t*>(&sp), sizeof(sp), st);
   const StaticPlan* dsp = reinterpret_cast<const StaticPlan*>(base);
 
   const DeviceInfo& di = g_dev[dev];
@@ -1632,6 +2025,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     np.wd = 0.0f;
     np.ca = 1.5f;
     np.cb = -0.5f;
+    np.cc = 0.0f;
+    np.quintic = 0;
     np.err = di.err;
     np.wait_limit_ns = kWaitLimitNs;
     for (int s = 0; s < steps; ++s) {
@@ -1647,7 +2042,7 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
       g_launches += 2;
     }
   }
-  e = cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return DMUON_OK;
 }

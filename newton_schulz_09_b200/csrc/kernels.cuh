@@ -8,12 +8,15 @@
 //   ns_stage_kernel     one Newton-Schulz stage for every matrix of a group
 //                       in one persistent launch:
 //                         SYRK  A = s^2 X X^T  (upper tiles, mirrored store)
+//                         SQUARE P = b A + c A A  (quintic coefficients only)
 //                         GEMM  X' = c (1.5 X - 0.5 A X), or on the last step
 //                               the weight update / output write.   [tensor]
 //   apply_kernel        the update for ns_steps == 0 (X = s M).
 //   grad_norm_kernel,   Muon-only global-norm gradient clipping: per-item
 //   clip_coef_kernel    sums of g^2 (fp64), then the clip coefficient.
 //   adamw_kernel        AdamW of the parameters Muon does not orthogonalise.
+//   clip_*_kernel       per-segment gradient clipping (norms, coefficients,
+//                       in-place scaling) of several gradient groups.
 //   wait_timeout_kernel test kernel of the bounded-wait path.
 //
 // Sources: DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销",
@@ -46,7 +49,8 @@ static_assert(kNsSmemBytes <= 232448, "exceeds the 227 KB of shared memory per b
 constexpr int kPThreads = 256;
 
 enum { kModeMuon = 0, kModeOrtho = 1 };
-enum { kSyrk = 0, kGemm = 1 };
+// kSquare: P = b A + c A A over upper tiles (quintic coefficients), A symmetric.
+enum { kSyrk = 0, kGemm = 1, kSquare = 2 };
 
 // One matrix of a launch group.  X is the m x n "wide" view (m <= n) of the
 // parameter: X = M when rows <= cols, X = M^T otherwise (T = 1), stored
@@ -60,6 +64,7 @@ struct MatDesc {
   void* X[2];          // ping-pong iterates
   void* Xop[2];        // tensor-core operand copies of X (tf32-rounded for fp32; == X for bf16)
   void* A;             // Gram matrix m x m
+  void* P;             // quintic coefficients: b A + c A A (m x m, pitch lda), else nullptr
   float* scale;        // s = 1 / (||M||_F + 1e-7), written by finalize_kernel
   float lr_mult;       // per-matrix multiplier of lr (1 on the pages' update)
   int m, n, T;
@@ -78,6 +83,8 @@ struct alignas(64) MatMaps {
   CUtensorMap xmn[2];  // Xop as MN-major operand, box (128 B of N) x (BK rows of K); with b3d a
                        // 3-D view {64 columns, rows, column blocks of 64} and a box of 4 blocks
   CUtensorMap a;       // A as K-major operand, box (128 B of K) x 128 rows
+  CUtensorMap aw;      // A, box (128 B of K) x 256 rows: the B operand of A A in one load
+  CUtensorMap p;       // P as K-major operand (the GEMM's A operand in quintic mode)
 };
 
 struct NsParams {
@@ -91,7 +98,9 @@ struct NsParams {
   int first;               // fold s into this stage (first NS step)
   int last;                // GEMM writes the final result (last NS step)
   float lr, wd;            // update scalars (used when last)
-  float ca, cb;            // cubic coefficients: X <- ca X + cb (X X^T) X
+  float ca, cb;            // GEMM: X <- ca X + cb (A or P) X; SQUARE: P = cb A + cc A A
+  float cc;
+  int quintic;             // GEMM reads P instead of A
   int* err;                // device error word
   uint64_t wait_limit_ns;
 };
@@ -219,9 +228,9 @@ __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
   const int local = t - __ldg(p.tile_prefix + slot);
   const MatDesc& md = p.mats[ti.mi];
   ti.half = 0;
-  if (kMode == kSyrk) {
+  if (kMode == kSyrk || kMode == kSquare) {
     syrk_tile_coords(local, ti.tm, ti.tn);
-    ti.nkb = (md.n + BK - 1) / BK;
+    ti.nkb = ((kMode == kSyrk ? md.n : md.m) + BK - 1) / BK;
     ti.half = (ti.tm == 2 * ti.tn + 1) ? 1 : 0;
   } else {
     const int nI = (md.m + kBM - 1) / kBM;
@@ -255,6 +264,7 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
     const bool leader = (warp == 2 && lane == 0);
     int ld_t = t0, ld_q = 0;               // next quarter to load (leader only)
     uint32_t ld_g = 0;
+    int fenced = -1;                       // matrix whose maps the leader has acquired
     bool slot_busy[kEpiSlots] = {false, false};
     uint32_t slot_phase[kEpiSlots] = {0u, 0u};
     auto quarters_of = [&](const TileInfo& ti) -> int {
@@ -265,6 +275,11 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
     auto load_next = [&]() {
       if (ld_t >= p.ntiles) return;
       const TileInfo ti = decode_tile<kMode, BK>(p, ld_t);
+      if (ti.mi != fenced) {
+        tensormap_acquire_gpu(&p.maps[ti.mi].xk[p.cur]);
+        tensormap_acquire_gpu(&p.maps[ti.mi].xk[p.cur ^ 1]);
+        fenced = ti.mi;
+      }
       const int slot = static_cast<int>(ld_g & 1u);
       mbar_arrive_expect_tx(&xfull[slot], kEpiSlotBytes);
       tma_load_2d(epi + slot * kEpiSlotBytes, &p.maps[ti.mi].xk[p.cur], &xfull[slot],
@@ -349,9 +364,12 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(b * kBN);
     const int R = ti.tm * kBM + row_in_tile;
     const int m = md.m, n = md.n;
-    if (kMode == kSyrk) {
-      const float alpha = p.first ? s * s : 1.0f;
-      E* A = reinterpret_cast<E*>(md.A);
+    if (kMode == kSyrk || kMode == kSquare) {
+      // SYRK: A = s^2 X X^T on the first step.  SQUARE: P = cb A + cc A A,
+      // A read back in the tile's own rows and columns.
+      const float alpha = (kMode == kSquare) ? p.cc : (p.first ? s * s : 1.0f);
+      E* A = reinterpret_cast<E*>(kMode == kSquare ? md.P : md.A);
+      const E* Asrc = reinterpret_cast<const E*>(md.A);
       const int64_t lda = md.lda;
       const int nch = ti.half ? kBN / 64 : kBN / 32;
       const int col0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);
@@ -365,7 +383,21 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
         if (R < m && C0 < m && C0 + 31 >= R) {
           float y[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = op_round<E>(alpha * __uint_as_float(v[j]));
+          for (int j = 0; j < 32; ++j) y[j] = alpha * __uint_as_float(v[j]);
+          if (kMode == kSquare) {
+            float a0[32];
+            const E* srow = Asrc + static_cast<int64_t>(R) * lda + C0;
+            if (C0 + 32 <= m) {
+              load32<E>(srow, a0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) a0[j] = (C0 + j < m) ? to_f<E>(srow[j]) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = fmaf(p.cb, a0[j], y[j]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = op_round<E>(y[j]);
           E* arow = A + static_cast<int64_t>(R) * lda;
           if (C0 >= R && C0 + 32 <= m) {
             store32<E>(arow + C0, y);
@@ -497,7 +529,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   constexpr int KSTEPS = BK / MMA_K;        // = 4
   constexpr uint32_t FMT = (EB == 2) ? 1u : 2u;
   constexpr uint32_t IDESC = make_idesc(FMT, 0u, kMode == kGemm ? 1u : 0u, kBM, kBN);
-  constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);   // SYRK half tiles
+  constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);   // SYRK / SQUARE half tiles
   constexpr int NBOX_B = (kMode == kGemm) ? kBN / BK : 2;
   constexpr uint32_t BOX_B_BYTES = (kMode == kGemm) ? BK * 128 : kAStageBytes;
 
@@ -549,15 +581,21 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
     bool issued[kStages];
 #pragma unroll
     for (int s = 0; s < kStages; ++s) { issued[s] = false; issued_phase[s] = 0; }
+    int fenced = -1;     // matrix whose tensor maps this thread has acquired
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
       const TileInfo ti = decode_tile<kMode, BK>(p, t);
       const MatDesc& md = p.mats[ti.mi];
       const MatMaps& mp = p.maps[ti.mi];
-      const CUtensorMap* mapA = (kMode == kSyrk) ? &mp.xk[p.cur] : &mp.a;
-      const CUtensorMap* mapB = (kMode == kSyrk) ? &mp.xk[p.cur] : &mp.xmn[p.cur];
+      // SYRK: X X^T (both operands X, K-major).  SQUARE: A A (both operands A,
+      // K-major; A is symmetric, so A A = A A^T).  GEMM: A (or P) times X (MN-major).
+      const CUtensorMap* mapA = (kMode == kSyrk) ? &mp.xk[p.cur]
+                              : (kMode == kSquare) ? &mp.a : (p.quintic ? &mp.p : &mp.a);
+      const CUtensorMap* mapB = (kMode == kSyrk) ? &mp.xk[p.cur]
+                              : (kMode == kSquare) ? &mp.a : &mp.xmn[p.cur];
+      const CUtensorMap* mapBw = (kMode == kSyrk) ? &mp.xkw[p.cur] : &mp.aw;
       int nb = 0;
-      const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK B operand rows
-      if (kMode == kSyrk) {
+      const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK / SQUARE B operand rows
+      if (kMode == kSyrk || kMode == kSquare) {
         nb = (ti.half || ti.tn * kBN + 128 >= md.m) ? 1 : 2;
       } else if (md.b3d) {
         nb = NBOX_B;   // the 3-D box is always whole: blocks past the last column arrive as zeros
@@ -567,6 +605,14 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         if (nb > NBOX_B) nb = NBOX_B;
       }
       const uint32_t bytes = kAStageBytes + static_cast<uint32_t>(nb) * BOX_B_BYTES;
+      if (lane == 0 && ti.mi != fenced) {
+        // The maps were written by a kernel (plan upload): order that write
+        // before TMA reads them.
+        tensormap_acquire_gpu(mapA);
+        tensormap_acquire_gpu(mapB);
+        if (kMode != kGemm) tensormap_acquire_gpu(mapBw);
+        fenced = ti.mi;
+      }
       for (int kb = 0; kb < ti.nkb; ++kb) {
         bool w = mbar_wait(&empty[stage], phase ^ 1u, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
@@ -578,12 +624,12 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           if (kMode == kGemm && md.b3d) {
             // The four 64-column blocks of the tile in one load, same smem layout.
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
-          } else if (kMode == kSyrk && nb == 2) {
+          } else if (kMode != kGemm && nb == 2) {
             // Both 128-row halves of the B operand in one 256-row load.
-            tma_load_2d(b_dst, &mp.xkw[p.cur], &full[stage], kb * BK, b_row0);
+            tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
           } else {
             for (int j = 0; j < nb; ++j) {
-              if (kMode == kSyrk)
+              if (kMode != kGemm)
                 tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
               else
                 tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);
@@ -614,7 +660,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
-      const uint32_t idesc = (kMode == kSyrk && ti.half) ? IDESC_HALF : IDESC;
+      const uint32_t idesc = (kMode != kGemm && ti.half) ? IDESC_HALF : IDESC;
       for (int kb = 0; kb < ti.nkb; ++kb) {
         w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
@@ -628,7 +674,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
             // MN-major B: 16-bit operands use the 16-byte-unit swizzle (8-line
             // K groups); 32-bit operands must use 32-byte units (4-line groups).
             const uint64_t bd =
-                (kMode == kSyrk)
+                (kMode != kGemm)
                     ? sw128_desc(b_base + k * 32, 16, 1024)
                     : sw128_desc(b_base + k * MMA_K * 128, BK * 128, EB == 2 ? 1024 : 512,
                                  EB == 2 ? kSwizzle128B : kSwizzle128B32);
@@ -1268,6 +1314,190 @@ __global__ void __launch_bounds__(kPThreads) adamw_kernel(const __grid_constant_
       if (T.p_bf16) store8_x<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(T.p) + e, vp, valid, w);
       else store8_f32(reinterpret_cast<float*>(T.p) + e, vp, valid, w);
     }
+  }
+}
+
+// ======================================================================
+// Clipping of several gradient segments, each with its own norm and
+// coefficient (the training guide's fused regular / Muon / AdamW clipping,
+// "梯度裁剪").  Three kernels:
+//   clip_norm_kernel      one fp64 sum of squares per 8192-element work item
+//   clip_finalize_kernel  one block per segment: fixed-order sum of its
+//                         items, ||g||_s, c_s = fl32(min(1, max_s / (||g||_s + 1e-6)))
+//   clip_scale_kernel     g <- fl32(g * c_s), rounded to the storage type,
+//                         skipped for items of segments with c_s == 1
+// The host sorts the tensors by segment, so each segment's items are one
+// contiguous range.  The scale pass walks the items in reverse: the end of
+// the norm pass is still in L2 when it starts.
+// ======================================================================
+constexpr int kClipMaxTensors = 512;     // tensors per launch (kernel parameter space)
+constexpr int kClipMaxSegs = 64;
+constexpr int kClipChunk = 8192;         // elements per work item (256 threads x 4 x 8)
+
+struct ClipTensor {
+  void* g;
+  int64_t numel;
+  int64_t item0;     // first work item of this tensor (global numbering)
+  int32_t seg;
+  int32_t bf16;
+};
+
+struct ClipBucketParams {
+  ClipTensor t[kClipMaxTensors];
+  int count;            // tensors of this launch, in item order
+  int64_t item_begin;   // global items [item_begin, item_end) of this launch
+  int64_t item_end;
+  double* partials;     // one per global item
+  const float* coef;    // scale kernel: per-segment coefficient
+};
+
+struct ClipFinalizeParams {
+  int64_t seg_item0[kClipMaxSegs + 1];
+  float max_norm[kClipMaxSegs];
+  const double* partials;
+  float* coef;          // out: per-segment coefficient (scratch)
+  float* norms_out;     // out (optional): per-segment norm before clipping
+  float* coefs_out;     // out (optional): copy of the coefficients
+};
+
+__device__ __forceinline__ int clip_tensor_of(const ClipBucketParams& p, int64_t item) {
+  int lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.t[mid].item0 <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kPThreads) clip_norm_kernel(const __grid_constant__ ClipBucketParams p) {
+  __shared__ double red[kPThreads / 32];
+  const int tid = threadIdx.x;
+  for (int64_t it = p.item_begin + blockIdx.x; it < p.item_end; it += gridDim.x) {
+    const ClipTensor& T = p.t[clip_tensor_of(p, it)];
+    const int64_t base = (it - T.item0) * kClipChunk;
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(T.g) & 15) == 0;
+    // All four rounds' loads first, so 4 x 8 elements per thread are in flight.
+    float x[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
+      if (valid > 0) load8_any(T.g, T.bf16 != 0, e, aligned16 && valid == 8, valid, x[j]);
+      else
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[j][k] = 0.0f;
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss = fma(static_cast<double>(x[j][k]), static_cast<double>(x[j][k]), ss);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      double acc = 0.0;
+#pragma unroll
+      for (int w = 0; w < kPThreads / 32; ++w) acc += red[w];
+      p.partials[it] = acc;
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) clip_finalize_kernel(const __grid_constant__ ClipFinalizeParams p) {
+  __shared__ double red[8];
+  const int s = blockIdx.x;
+  double acc = 0.0;
+  for (int64_t i = p.seg_item0[s] + threadIdx.x; i < p.seg_item0[s + 1]; i += blockDim.x) acc += p.partials[i];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const double nrm = sqrt(tot);
+    const double c = static_cast<double>(p.max_norm[s]) / (nrm + 1e-6);
+    const float cf = static_cast<float>(c < 1.0 ? c : 1.0);   // a NaN norm gives 1
+    p.coef[s] = cf;
+    if (p.norms_out) p.norms_out[s] = static_cast<float>(nrm);
+    if (p.coefs_out) p.coefs_out[s] = cf;
+  }
+}
+
+__global__ void __launch_bounds__(kPThreads) clip_scale_kernel(const __grid_constant__ ClipBucketParams p) {
+  const int tid = threadIdx.x;
+  const int64_t n = p.item_end - p.item_begin;
+  for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
+    const int64_t it = p.item_end - 1 - r;
+    const ClipTensor& T = p.t[clip_tensor_of(p, it)];
+    const float c = p.coef[T.seg];
+    if (c == 1.0f) continue;          // the identity: nothing to write
+    const int64_t base = (it - T.item0) * kClipChunk;
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(T.g) & 15) == 0;
+    float x[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
+      if (valid > 0) load8_any(T.g, T.bf16 != 0, e, aligned16 && valid == 8, valid, x[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
+      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
+      if (valid <= 0) continue;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[j][k] = __fmul_rn(x[j][k], c);
+      const bool vec = aligned16 && valid == 8;
+      if (T.bf16) store8_x<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(T.g) + e, vec, valid, x[j]);
+      else store8_f32(reinterpret_cast<float*>(T.g) + e, vec, valid, x[j]);
+    }
+  }
+}
+
+// ======================================================================
+// Stream-ordered writes of library memory from kernel parameters (no host
+// staging, no synchronous copy):
+//   upload_kernel  copies up to kUploadWords 16-byte words (a launch plan:
+//                  descriptors, tensor maps, tile tables) to device memory;
+//                  the tensor maps among them are released to TMA.
+//   patch_kernel   writes the caller's tensor addresses of one call into the
+//                  matrix descriptors of a cached plan.
+// ======================================================================
+constexpr int kUploadWords = 1920;   // 30 KB of parameters
+struct UploadParams {
+  uint4* dst;
+  int nwords;
+  uint4 w[kUploadWords];
+};
+__global__ void __launch_bounds__(256) upload_kernel(const __grid_constant__ UploadParams p) {
+  for (int i = threadIdx.x; i < p.nwords; i += blockDim.x) p.dst[i] = p.w[i];
+  tensormap_release_gpu();
+}
+
+struct PatchEntry {
+  void* W;
+  const void* G;
+  float* buf;
+  int32_t index;    // matrix descriptor to patch
+  int32_t vec4;
+};
+constexpr int kPatchMax = 480;        // entries per launch (about 15 KB of parameters)
+struct PatchParams {
+  MatDesc* mats;
+  int n;
+  PatchEntry e[kPatchMax];
+};
+__global__ void __launch_bounds__(256) patch_kernel(const __grid_constant__ PatchParams p) {
+  for (int i = threadIdx.x; i < p.n; i += blockDim.x) {
+    MatDesc& d = p.mats[p.e[i].index];
+    d.W = p.e[i].W;
+    d.G = p.e[i].G;
+    d.buf = p.e[i].buf;
+    d.vec4 = p.e[i].vec4;
   }
 }
 

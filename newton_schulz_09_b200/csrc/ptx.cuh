@@ -144,6 +144,16 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
       : "memory");
   return out != 0;
 }
+// Tensor maps written by a kernel (generic stores) and read by TMA (the
+// tensor-map proxy): the writer releases after its stores, the reader
+// acquires on the map's 128 bytes before its first use.
+__device__ __forceinline__ void tensormap_release_gpu() {
+  asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
+}
+__device__ __forceinline__ void tensormap_acquire_gpu(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

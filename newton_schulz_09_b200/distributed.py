@@ -6,20 +6,29 @@ partition of the Newton-Schulz cost 3 m^2 n per step (the DMuon quick start,
 LPT partition; the blog's "参数分片减少 N-S 计算量": each rank runs N-S only
 on its share).  One step:
 
-1. the gradients are reduced to their owners (sum, then divided by the
-   number of ranks: the data-parallel mean), every reduction issued at once;
+1. every rank's gradient of a matrix reaches the matrix's owner unreduced
+   (point-to-point sends, one batch per chunk of the schedule below, all
+   batches issued at once); the caller's gradients are only read;
 2. every owner updates the matrices it owns in a few chunks, one batched
-   call each (only owners keep momentum buffers); a chunk waits only for its
-   own reductions, so later reductions run while earlier chunks compute;
+   call each (only owners keep momentum buffers).  The call is
+   ``dmuon_muon_step_batched_reduce``: its prologue forms the data-parallel
+   mean of the ranks' gradients itself, an fp32 sum in rank order and one
+   fp32 division by the number of ranks, so the mean does not depend on how
+   a collective happens to order or round its sums.  A chunk waits only for
+   its own transfers, so later transfers run while earlier chunks compute;
 3. every updated matrix is broadcast from its owner as soon as its chunk is
    done, while later chunks compute.
 
-All ranks issue the same collectives in the same order: every reduction,
-then the broadcasts chunk by chunk in one global schedule that interleaves
-the owners.  The collectives go through ``torch.distributed`` (NCCL on
-GPUs, gloo on CPUs), whose waits are stream-ordered on GPUs; the update
-itself is ``dmuon_muon_step_batched`` unless a step function is given (the
-CPU tests pass one).
+All ranks issue the same communication in the same order: the transfer
+batches, then the broadcasts, chunk by chunk in one global schedule that
+interleaves the owners.  It goes through ``torch.distributed`` (NCCL on
+GPUs, gloo on CPUs), whose waits are stream-ordered on GPUs.  The owner's
+update is the library's unless a function is given (the CPU tests pass the
+oracle).
+
+Memory: an owner keeps one receive buffer per other rank for each matrix it
+owns, (world - 1) times its share of the gradients, allocated on the first
+step and reused.
 """
 from __future__ import annotations
 
@@ -64,9 +73,10 @@ def imbalance(costs: Sequence[float], owner: Sequence[int], world: int) -> float
 StepFn = Callable[..., None]
 
 
-def _default_step(params, grads, bufs, **kw) -> None:
-    from . import dmuon_muon_step_batched
-    dmuon_muon_step_batched(params, grads, bufs, **kw)
+def _default_reduce_step(params, rank_grads, bufs, **kw) -> None:
+    """The owner's update on every rank's gradients (``rank_grads[r][k]``)."""
+    from . import dmuon_muon_step_batched_reduce
+    dmuon_muon_step_batched_reduce(params, rank_grads, bufs, **kw)
 
 
 def owner_chunks(owner: Sequence[int], numel: Sequence[int], world: int,
@@ -105,13 +115,18 @@ class OwnerPartitionedMuon:
     ``params`` are the full replicated weights (same on every rank).  Each
     rank allocates momentum buffers only for the matrices it owns.
 
-    ``grad_exchange``: "nccl" (default) reduces each gradient to its owner
-    with a collective.  "peer" keeps the gradients in symmetric memory
-    (``self.grads``, one view per parameter in the parameter's dtype, which
+    ``grad_exchange``: "nccl" (default) sends every rank's gradient to the
+    owner, whose update averages them.  "peer" keeps the gradients in
+    symmetric memory (``self.grads``, one view per parameter in the parameter's dtype, which
     the caller fills): after a stream-ordered barrier each owner reads every
     rank's gradient of the matrices it owns straight from peer memory inside
     its update (``dmuon_muon_step_batched_reduce``), so no reduced copy is
     written; the updated weights are then broadcast as in the NCCL mode.
+
+    ``step_fn(params, rank_grads, bufs, lr=, momentum=, nesterov=,
+    weight_decay=, ns_steps=)`` replaces the owner's update (the CPU tests
+    pass the oracle); ``rank_grads[r][k]`` is rank r's gradient of
+    ``params[k]``.
     """
 
     def __init__(self, params: Sequence[torch.Tensor], group=None, ns_steps: int = 5,
@@ -127,7 +142,8 @@ class OwnerPartitionedMuon:
         self.owned = [i for i, r in enumerate(self.owner) if r == self.rank]
         self.bufs = {i: torch.zeros(self.params[i].shape, dtype=torch.float32,
                                     device=self.params[i].device) for i in self.owned}
-        self.step_fn = step_fn or _default_step
+        self.step_fn = step_fn or _default_reduce_step
+        self._recv: dict = {}           # (matrix, rank) -> receive buffer on the owner
         self.imbalance = imbalance(costs, self.owner, self.world)
         self.chunks = owner_chunks(self.owner, [p.numel() for p in self.params], self.world,
                                    chunks_per_owner)
@@ -215,43 +231,63 @@ class OwnerPartitionedMuon:
         for w in bcast:
             w.wait()
 
+    def _recv_buffer(self, i: int, q: int, like: torch.Tensor) -> torch.Tensor:
+        key = (i, q)
+        b = self._recv.get(key)
+        if b is None or b.shape != like.shape or b.dtype != like.dtype or b.device != like.device:
+            b = torch.empty_like(like, memory_format=torch.contiguous_format)
+            self._recv[key] = b
+        return b
+
     @torch.no_grad()
     def step(self, grads: Sequence[Optional[torch.Tensor]], lr: float = 0.02,
              momentum: float = 0.95, nesterov: bool = True, weight_decay: float = 0.0) -> None:
         """One step.  ``grads`` are this rank's local gradients (None for a
-        parameter without gradient on every rank); they are overwritten by
-        the reduction on the owner.  On GPUs the call only enqueues work (the
-        collectives' waits are stream-ordered); the parameters are final once
-        the current stream reaches the end of the step."""
-        # 1. every reduction to its owner, all in flight at once
-        red = {}
-        for i, g in enumerate(grads):
-            if g is not None:
-                red[i] = dist.reduce(g, dst=self._global_rank(self.owner[i]), op=dist.ReduceOp.SUM,
-                                     group=self.group, async_op=True)
+        parameter without gradient on every rank); they are read, not
+        modified.  On GPUs the call only enqueues work (the collectives'
+        waits are stream-ordered); the parameters are final once the current
+        stream reaches the end of the step."""
+        # 1. per chunk of the schedule, one batch of point-to-point transfers:
+        # every other rank's gradient of the chunk's matrices to their owner
+        pending = {}
+        for r, c in self.schedule:
+            idx = [i for i in self.chunks[r][c] if grads[i] is not None]
+            if not idx or self.world == 1:
+                continue
+            ops = []
+            if r == self.rank:
+                for i in idx:
+                    for q in range(self.world):
+                        if q != self.rank:
+                            ops.append(dist.P2POp(dist.irecv, self._recv_buffer(i, q, grads[i]),
+                                                  self._global_rank(q), self.group))
+            else:
+                for i in idx:
+                    ops.append(dist.P2POp(dist.isend, grads[i].contiguous(), self._global_rank(r),
+                                          self.group))
+            pending[(r, c)] = dist.batch_isend_irecv(ops)
         # 2.-3. chunk by chunk in the global schedule: the owner updates its
-        # chunk once that chunk's reductions are done, then every rank takes
-        # part in the chunk's broadcasts
+        # chunk on every rank's gradients once they have arrived, then every
+        # rank takes part in the chunk's broadcasts
         bcast = []
         for r, c in self.schedule:
             idx = [i for i in self.chunks[r][c] if grads[i] is not None]
             if not idx:
                 continue
             if r == self.rank:
-                for i in idx:
-                    red[i].wait()
-                gs = [grads[i] for i in idx]
-                if self.world > 1:
-                    for g in gs:
-                        g.div_(self.world)
-                self.step_fn([self.params[i] for i in idx], gs, [self.bufs[i] for i in idx], lr=lr,
-                             momentum=momentum, nesterov=nesterov, weight_decay=weight_decay,
+                for w in pending.get((r, c), []):
+                    w.wait()
+                rank_grads = [[grads[i] if q == self.rank else self._recv[(i, q)] for i in idx]
+                              for q in range(self.world)]
+                self.step_fn([self.params[i] for i in idx], rank_grads, [self.bufs[i] for i in idx],
+                             lr=lr, momentum=momentum, nesterov=nesterov, weight_decay=weight_decay,
                              ns_steps=self.ns_steps)
             for i in idx:
                 bcast.append(dist.broadcast(self.params[i], src=self._global_rank(r), group=self.group,
                                             async_op=True))
-        for i, w in red.items():
-            if self.owner[i] != self.rank:
-                w.wait()
+        for (r, c), works in pending.items():
+            if r != self.rank:
+                for w in works:
+                    w.wait()
         for w in bcast:
             w.wait()

@@ -279,3 +279,56 @@ def test_missing_library_fails_loudly(monkeypatch):
         dm.dmuon_muon_step_batched([], [], [])
     with pytest.raises(RuntimeError, match="missing"):
         dm.dmuon_ns_orthogonalize(torch.zeros(4, 4, dtype=torch.bfloat16))
+
+
+def test_clip_buckets_argument_checks(lib):
+    D = (dm.DmuonGradDesc * 3)(dm.DmuonGradDesc(10000, dm.DMUON_BF16, 0),
+                               dm.DmuonGradDesc(5, dm.DMUON_F32, 2),
+                               dm.DmuonGradDesc(8192, dm.DMUON_BF16, 1))
+    # 10000 -> 2 items, 5 -> 1, 8192 -> 1: four fp64 partials (256 bytes) and
+    # three coefficients (256 bytes)
+    assert lib.dmuon_clip_workspace_bytes(D, 3, 3) == 512
+    assert lib.dmuon_clip_workspace_bytes(D, 3, 2) == 0          # segment 2 out of range
+    G = (ctypes.c_void_p * 3)(0x10000, 0x20000, 0x30000)
+    M = (ctypes.c_float * 3)(1.0, 1.0, 1.0)
+
+    def call(G=G, D=D, n=3, M=M, nseg=3):
+        return lib.dmuon_clip_grad_norm_buckets(G, D, n, M, nseg, None, None, None, 0, None)
+
+    assert call(nseg=0) == -1
+    assert call(nseg=dm.DMUON_MAX_SEGMENTS + 1) == -1
+    assert call(n=-1) == -1
+    assert call(nseg=2) == -1 and "segment 2" in dm.dmuon_last_error()
+    assert call(M=(ctypes.c_float * 3)(1.0, 0.0, 1.0)) == -1 and "max_norms[1]" in dm.dmuon_last_error()
+    assert call(M=(ctypes.c_float * 3)(1.0, float("nan"), 1.0)) == -1
+    bad = (dm.DmuonGradDesc * 1)(dm.DmuonGradDesc(0, dm.DMUON_BF16, 0))
+    assert call(D=bad, n=1, nseg=1) == -1
+    bad = (dm.DmuonGradDesc * 1)(dm.DmuonGradDesc(4, 9, 0))
+    assert call(D=bad, n=1, nseg=1) == -2
+    odd = (ctypes.c_void_p * 3)(0x10001, 0x20000, 0x30000)   # odd bf16 address
+    assert call(G=odd) == -1 and "aligned" in dm.dmuon_last_error()
+
+
+def test_options_struct_sizes_and_quintic_workspace(lib):
+    o = dm.DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    assert o.ns_c == 0.0
+    P, G, B = _ptrs(0x10000), _ptrs(None), _ptrs(0x30000)
+    S = _shapes((4, 4))
+    # a caller built before ns_c existed passes the shorter size: accepted
+    o.struct_size = dm.DmuonStepOptions.ns_c.offset
+    assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, ctypes.byref(o), None, 0, None) == 0
+    o.struct_size = ctypes.sizeof(dm.DmuonStepOptions) + 4
+    assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, ctypes.byref(o), None, 0, None) == -1
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    o.ns_c = float("inf")
+    assert lib.dmuon_muon_step_batched_opts(P, G, B, S, 1, ctypes.byref(o), None, 0, None) == -1
+    # workspace: cubic as dmuon_workspace_bytes; quintic adds P (m x lda) per matrix
+    S2 = _shapes((256, 512), (512, 256))
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    cubic = lib.dmuon_workspace_bytes_opts(S2, 2, ctypes.byref(o))
+    assert cubic == lib.dmuon_workspace_bytes(S2, 2, 5)
+    o.ns_c = 2.0315
+    assert lib.dmuon_workspace_bytes_opts(S2, 2, ctypes.byref(o)) == cubic + 2 * 256 * 256 * 2
+    o.ns_steps = 0
+    assert lib.dmuon_workspace_bytes_opts(S2, 2, ctypes.byref(o)) == lib.dmuon_workspace_bytes(S2, 2, 0)

@@ -1,9 +1,12 @@
-"""Owner-partitioned Muon over data-parallel ranks, on CPU (gloo, 2 ranks).
+"""Owner-partitioned Muon over data-parallel ranks, on CPU (gloo, 2-3 ranks).
 
-The per-owner update is the fp64 oracle (injected as the step function), so
-these tests check the partition, the reduction to owners, the owners' batched
-step and the broadcast: the result on every rank must equal one step of the
-oracle on the rank-averaged gradients.
+The per-owner update is the fp64 oracle (injected as the step function, with
+the oracle's rank mean: an fp32 sum in rank order, then one division), so
+these tests check the partition, the transfer of every rank's gradient to its
+owner in rank order, the owners' batched step and the broadcast: the result
+on every rank must equal one step of the oracle on the rank mean, bit for
+bit.  The gradients are random fp32 values whose sums round, so a different
+summation order or a reduction in another precision would show.
 """
 import os
 import socket
@@ -22,9 +25,10 @@ SHAPES = [(48, 96), (96, 48), (64, 64), (32, 128), (24, 40), (128, 32), (16, 16)
 HP = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.01)
 
 
-def oracle_step_fn(ps, gs, bs, *, lr, momentum, nesterov, weight_decay, ns_steps):
-    for p, g, b in zip(ps, gs, bs):
-        buf_new, X, W_new = oracle.muon_step(p.numpy(), g.numpy(), b.numpy(), lr=lr, momentum=momentum,
+def oracle_step_fn(ps, rank_grads, bs, *, lr, momentum, nesterov, weight_decay, ns_steps):
+    for k, (p, b) in enumerate(zip(ps, bs)):
+        g = oracle.rank_mean([rank_grads[r][k].numpy() for r in range(len(rank_grads))])
+        buf_new, X, W_new = oracle.muon_step(p.numpy(), g, b.numpy(), lr=lr, momentum=momentum,
                                              nesterov=nesterov, weight_decay=weight_decay,
                                              ns_steps=ns_steps)
         b.copy_(torch.from_numpy(buf_new))
@@ -37,10 +41,10 @@ def _params():
 
 
 def _grads(rank, step):
-    # small multiples of 2^-20: fp32 sums over ranks are exact in any order,
-    # so the mean is one rounding whatever order the reduction takes
+    # random fp32 values of varied magnitude: their sums over ranks round, so
+    # the mean depends on the order and precision of the sum
     gen = torch.Generator().manual_seed(1000 * step + rank)
-    gs = [torch.randint(-1000, 1001, s, generator=gen).float() * 2.0 ** -20 for s in SHAPES]
+    gs = [torch.randn(s, generator=gen) * 10.0 ** (-3 + rank) for s in SHAPES]
     gs[4] = None if step == 1 else gs[4]          # no gradient for one matrix on step 1
     return gs
 
@@ -51,9 +55,13 @@ def _worker(rank, world, port, out_dir):
     try:
         params = _params()
         opt = dmd.OwnerPartitionedMuon(params, ns_steps=3, step_fn=oracle_step_fn)
+        untouched = True
         for step in range(2):
-            opt.step(_grads(rank, step), **HP)
-        torch.save({"params": [p.clone() for p in params], "owner": opt.owner,
+            gs = _grads(rank, step)
+            g0 = [None if g is None else g.clone() for g in gs]
+            opt.step(gs, **HP)
+            untouched = untouched and all(a is None or torch.equal(a, b) for a, b in zip(gs, g0))
+        torch.save({"params": [p.clone() for p in params], "owner": opt.owner, "untouched": untouched,
                     "owned": opt.owned, "bufs": {i: b.clone() for i, b in opt.bufs.items()}},
                    os.path.join(out_dir, f"rank{rank}.pt"))
     finally:
@@ -135,7 +143,10 @@ def test_ranks_match_one_step_on_averaged_gradients(scratch_dir, world):
             assert torch.equal(a, b)
     # every matrix has exactly one owner, and only owners keep buffers
     assert sorted(sum((res[r]["owned"] for r in range(world)), [])) == list(range(len(SHAPES)))
-    # reference: two oracle steps on the mean gradient (exact fp32 sum, then / world)
+    # the callers' gradients are only read
+    assert all(res[r]["untouched"] for r in range(world))
+    # reference: two oracle steps on the oracle's rank mean (fp32 sum in rank
+    # order, then one division)
     W = [p.numpy().copy() for p in _params()]
     bufs = [np.zeros(s, np.float32) for s in SHAPES]
     for step in range(2):
@@ -143,7 +154,12 @@ def test_ranks_match_one_step_on_averaged_gradients(scratch_dir, world):
         for i in range(len(SHAPES)):
             if gr[0][i] is None:
                 continue
-            gm = (sum(g[i] for g in gr) / world).numpy()
+            gm = oracle.rank_mean([g[i].numpy() for g in gr])
+            # the gradients are not exactly summable: another order of the
+            # fp32 sum, or a sum in fp64, gives a different mean somewhere
+            wide = (sum(g[i].numpy().astype(np.float64) for g in gr) / world).astype(np.float32)
+            if world > 2:
+                assert not np.array_equal(gm, wide)
             bufs[i], _, Wn = oracle.muon_step(W[i], gm, bufs[i], ns_steps=3, **HP)
             W[i] = Wn.astype(np.float32)
     for i in range(len(SHAPES)):

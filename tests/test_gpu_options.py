@@ -112,3 +112,62 @@ def test_gradient_clipping(cuda_lib, max_norm):
     # gradients are read only
     for g, gh in zip(grads, g_host):
         assert np.array_equal(host(g), gh)
+
+
+QUINTIC = [(3.4445, -4.7750, 2.0315), (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0)]
+
+
+@pytest.mark.parametrize("coeffs", QUINTIC, ids=["jordan", "textbook"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("steps", [1, 5])
+def test_quintic_coefficients(cuda_lib, coeffs, dtype, steps):
+    """X <- a X + b A X + c A^2 X (A = X X^T): the SYRK, the symmetric square
+    P = b A + c A A and the GEMM X <- a X + P X, against the oracle's quintic
+    step; tall, square and multi-band wide shapes with ragged sizes."""
+    dm = cuda_lib
+    shapes = [(384, 1024), (1200, 264), (256, 256), (520, 600)]
+    params = [torch.zeros(s, dtype=dtype, device=DEV) for s in shapes]
+    grads = [_rand(s, dtype, 60 + i, 1e-3) for i, s in enumerate(shapes)]
+    bufs = [_rand(s, torch.float32, 70 + i, 1e-3) for i, s in enumerate(shapes)]
+    b0 = [host(b) for b in bufs]
+    dm.dmuon_muon_step_batched_opts(params, grads, bufs, lr=0.05, nesterov=True, ns_steps=steps,
+                                    ns_coefficients=coeffs)
+    torch.cuda.synchronize()
+    assert dm.dmuon_device_status() == 0
+    for i, s in enumerate(shapes):
+        buf_ref, X, W_ref = oracle.muon_step(np.zeros(s, np.float32), host(grads[i]), b0[i], lr=0.05,
+                                             momentum=0.95, nesterov=True, weight_decay=0.0,
+                                             ns_steps=steps, ns_coeffs=coeffs)
+        assert np.array_equal(host(bufs[i]).view(np.uint32), buf_ref.view(np.uint32))
+        tol = TOL_BF16 if dtype == torch.bfloat16 else TOL_F32
+        check_rel(host(params[i]), W_ref, tol, f"quintic {coeffs} {s} k={steps}")
+
+
+def test_quintic_caller_workspace_size(cuda_lib):
+    """The quintic step needs one more m x m matrix of scratch: the size query
+    with the options says so, and a workspace of exactly that size works."""
+    dm = cuda_lib
+    import ctypes
+    shapes = [(300, 700), (900, 130)]
+    S = (dm.DmuonShape * 2)(*[dm.DmuonShape(r, c, dm.DMUON_BF16, dm.DMUON_BF16) for r, c in shapes])
+    lib = dm.load_library()
+    o = dm.DmuonStepOptions()
+    lib.dmuon_step_options_default(ctypes.byref(o))
+    cubic = lib.dmuon_workspace_bytes_opts(S, 2, ctypes.byref(o))
+    assert cubic == lib.dmuon_workspace_bytes(S, 2, 5)
+    o.ns_a, o.ns_b, o.ns_c = QUINTIC[0]
+    need = lib.dmuon_workspace_bytes_opts(S, 2, ctypes.byref(o))
+    assert need >= cubic + 2 * (300 * 304 + 130 * 136)
+    params = [torch.zeros(s, dtype=torch.bfloat16, device=DEV) for s in shapes]
+    grads = [_rand(s, torch.bfloat16, 80 + i, 1e-3) for i, s in enumerate(shapes)]
+    bufs = [torch.zeros(s, dtype=torch.float32, device=DEV) for s in shapes]
+    p2, b2 = [p.clone() for p in params], [b.clone() for b in bufs]
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    dm.dmuon_muon_step_batched_opts(params, grads, bufs, ns_coefficients=QUINTIC[0], workspace=ws)
+    dm.dmuon_muon_step_batched_opts(p2, grads, b2, ns_coefficients=QUINTIC[0])
+    torch.cuda.synchronize()
+    for a, b in zip(params + bufs, p2 + b2):
+        assert torch.equal(a, b)
+    with pytest.raises(dm.DmuonError):
+        dm.dmuon_muon_step_batched_opts(params, grads, bufs, ns_coefficients=QUINTIC[0],
+                                        workspace=ws[:cubic])

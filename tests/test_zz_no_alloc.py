@@ -4,9 +4,11 @@ It exists for callers that may not allocate device memory (a host framework
 that owns all of it, a sandbox without cudaMalloc, a path that must not block
 on an allocation).  Its scratch is a fixed array inside the library, shared by
 every call.  These tests check it against the regular entry point,
-dmuon_ns_orthogonalize, on two calls in a row, so the second call runs on the
-scratch the first one left behind.  They also check that oversized matrices
-are refused and that a call takes no device memory.
+dmuon_ns_orthogonalize, and against the fp64 oracle, on calls in a row, so
+each call runs on the scratch the one before it left behind (different shapes
+back to back, so the launch description and tensor maps in the shared array
+change between calls).  They also check that oversized matrices are refused
+and that a call takes no device memory.
 
 The file is named to be collected last: if it fails, a run that stops at the
 first failure has already run every other test.
@@ -14,6 +16,7 @@ first failure has already run every other test.
 import pytest
 import torch
 
+import oracle
 from tests.gpu_helpers import TOL_BF16, check_rel, host
 
 pytestmark = pytest.mark.gpu
@@ -39,6 +42,8 @@ def test_noalloc_matches_regular_entry_on_two_calls_in_a_row(cuda_lib):
         torch.cuda.synchronize()
         assert dm.dmuon_device_status() == 0
         check_rel(host(got), host(want), TOL_BF16, f"noalloc {shape} k={steps}")
+        X_ref = oracle.newton_schulz(host(G), steps)
+        check_rel(host(got), X_ref, TOL_BF16, f"noalloc vs oracle {shape} k={steps}")
 
 
 def test_noalloc_takes_no_device_memory(cuda_lib):
