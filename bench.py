@@ -59,6 +59,12 @@ def parse_args():
     ap.add_argument("--adamw-only", type=int, default=0, metavar="ROWS",
                     help="time only the AdamW leg, with embedding and head of ROWS x 4096 "
                          "(128256 for Llama-8B; smaller for a profiler capture)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' lines (the `configs` key)")
+    ap.add_argument("--no-clip", action="store_true")
+    ap.add_argument("--no-quintic", action="store_true")
+    ap.add_argument("--clip-only", action="store_true",
+                    help="time only the per-segment clipping leg (for a profiler capture)")
     return ap.parse_args()
 
 
@@ -288,6 +294,240 @@ def measure_adamw(dm, dev, stream, world, peaks, steps, rows=128256):
     return out
 
 
+QUINTIC = (3.4445, -4.7750, 2.0315)   # a widely used quintic set (not from the pages)
+
+
+def llama_clip_segments(t, dev, rows=128256):
+    """The three gradient groups of a Llama-8B step for the per-segment clip:
+    regular (embedding and LM head, rows x 4096 each), Muon (the 224
+    projections' gradients) and AdamW (65 norm vectors), bf16."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    regular = [(torch.randn((rows, 4096), generator=gen, device=dev) * 1e-4).to(torch.bfloat16)
+               for _ in range(2)]
+    norms = [(torch.randn((4096,), generator=gen, device=dev) * 1e-4).to(torch.bfloat16) for _ in range(65)]
+    return [regular, list(t.grads), norms]
+
+
+def measure_clip(dm, dev, stream, world, peaks, steps, segments):
+    """Per-segment clipping of the three gradient groups.  Every timed pass
+    clips every segment (each step's bound is half the norm the gradients
+    had before it, so every coefficient is about 0.5 and the scale pass
+    rewrites everything): algorithmic bytes per bf16 element are 2 (norm pass)
+    + 2 + 2 (scale pass read and write)."""
+    import math
+    import torch
+    n = sum(g.numel() for seg in segments for g in seg)
+    norms, _ = dm.dmuon_clip_grad_norm_buckets(segments, [math.inf] * len(segments))
+    torch.cuda.synchronize(dev)
+    cur = [float(x) for x in norms.cpu()]
+    for _ in range(3):                                         # warm-up passes, also clipping
+        dm.dmuon_clip_grad_norm_buckets(segments, [0.5 * c for c in cur])
+        cur = [0.5 * c for c in cur]
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        dm.dmuon_clip_grad_norm_buckets(segments, [0.5 * c for c in cur])
+        cur = [0.5 * c for c in cur]
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    gbs = 6.0 * n / (ms_step * 1e-3) / 1e9
+    return {"elements": n, "segments": [sum(g.numel() for g in seg) for seg in segments],
+            "ms_per_step": ms_step, "achieved": gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "bound": "hbm", "bytes_per_element": 6,
+            "note": "three segments (regular: embedding + head, Muon: 224 projections, AdamW: norms), "
+                    "each clipped with its own norm; bf16"}
+
+
+def measure_quintic(dm, t, wl, dev, stream, world, peaks, steps):
+    """The Llama-8B step with quintic coefficients: SYRK, the symmetric square
+    P = b A + c A A and the GEMM X <- a X + P X per NS step.  Useful FLOPs per
+    matrix and NS step: m^2 n + m^3 + 2 m^2 n."""
+    import torch
+    fl = wl.ns_steps * sum(3.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) + min(s.rows, s.cols) ** 3
+                           for s in wl.specs)
+
+    def step():
+        dm.dmuon_muon_step_batched_opts(t.params, t.grads, t.bufs, lr=wl.lr, momentum=wl.momentum,
+                                        nesterov=wl.nesterov, weight_decay=wl.weight_decay,
+                                        ns_steps=wl.ns_steps, ns_coefficients=QUINTIC)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    dm.dmuon_stage_times(reset=True)
+    dm.dmuon_stage_timing(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dm.dmuon_stage_timing(False)
+    stages = dm.dmuon_stage_times(reset=True)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"coefficients": list(QUINTIC), "ms_per_step": ms, "useful_flops_per_step": fl,
+            "tflops": tf, "frac_sustained": tf / peaks["bf16_tflops_sustained"],
+            "stage_ms_per_step": {k: v[0] / steps for k, v in stages.items() if v[1]}}
+
+
+def config_sample(wl, budget):
+    """Matrices of a workload for the oracle: all of them when their useful
+    FLOPs fit the budget, else the first ones in draw order up to it."""
+    chosen, fl = [], 0.0
+    for i, s in enumerate(wl.specs):
+        f = 3.0 * min(s.rows, s.cols) ** 2 * max(s.rows, s.cols) * wl.ns_steps
+        if chosen and fl + f > budget:
+            break
+        chosen.append(i)
+        fl += f
+    return chosen, fl
+
+
+def measure_config(name, dm, dev, peaks, steps, cpu):
+    """One of the other workloads: Muon-step time on the GPU (inputs resident,
+    CUDA events), useful TFLOP/s and the fractions of the peaks, and, when
+    ``cpu``, the fp64 oracle's time for the same step on the host cores (in
+    full for the small workloads, else on a stated sample).  square4096 adds
+    the step-count sweep of the orthogonality error."""
+    import torch
+    from newton_schulz_09_b200 import synthetic
+    wl = synthetic.workload(name)
+    t = synthetic.make_tensors(wl, device=dev, flat=True)
+    fl = synthetic.ns_flops(wl)
+    stream = torch.cuda.current_stream(dev)
+    host = None
+    if cpu:
+        sub, _ = config_sample(wl, 2.2e12)
+        host = [(t.params[i].float().cpu().numpy(), t.grads[i].float().cpu().numpy(),
+                 t.bufs[i].cpu().numpy()) for i in sub]
+        prior = [[g.float().cpu().numpy() for j, g in enumerate(step_g) if j in sub]
+                 for step_g in t.prior_grads]
+    # the momentum history (R14): prior steps with lr = 0, then the measured step
+    for gs in t.prior_grads:
+        dm.dmuon_muon_step_batched(t.params, gs, t.bufs, lr=0.0, momentum=wl.momentum,
+                                   nesterov=wl.nesterov, weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+
+    def step():
+        dm.dmuon_muon_step_batched(t.params, t.grads, t.bufs, lr=wl.lr, momentum=wl.momentum,
+                                   nesterov=wl.nesterov, weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    tf = fl / (ms * 1e-3) / 1e12
+    out = {"workload": name, "matrices": len(wl.specs), "ns_steps": wl.ns_steps,
+           "dtype": "f32 (tf32 operands)" if wl.dtype == torch.float32 else "bf16",
+           "useful_flops_per_step": fl, "ms_per_step": ms, "tflops": tf,
+           "pct_of_bf16_peak": {"measured_sustained": tf / peaks["bf16_tflops_sustained"],
+                                "measured_burst": tf / peaks["bf16_tflops"],
+                                "nominal_2250": tf / NOMINAL_BF16_TFLOPS}}
+    sweep = None
+    if name == "square4096":
+        sweep = []
+        G = t.grads[0]
+        eye = torch.eye(G.shape[0], dtype=torch.float64, device=dev)
+        for k in (3, 5, 7, 10):
+            Y = G.clone()
+            dm.dmuon_ns_orthogonalize(Y, k)
+            Yd = Y.double()
+            err = float(torch.linalg.norm(Yd @ Yd.T - eye))
+            sweep.append({"k": k, "orthogonality_error_gpu": err})
+        out["sweep"] = sweep
+    if cpu:
+        out["cpu_baseline"] = oracle_config_time(wl, host, prior, sub, sweep, G=t.grads[0] if sweep else None)
+    del t
+    torch.cuda.empty_cache()
+    return out
+
+
+def oracle_config_time(wl, host, prior, sub, sweep, G=None):
+    """The fp64 oracle on the host cores: the same Muon step (after the same
+    momentum history) for the sampled matrices; for square4096 also the
+    orthogonality error of the oracle's iterate after 3, 5, 7 and 10 steps."""
+    import numpy as np
+    import oracle
+    threads = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info
+        info = [d for d in threadpool_info() if d.get("internal_api") == "openblas"]
+        if info:
+            threads = int(info[0]["num_threads"])
+    except Exception:
+        pass
+    fl = sum(3.0 * min(wl.specs[i].rows, wl.specs[i].cols) ** 2 * max(wl.specs[i].rows, wl.specs[i].cols)
+             * wl.ns_steps for i in sub)
+    t0 = time.perf_counter()
+    for k, (W, g, b) in enumerate(host):
+        for gs in prior:
+            b, _, _ = oracle.muon_step(W, gs[k], b, lr=0.0, momentum=wl.momentum, nesterov=wl.nesterov,
+                                       weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+        oracle.muon_step(W, g, b, lr=wl.lr, momentum=wl.momentum, nesterov=wl.nesterov,
+                         weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+    secs = time.perf_counter() - t0
+    steps_run = 1 + len(prior)
+    res = {"value": fl * steps_run / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "seconds": secs,
+           "sample": (f"all {len(sub)} matrices" if len(sub) == len(wl.specs) else
+                      f"the first {len(sub)} of {len(wl.specs)} matrices in draw order") +
+                     f", {steps_run} Muon step(s) of {fl:.3e} useful FLOPs each, fp64 numpy/OpenBLAS"}
+    if sweep is not None:
+        X = oracle.frobenius_normalize(G.float().cpu().numpy())
+        done = 0
+        for entry in sweep:
+            for _ in range(entry["k"] - done):
+                X = oracle.ns_iteration(X)
+            done = entry["k"]
+            entry["orthogonality_error_oracle"] = oracle.orthogonality_error(X)
+    return res
+
+
+def run_clip_only(args):
+    """The per-segment clipping leg alone on the Llama-8B gradients (one
+    GPU): its own JSON line, GB/s of algorithmic traffic against the
+    measured copy bandwidth."""
+    import torch
+    import newton_schulz_09_b200 as dm
+    from newton_schulz_09_b200 import synthetic
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dm.load_library()
+    peaks, peak_src = load_peaks()
+    wl = synthetic.workload(args.workload)
+    t = synthetic.make_tensors(wl, device=dev, flat=True)
+    segs = llama_clip_segments(t, dev, rows=128256 if wl.name == "llama8b" else 8192)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    c = measure_clip(dm, dev, torch.cuda.current_stream(dev), 1, peaks, args.steps, segs)
+    clocks = sampler.stop()
+    print(json.dumps({
+        "metric": "per-segment gradient clipping GB/s", "value": c["achieved"], "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": 3, "ms_per_step": c["ms_per_step"],
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "clocks": clocks,
+        "config": {"workload": f"{wl.name} gradients in three segments", "elements": c["elements"],
+                   "bytes_per_element": 6},
+        "roofline": {"bound": "hbm", "achieved": c["achieved"], "peak": c["peak"], "unit": "GB/s",
+                     "frac": c["frac"], "peak_source": f"{peak_src} hbm_gbs"}}))
+    return 0
+
+
 def run_ours(args):
     import torch
     import newton_schulz_09_b200 as dm
@@ -436,6 +676,19 @@ def run_ours(args):
                "api": "dmuon_muon_step_batched_host (pinned host buffers, copies overlapped)"}
         del h_g, h_w, hg, hw
 
+    # ---- per-segment clipping of the step's three gradient groups (HBM-bound)
+    clip = None
+    if not args.no_clip and wl.name == "llama8b":
+        segs = llama_clip_segments(t, dev)
+        clip = measure_clip(dm, dev, stream, world, peaks, args.steps, segs)
+        del segs
+        torch.cuda.empty_cache()
+
+    # ---- the same stack with quintic coefficients (one more symmetric product)
+    quintic = None
+    if not args.no_quintic and wl.name == "llama8b":
+        quintic = measure_quintic(dm, t, wl, dev, stream, world, peaks, 3)
+
     status = dm.dmuon_device_status()
     if status != 0:
         raise RuntimeError(f"device error word {status}")
@@ -443,6 +696,19 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
+
+    # ---- the other workloads, one entry each (single-GPU runs only)
+    configs = None
+    if world == 1 and not args.no_configs:
+        del t
+        dm.dmuon_release_cache()
+        torch.cuda.empty_cache()
+        configs = []
+        for name in ("fp32_256x512", "tinymlp", "square4096", "mixed1024"):
+            if name == wl.name:
+                continue
+            configs.append(measure_config(name, dm, dev, peaks, 3 if name == "mixed1024" else 10,
+                                          cpu=not args.no_cpu_baseline))
 
     if rank == 0:
         line = {
@@ -460,7 +726,8 @@ def run_ours(args):
                        "l2": f"inputs larger than L2 ({wl.numel * 8 / 1e9:.0f} GB per GPU)",
                        "parallelism": f"replicas x{world}"},
             "clocks": clocks, "e2e": e2e, "gpu_launches": launches, "adamw": adamw,
-            "roofline": roofline, "cpu_baseline": cpu,
+            "roofline": roofline, "cpu_baseline": cpu, "clip": clip, "quintic": quintic,
+            "configs": configs,
         }
         print(json.dumps(line))
     if world > 1:
@@ -571,6 +838,8 @@ def main():
     args = parse_args()
     if args.adamw_only > 0:
         return run_adamw_only(args)
+    if args.clip_only:
+        return run_clip_only(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.impl == "torch":
