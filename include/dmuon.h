@@ -45,6 +45,13 @@
  *     (cudaMallocFromPoolAsync / cudaFreeAsync); a plan evicted from the cache
  *     (more than 64) is freed after the latest work that used it.  The first
  *     call on a device also sets the device up (kernel attributes, the pool).
+ *   - CUDA graphs: the Muon-step entry points can be captured once their
+ *     shapes have a plan (an eager call first).  While the stream captures,
+ *     every tensor address is written into the plan by a captured patch
+ *     kernel, so each replay updates the tensors it was captured with,
+ *     whatever eager calls ran in between.  A call that would need a new plan
+ *     or a larger scratch arena during capture is refused with
+ *     DMUON_ERR_UNSUPPORTED before anything is enqueued.
  */
 #ifndef DMUON_H_
 #define DMUON_H_

@@ -314,6 +314,21 @@ struct Arena {
   size_t bytes = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Arena> g_arenas;
+// Library memory whose stream-ordered free could not be enqueued (it may
+// still be in use): freed by dmuon_release_cache after its device sync.
+std::vector<void*> g_parked;
+
+// Frees library memory after the work enqueued on `st` so far (and, with
+// `after`, after that event too).  Never frees memory that may be in use:
+// when the free cannot be enqueued, the memory is parked instead.
+void free_in_order(void* p, cudaStream_t st, cudaEvent_t after = nullptr) {
+  cudaError_t e = after ? cudaStreamWaitEvent(st, after, 0) : cudaSuccess;
+  if (e == cudaSuccess) e = cudaFreeAsync(p, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_parked.push_back(p);
+  }
+}
 
 // DMUON_LOG set to anything but "0": one stderr line per launch plan built.
 bool log_enabled() {
@@ -458,6 +473,15 @@ PtrSet ptrs_of(const MatIn& x) {
 
 // Builds (or finds) the plan for these shapes and this workspace; a new
 // plan's device memory is allocated from the pool and uploaded on `st`.
+bool capturing(cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return cs != cudaStreamCaptureStatusNone;
+}
+
 int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, int dev, cudaStream_t st,
              Plan** out) {
   std::vector<uint8_t> key;
@@ -482,6 +506,11 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     }
   }
 
+  if (capturing(st))
+    // A plan's memory and upload must not belong to a graph: the shapes are
+    // planned by an eager call first.
+    return fail(DMUON_ERR_UNSUPPORTED, "these shapes have no launch plan yet and the stream is "
+                "capturing a graph: make one call with them before the capture");
   const Layout L = make_layout(in, steps, quintic);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const int nmat = static_cast<int>(in.size());
@@ -561,10 +590,16 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
                              dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                              : CU_TENSOR_MAP_SWIZZLE_128B);
         }
-        if (d.A) okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+        const CUtensorMapSwizzle mn_sw =
+            dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+        if (d.A) {
+          okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+          okm &= encode_2d(&mm.amn, dt, d.A, ml.m, ml.m, ml.lda, BK, BK, mn_sw);
+        }
         if (d.P) {
           okm &= encode_2d(&mm.aw, dt, d.A, ml.m, ml.m, ml.lda, BK, kBN);
           okm &= encode_2d(&mm.p, dt, d.P, ml.m, ml.m, ml.lda, BK, kBM);
+          okm &= encode_2d(&mm.pmn, dt, d.P, ml.m, ml.m, ml.lda, BK, BK, mn_sw);
         }
         if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed for matrix %d", i);
       }
@@ -691,8 +726,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     // freed in stream order after the latest work that used it.
     Plan& old = *g_plans.back();
     if (old.dmem) {
-      cudaStreamWaitEvent(st, old.last, 0);
-      cudaFreeAsync(old.dmem, st);
+      free_in_order(old.dmem, st, old.last);
       old.dmem = nullptr;
     }
     g_plans.pop_back();
@@ -704,9 +738,16 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
 // Before a plan's kernels run on `st`: order after the plan's latest use on
 // another stream, then write the caller's addresses where they differ from
 // the ones the descriptors hold.
+//
+// While `st` captures a graph, every address is patched (so that each replay
+// writes the addresses it was captured with, whatever eager calls did in
+// between) and the host's record of the addresses is invalidated (a replay may
+// rewrite them at any time); the ordering against other streams is the
+// graph's, so no event is waited on or recorded.
 int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
+  const bool cap = capturing(st);
   cudaError_t e = cudaSuccess;
-  if (P.last_st != st) e = cudaStreamWaitEvent(st, P.last, 0);
+  if (!cap && P.last_st != st) e = cudaStreamWaitEvent(st, P.last, 0);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   std::unique_ptr<PatchParams> pp;
   auto flush = [&]() {
@@ -718,7 +759,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
   for (size_t i = 0; i < in.size(); ++i) {
     const int d = P.desc_of[i];
     const PtrSet now = ptrs_of(in[i]);
-    if (now == P.cur[d]) continue;
+    if (!cap && now == P.cur[d]) continue;
     if (!pp) {
       pp.reset(new PatchParams());
       pp->mats = const_cast<MatDesc*>(P.d_mats);
@@ -731,6 +772,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
     en.index = d;
     en.vec4 = now.vec4;
     P.cur[d] = now;
+    if (cap) P.cur[d].vec4 = -1;    // unknown after a replay: the next eager call patches
     if (pp->n == kPatchMax) flush();
   }
   flush();
@@ -739,6 +781,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
 
 // After a plan's kernels were enqueued on `st`.
 int finish_plan(Plan& P, cudaStream_t st) {
+  if (capturing(st)) return DMUON_OK;
   cudaError_t e = cudaEventRecord(P.last, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   P.last_st = st;
@@ -861,6 +904,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   np.lr = lr;
   np.wd = wd;
   np.quintic = P.quintic ? 1 : 0;
+  np.mirror = P.quintic ? 1 : 0;     // the SQUARE stage reads all of A
+  np.a_upper = 1;                    // the GEMM reads A (or P) from its upper triangle
   np.ca = o.ca;
   np.cb = P.quintic ? 1.0f : o.cb;   // quintic: X <- a X + P X with P = b A + c A A
   np.cc = 0.0f;
@@ -881,6 +926,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
       NsParams sq = np;
       sq.cb = o.cb;
       sq.cc = o.cc;
+      sq.mirror = 0;
       sq.order = g.gemm_order;
       sq.tile_prefix = g.square_prefix;
       sq.ntiles = g.square_tiles;
@@ -939,9 +985,12 @@ int current_device(int* dev) {
 // order (the old region is freed after the work queued on `st` before it).
 int arena_get(int dev, cudaStream_t st, size_t bytes, void** out) {
   Arena& a = g_arenas[std::make_pair(dev, st)];
+  if (a.bytes < bytes && capturing(st))
+    return fail(DMUON_ERR_UNSUPPORTED, "the stream's scratch arena must grow and the stream is "
+                "capturing a graph: make one call with these shapes before the capture");
   if (a.bytes < bytes) {
     if (a.ptr) {
-      cudaFreeAsync(a.ptr, st);
+      free_in_order(a.ptr, st);
       a.ptr = nullptr;
       a.bytes = 0;
     }
@@ -1570,6 +1619,8 @@ void dmuon_release_cache(void) {
   for (auto& kv : g_arenas)
     if (kv.second.ptr) cudaFree(kv.second.ptr);
   g_arenas.clear();
+  for (void* p : g_parked) cudaFree(p);
+  g_parked.clear();
   for (DeviceInfo& d : g_dev)
     if (d.pool) cudaMemPoolTrimTo(d.pool, 0);
 }
@@ -1986,7 +2037,10 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     okm &= encode_2d(&sp.maps.xkw[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, kBN);
     if (!d.b3d) okm &= encode_2d(&sp.maps.xmn[b], DMUON_BF16, xb, ml.n, ml.m, ml.ldx, BK, BK);
   }
-  if (d.A) okm &= encode_2d(&sp.maps.a, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+  if (d.A) {
+    okm &= encode_2d(&sp.maps.a, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, kBM);
+    okm &= encode_2d(&sp.maps.amn, DMUON_BF16, d.A, ml.m, ml.m, ml.lda, BK, BK);
+  }
   if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
   // The launch description travels as kernel parameters of an upload kernel
@@ -2027,6 +2081,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     np.cb = -0.5f;
     np.cc = 0.0f;
     np.quintic = 0;
+    np.mirror = 0;
+    np.a_upper = 1;
     np.err = di.err;
     np.wait_limit_ns = kWaitLimitNs;
     for (int s = 0; s < steps; ++s) {

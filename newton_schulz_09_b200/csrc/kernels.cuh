@@ -7,7 +7,8 @@
 //                       s = 1 / (||M||_F + 1e-7).
 //   ns_stage_kernel     one Newton-Schulz stage for every matrix of a group
 //                       in one persistent launch:
-//                         SYRK  A = s^2 X X^T  (upper tiles, mirrored store)
+//                         SYRK  A = s^2 X X^T  (upper tiles; mirrored only when
+//                               the quintic SQUARE stage reads A)
 //                         SQUARE P = b A + c A A  (quintic coefficients only)
 //                         GEMM  X' = c (1.5 X - 0.5 A X), or on the last step
 //                               the weight update / output write.   [tensor]
@@ -85,6 +86,8 @@ struct alignas(64) MatMaps {
   CUtensorMap a;       // A as K-major operand, box (128 B of K) x 128 rows
   CUtensorMap aw;      // A, box (128 B of K) x 256 rows: the B operand of A A in one load
   CUtensorMap p;       // P as K-major operand (the GEMM's A operand in quintic mode)
+  CUtensorMap amn;     // A as MN-major operand, box (128 B of M) x (BK rows of K): the GEMM
+  CUtensorMap pmn;     // reads A's (or P's) lower k-blocks transposed from the upper triangle
 };
 
 struct NsParams {
@@ -101,6 +104,9 @@ struct NsParams {
   float ca, cb;            // GEMM: X <- ca X + cb (A or P) X; SQUARE: P = cb A + cc A A
   float cc;
   int quintic;             // GEMM reads P instead of A
+  int mirror;              // SYRK / SQUARE: also write the lower triangle (A^T of the upper)
+  int a_upper;             // GEMM: A (or P) holds its upper triangle and the diagonal 128-blocks
+                           // only; the k-blocks left of the diagonal block are read transposed
   int* err;                // device error word
   uint64_t wait_limit_ns;
 };
@@ -380,7 +386,7 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
         tmem_ld_wait();
         if (c == nch - 1) release(b);
         const int C0 = col0 + c * 32;
-        if (R < m && C0 < m && C0 + 31 >= R) {
+        if (R < m && C0 < m && (!p.mirror || C0 + 31 >= R)) {
           float y[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[j] = alpha * __uint_as_float(v[j]);
@@ -399,6 +405,19 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[j] = op_round<E>(y[j]);
           E* arow = A + static_cast<int64_t>(R) * lda;
+          if (!p.mirror) {
+            // Upper tiles and whole diagonal 128-blocks: every computed element
+            // is stored once, nothing is mirrored (the GEMM reads the lower
+            // part transposed).
+            if (C0 + 32 <= m) {
+              store32<E>(arow + C0, y);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (C0 + j < m) arow[C0 + j] = from_f<E>(y[j]);
+            }
+            continue;
+          }
           if (C0 >= R && C0 + 32 <= m) {
             store32<E>(arow + C0, y);
           } else {
@@ -530,6 +549,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   constexpr uint32_t FMT = (EB == 2) ? 1u : 2u;
   constexpr uint32_t IDESC = make_idesc(FMT, 0u, kMode == kGemm ? 1u : 0u, kBM, kBN);
   constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);   // SYRK / SQUARE half tiles
+  constexpr uint32_t IDESC_AT = make_idesc(FMT, 1u, 1u, kBM, kBN);         // GEMM, A k-block MN-major
   constexpr int NBOX_B = (kMode == kGemm) ? kBN / BK : 2;
   constexpr uint32_t BOX_B_BYTES = (kMode == kGemm) ? BK * 128 : kAStageBytes;
 
@@ -593,6 +613,10 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const CUtensorMap* mapB = (kMode == kSyrk) ? &mp.xk[p.cur]
                               : (kMode == kSquare) ? &mp.a : &mp.xmn[p.cur];
       const CUtensorMap* mapBw = (kMode == kSyrk) ? &mp.xkw[p.cur] : &mp.aw;
+      const CUtensorMap* mapAt = p.quintic ? &mp.pmn : &mp.amn;
+      // GEMM with an upper-only A: k-blocks left of the row block's diagonal
+      // block come from the upper triangle, A[k rows][M columns], MN-major.
+      const int kb_t = (kMode == kGemm && p.a_upper) ? ti.tm * (kBM / BK) : 0;
       int nb = 0;
       const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK / SQUARE B operand rows
       if (kMode == kSyrk || kMode == kSquare) {
@@ -611,6 +635,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         tensormap_acquire_gpu(mapA);
         tensormap_acquire_gpu(mapB);
         if (kMode != kGemm) tensormap_acquire_gpu(mapBw);
+        if (kMode == kGemm && p.a_upper) tensormap_acquire_gpu(mapAt);
         fenced = ti.mi;
       }
       for (int kb = 0; kb < ti.nkb; ++kb) {
@@ -620,7 +645,15 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* a_dst = sa + stage * kAStageBytes;
           uint8_t* b_dst = sb + stage * kBStageBytes;
-          tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
+          if (kMode == kGemm && kb < kb_t) {
+            // 128 M columns in 128-byte chunks (2 for bf16, 4 for fp32), each
+            // BK rows of K: the MN-major layout of the B operand.
+#pragma unroll
+            for (int h = 0; h < EB; ++h)
+              tma_load_2d(a_dst + h * (BK * 128), mapAt, &full[stage], ti.tm * kBM + h * (128 / EB), kb * BK);
+          } else {
+            tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
+          }
           if (kMode == kGemm && md.b3d) {
             // The four 64-column blocks of the tile in one load, same smem layout.
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
@@ -661,6 +694,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
       const uint32_t idesc = (kMode != kGemm && ti.half) ? IDESC_HALF : IDESC;
+      const int kb_t = (kMode == kGemm && p.a_upper) ? ti.tm * (kBM / BK) : 0;
       for (int kb = 0; kb < ti.nkb; ++kb) {
         w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
@@ -668,9 +702,13 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         if (lane == 0) {
           const uint32_t a_base = smem_u32(sa + stage * kAStageBytes);
           const uint32_t b_base = smem_u32(sb + stage * kBStageBytes);
+          const bool at = kb < kb_t;      // A k-block transposed (MN-major)
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
-            const uint64_t ad = sw128_desc(a_base + k * 32, 16, 1024);
+            const uint64_t ad =
+                at ? sw128_desc(a_base + k * MMA_K * 128, BK * 128, EB == 2 ? 1024 : 512,
+                                EB == 2 ? kSwizzle128B : kSwizzle128B32)
+                   : sw128_desc(a_base + k * 32, 16, 1024);
             // MN-major B: 16-bit operands use the 16-byte-unit swizzle (8-line
             // K groups); 32-bit operands must use 32-byte units (4-line groups).
             const uint64_t bd =
@@ -679,8 +717,9 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
                     : sw128_desc(b_base + k * MMA_K * 128, BK * 128, EB == 2 ? 1024 : 512,
                                  EB == 2 ? kSwizzle128B : kSwizzle128B32);
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-            if (EB == 2) umma_f16(d_tmem, ad, bd, idesc, acc);
-            else umma_tf32(d_tmem, ad, bd, idesc, acc);
+            const uint32_t id = at ? IDESC_AT : idesc;
+            if (EB == 2) umma_f16(d_tmem, ad, bd, id, acc);
+            else umma_tf32(d_tmem, ad, bd, id, acc);
           }
           umma_commit(&empty[stage]);
         }

@@ -80,3 +80,51 @@ def test_captured_host_buffer_step(cuda_lib):
             assert torch.equal(params[i], ref_p[i]), (step, i)
             assert torch.equal(bufs[i], ref_b[i]), (step, i)
             assert torch.equal(hw[i], ref_p[i].cpu()), (step, i)
+
+
+def test_replay_after_eager_calls_with_other_tensors(cuda_lib):
+    """Launch plans are cached by shape, and a cached plan's descriptors are
+    patched with each call's tensor addresses.  A graph captured on tensors A
+    must keep updating A when it is replayed after an eager call on tensors B
+    of the same shapes (same workspace, so the same plan); capture also
+    refuses shapes that have no plan yet, before anything is enqueued."""
+    dm = cuda_lib
+    pa, ga, ba = _state(3)
+    pb, gb, bb = _state(4)
+    ra_p, ra_b = [p.clone() for p in pa], [b.clone() for b in ba]
+    rb_p, rb_b = [p.clone() for p in pb], [b.clone() for b in bb]
+    ws = torch.empty(dm.dmuon_workspace_bytes(pa, HP["ns_steps"], ga), dtype=torch.uint8, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dm.dmuon_muon_step_batched_ex(pa, ga, ba, workspace=ws, **HP)     # plan for these shapes
+    dm.dmuon_muon_step_batched_ex(ra_p, ga, ra_b, **HP)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dm.dmuon_muon_step_batched_ex(pa, ga, ba, workspace=ws, **HP)
+    with torch.cuda.stream(s):
+        dm.dmuon_muon_step_batched_ex(pb, gb, bb, workspace=ws, **HP)     # same plan, tensors B
+    dm.dmuon_muon_step_batched_ex(rb_p, gb, rb_b, **HP)
+    torch.cuda.synchronize()
+    g.replay()                                                             # must update A again
+    dm.dmuon_muon_step_batched_ex(ra_p, ga, ra_b, **HP)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        dm.dmuon_muon_step_batched_ex(pb, gb, bb, workspace=ws, **HP)     # and B again, eagerly
+    dm.dmuon_muon_step_batched_ex(rb_p, gb, rb_b, **HP)
+    torch.cuda.synchronize()
+    for x, y in zip(pa + ba + pb + bb, ra_p + ra_b + rb_p + rb_b):
+        assert torch.equal(x, y)
+    # new shapes during a capture: refused, nothing captured
+    new_p = [torch.zeros((136, 200), dtype=torch.bfloat16, device=DEV)]
+    new_g = [_rand((136, 200), torch.bfloat16, 9, 1e-3)]
+    new_b = [torch.zeros((136, 200), dtype=torch.float32, device=DEV)]
+    ws2 = torch.empty(dm.dmuon_workspace_bytes(new_p, HP["ns_steps"], new_g), dtype=torch.uint8, device=DEV)
+    g2 = torch.cuda.CUDAGraph()
+    with pytest.raises(dm.DmuonError) as e:
+        with torch.cuda.graph(g2, stream=s):
+            dm.dmuon_muon_step_batched_ex(new_p, new_g, new_b, workspace=ws2, **HP)
+    assert "capturing" in str(e.value)
+    torch.cuda.synchronize()
+    assert not new_p[0].any()
+    assert dm.dmuon_device_status() == 0
