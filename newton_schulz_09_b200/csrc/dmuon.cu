@@ -291,6 +291,7 @@ struct Plan {
   std::vector<GroupPlan> groups;
   std::vector<int> desc_of;       // input matrix -> descriptor index
   std::vector<PtrSet> cur;        // per descriptor: the addresses its device copy holds
+  bool captured = false;          // used in a graph capture: replays rewrite the addresses
   cudaEvent_t last = nullptr;     // recorded after the latest work that used the plan
   cudaStream_t last_st = nullptr; // ... on this stream
   ~Plan() {
@@ -741,9 +742,10 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
 //
 // While `st` captures a graph, every address is patched (so that each replay
 // writes the addresses it was captured with, whatever eager calls did in
-// between) and the host's record of the addresses is invalidated (a replay may
-// rewrite them at any time); the ordering against other streams is the
-// graph's, so no event is waited on or recorded.
+// between), and from then on every call on the plan patches every address: a
+// replay may rewrite them at any time, so the host's record is no longer the
+// device's.  The ordering against other streams is the graph's, so no event
+// is waited on or recorded during capture.
 int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
   const bool cap = capturing(st);
   cudaError_t e = cudaSuccess;
@@ -759,7 +761,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
   for (size_t i = 0; i < in.size(); ++i) {
     const int d = P.desc_of[i];
     const PtrSet now = ptrs_of(in[i]);
-    if (!cap && now == P.cur[d]) continue;
+    if (!cap && !P.captured && now == P.cur[d]) continue;
     if (!pp) {
       pp.reset(new PatchParams());
       pp->mats = const_cast<MatDesc*>(P.d_mats);
@@ -772,10 +774,10 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
     en.index = d;
     en.vec4 = now.vec4;
     P.cur[d] = now;
-    if (cap) P.cur[d].vec4 = -1;    // unknown after a replay: the next eager call patches
     if (pp->n == kPatchMax) flush();
   }
   flush();
+  if (cap) P.captured = true;
   return DMUON_OK;
 }
 

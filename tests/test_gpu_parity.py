@@ -254,3 +254,33 @@ def test_bounded_wait_reports_timeout(cuda_lib):
     dm.dmuon_ns_orthogonalize(X, 2)
     torch.cuda.synchronize()
     assert dm.dmuon_device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_update_on_real_weights_is_visible(cuda_lib, dtype):
+    """With real (nonzero) weights and an lr large enough that lr X is many
+    weight ulps, the change of the weights, W' - W, must match the oracle's
+    within the X tolerance: a missing, halved or mis-signed update, or weight
+    decay applied twice, fails here (at the bench's lr the update is below half
+    a bf16 ulp of most weights, so the weight check alone could not see it)."""
+    dm = cuda_lib
+    shapes = [(384, 1024), (1200, 264), (256, 256)]
+    params = [_rand(s, dtype, 500 + i, 0.02) for i, s in enumerate(shapes)]
+    grads = [_rand(s, dtype, 510 + i, 1e-3) for i, s in enumerate(shapes)]
+    bufs = [_rand(s, torch.float32, 520 + i, 1e-3) for i, s in enumerate(shapes)]
+    W0 = [host(p).astype(np.float64) for p in params]
+    g0 = [host(g) for g in grads]
+    b0 = [host(b) for b in bufs]
+    lr, wd = 0.5, 0.1
+    dm.dmuon_muon_step_batched(params, grads, bufs, lr=lr, momentum=0.95, nesterov=True,
+                               weight_decay=wd, ns_steps=5)
+    torch.cuda.synchronize()
+    assert dm.dmuon_device_status() == 0
+    for i, s in enumerate(shapes):
+        _, X, W_ref = oracle.muon_step(W0[i].astype(np.float32), g0[i], b0[i], lr=lr, momentum=0.95,
+                                       nesterov=True, weight_decay=wd, ns_steps=5)
+        d_gpu = host(params[i]).astype(np.float64) - W0[i]
+        d_ref = W_ref - W0[i]
+        # the update is far above the weights' rounding: lr |X| against one ulp of |W|
+        assert np.median(np.abs(d_ref)) > 20 * np.median(np.abs(W0[i])) * 2.0 ** -8
+        check_rel(d_gpu, d_ref, tol_for(dtype), f"W' - W {s} {dtype}")
