@@ -254,6 +254,7 @@ Layout make_layout(const std::vector<MatIn>& in, int steps, bool quintic = false
 struct GroupPlan {
   int dtype;
   bool ranks = false;     // some matrix averages several ranks' gradients
+  bool g_f32 = false;     // some gradient is fp32 (the prologue stages 32 KB of gradient)
   int nmat;
   int first;              // first MatDesc index of the group
   int64_t ptiles;
@@ -569,6 +570,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       d.vec4 = vec4_of(x);
       d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
       if (d.world > 1) gp.ranks = true;
+      if (x.gdt == DMUON_F32) gp.g_f32 = true;
       d.Gr = nullptr;   // set once the plan's device memory exists
       d.ptiles_c = static_cast<int>(ml.ptiles_c);
       A.pp.push_back(A.pp.back() + ml.ptiles);
@@ -865,6 +867,7 @@ ElemParams elem_params(const Plan& P, const GroupPlan& g, const StepOpts& o) {
   ep.wd = o.wd;
   ep.clip = o.max_norm > 0.0f ? P.clip : nullptr;
   ep.gpartials = g.gpartials;
+  ep.stage_g = g.g_f32 ? kProStageG : kProStageG16;
   return ep;
 }
 
@@ -887,8 +890,9 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
-    else prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    const int smem = g.g_f32 ? kProSmemBytes : kProSmemBytes16;
+    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, smem, st>>>(ep);
+    else prologue_kernel<E, false><<<pgrid, kPThreads, smem, st>>>(ep);
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
@@ -1730,11 +1734,14 @@ static int clip_check(const dmuon_grad_desc descs[], int count, int nseg) {
   return DMUON_OK;
 }
 
-// Scratch of one clip call: one fp64 partial per 8192-element item, then the
+// Scratch of one clip call: one fp64 partial per 32 KB work item, then the
 // per-segment coefficients.
+static int64_t clip_items_of(const dmuon_grad_desc& d) {
+  return cdiv(d.numel * elem_bytes(d.dtype), kClipItemBytes);
+}
 static size_t clip_scratch_bytes(const dmuon_grad_desc descs[], int count, int nseg, size_t* coef_off) {
   int64_t items = 0;
-  for (int i = 0; i < count; ++i) items += cdiv(descs[i].numel, kClipChunk);
+  for (int i = 0; i < count; ++i) items += clip_items_of(descs[i]);
   const size_t off = align_up(sizeof(double) * static_cast<size_t>(std::max<int64_t>(items, 1)), 256);
   if (coef_off) *coef_off = off;
   return off + align_up(sizeof(float) * nseg, 256);
@@ -1781,7 +1788,7 @@ int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc desc
     ts[k].item0 = items;
     ts[k].seg = d.segment;
     ts[k].bf16 = d.dtype == DMUON_BF16;
-    items += cdiv(d.numel, kClipChunk);
+    items += clip_items_of(d);
   }
   while (seg < nseg) fp->seg_item0[++seg] = items;
   for (int s = 0; s < nseg; ++s) fp->max_norm[s] = max_norms[s];
@@ -1823,7 +1830,8 @@ int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc desc
       cp->item_end = (first + n < ts.size()) ? ts[first + n].item0 : items;
       const int64_t ni = cp->item_end - cp->item_begin;
       if (ni <= 0) continue;
-      const int grid = static_cast<int>(std::min<int64_t>(ni, static_cast<int64_t>(sms) * 8));
+      // four resident blocks per SM (64 registers a thread): one wave of them
+      const int grid = static_cast<int>(std::min<int64_t>(ni, static_cast<int64_t>(sms) * 4));
       LaunchScope ls(st, DMUON_KERNEL_CLIP);
       if (scale) clip_scale_kernel<<<grid, kPThreads, 0, st>>>(*cp);
       else clip_norm_kernel<<<grid, kPThreads, 0, st>>>(*cp);
@@ -2064,8 +2072,9 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   ep.wd = 0.0f;
   ep.clip = nullptr;
   ep.gpartials = nullptr;
+  ep.stage_g = kProStageG16;
   const int pgrid = static_cast<int>(std::min<int64_t>(ml.ptiles, static_cast<int64_t>(di.sms) * 8));
-  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, kProSmemBytes16, st>>>(ep);
   finalize_kernel<<<1, 32, 0, st>>>(ep);
   g_launches += 2;
   if (steps == 0) {

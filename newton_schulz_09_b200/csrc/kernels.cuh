@@ -122,6 +122,8 @@ struct ElemParams {
   float lr, wd;                 // apply_kernel only
   const float* clip;            // gradient scale (global-norm clipping) or nullptr
   double* gpartials;            // grad_norm_kernel: one partial sum of g^2 per item
+  int stage_g;                  // prologue: bytes of staged gradient before the staged buffer
+                                // (kProStageG16 when every gradient is bf16, else kProStageG)
 };
 
 // ------------------------------------------------------------------ helpers
@@ -765,7 +767,11 @@ constexpr int kTR = 64, kTC = 128;     // transposed item: 64 parameter rows x 1
 // fp32 transpose tile once every thread has read its staged inputs.
 constexpr int kProStageG = kFlatChunk * 4;
 constexpr int kProSmemBytes = kFlatChunk * 8;
-static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes, "transpose tile must fit the staging area");
+// With bf16 gradients only: 16 KB of gradient + 32 KB of buffer, so that four
+// blocks fit an SM (with the 64-register bound of the kernel).
+constexpr int kProStageG16 = kFlatChunk * 2;
+constexpr int kProSmemBytes16 = kFlatChunk * 6;
+static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes16, "transpose tile must fit the staging area");
 
 // Stage 8 consecutive input elements (one thread's segment) into shared
 // memory with 16-byte asynchronous copies: the gradient at sg (2 or 4 bytes
@@ -955,7 +961,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
   E* X = reinterpret_cast<E*>(md.X[0]);
   E* Xo = reinterpret_cast<E*>(md.Xop[0]);
   const int gb = md.g_bf16 ? 2 : 4;
-  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
+  float* sbuf = reinterpret_cast<float*>(stage + p.stage_g);
   // Four rounds of 8 consecutive elements per thread.  The whole, aligned
   // segments of all four rounds are staged into shared memory first, so
   // 4 x (8 g + 8 buf) elements per thread are in flight at once; each thread
@@ -1024,7 +1030,7 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   const bool has_buf = md.buf != nullptr;
   const int64_t c = c0 + tx * 8;
   const int gb = md.g_bf16 ? 2 : 4;
-  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
+  float* sbuf = reinterpret_cast<float*>(stage + p.stage_g);
   // Stage this thread's four row segments (whole, aligned ones) first.
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -1097,9 +1103,12 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   return ss;
 }
 
+// Four resident blocks per SM (64 registers, 48 KB of staging with bf16
+// gradients); the instantiation that averages several ranks' gradients needs
+// more registers and runs with fewer blocks.
 template <typename E, bool kRanks = false>
-__global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
-  extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
+__global__ void __launch_bounds__(kPThreads, kRanks ? 2 : 4) prologue_kernel(const __grid_constant__ ElemParams p) {
+  extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes16 or kProSmemBytes
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
   // A block's items only move forward through the matrices: one search,
@@ -1360,7 +1369,8 @@ __global__ void __launch_bounds__(kPThreads) adamw_kernel(const __grid_constant_
 // Clipping of several gradient segments, each with its own norm and
 // coefficient (the training guide's fused regular / Muon / AdamW clipping,
 // "梯度裁剪").  Three kernels:
-//   clip_norm_kernel      one fp64 sum of squares per 8192-element work item
+//   clip_norm_kernel      one fp64 sum of squares per 32 KB work item (eight
+//                         16-byte loads in flight per thread)
 //   clip_finalize_kernel  one block per segment: fixed-order sum of its
 //                         items, ||g||_s, c_s = fl32(min(1, max_s / (||g||_s + 1e-6)))
 //   clip_scale_kernel     g <- fl32(g * c_s), rounded to the storage type,
@@ -1371,7 +1381,8 @@ __global__ void __launch_bounds__(kPThreads) adamw_kernel(const __grid_constant_
 // ======================================================================
 constexpr int kClipMaxTensors = 512;     // tensors per launch (kernel parameter space)
 constexpr int kClipMaxSegs = 64;
-constexpr int kClipChunk = 8192;         // elements per work item (256 threads x 4 x 8)
+constexpr int kClipVecs = 8;             // 16-byte vectors per thread per work item, all in flight
+constexpr int kClipItemBytes = kPThreads * kClipVecs * 16;   // 32 KB of gradient per work item
 
 struct ClipTensor {
   void* g;
@@ -1408,29 +1419,109 @@ __device__ __forceinline__ int clip_tensor_of(const ClipBucketParams& p, int64_t
   return lo;
 }
 
-__global__ void __launch_bounds__(kPThreads) clip_norm_kernel(const __grid_constant__ ClipBucketParams p) {
+// Vector q of this thread in a work item: 16 bytes at byte offset
+// item * 32 KB + (q * 256 + thread) * 16 of the tensor (consecutive threads,
+// consecutive 16 bytes).  All kClipVecs vectors are loaded before any is used;
+// a vector that is not whole, or of a tensor that is not 16-byte aligned, is
+// read element by element, and elements past the tensor read as zero.
+// `streaming`: the data is not read again soon (evict first from L2).
+template <int EB, bool streaming>
+__device__ __forceinline__ void clip_load(const ClipTensor& T, int64_t base_el, bool aligned16,
+                                          uint4 (&v)[kClipVecs]) {
+  constexpr int PER = 16 / EB;                 // elements per vector
+#pragma unroll
+  for (int q = 0; q < kClipVecs; ++q) {
+    const int64_t e = base_el + static_cast<int64_t>(q * kPThreads + threadIdx.x) * PER;
+    if (aligned16 && e + PER <= T.numel) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(T.g) + e * EB);
+      v[q] = streaming ? __ldcs(src) : *src;
+    } else {
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        if (e + k < T.numel) {
+          if constexpr (EB == 2)
+            w[k >> 1] |= static_cast<uint32_t>(static_cast<const uint16_t*>(T.g)[e + k]) << (16 * (k & 1));
+          else
+            w[k] = static_cast<const uint32_t*>(T.g)[e + k];
+        }
+      }
+      v[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// Element k of a 16-byte vector as fp32 (bf16 widens exactly).
+template <int EB>
+__device__ __forceinline__ float clip_elem(const uint4& v, int k) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  if constexpr (EB == 2) return __uint_as_float((k & 1) ? (u[k >> 1] & 0xFFFF0000u) : (u[k >> 1] << 16));
+  else return __uint_as_float(u[k]);
+}
+
+template <int EB>
+__device__ __forceinline__ double clip_sumsq(const ClipTensor& T, int64_t it) {
+  constexpr int PER = 16 / EB;
+  const int64_t base_el = (it - T.item0) * (kClipItemBytes / EB);
+  uint4 v[kClipVecs];
+  clip_load<EB, false>(T, base_el, (reinterpret_cast<uintptr_t>(T.g) & 15) == 0, v);
+  double ss = 0.0;
+#pragma unroll
+  for (int q = 0; q < kClipVecs; ++q)
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const double x = static_cast<double>(clip_elem<EB>(v[q], k));
+      ss = fma(x, x, ss);
+    }
+  return ss;
+}
+
+template <int EB>
+__device__ __forceinline__ void clip_scale_item(const ClipTensor& T, int64_t it, float c) {
+  constexpr int PER = 16 / EB;
+  const int64_t base_el = (it - T.item0) * (kClipItemBytes / EB);
+  const bool aligned16 = (reinterpret_cast<uintptr_t>(T.g) & 15) == 0;
+  uint4 v[kClipVecs];
+  clip_load<EB, true>(T, base_el, aligned16, v);
+#pragma unroll
+  for (int q = 0; q < kClipVecs; ++q) {
+    const int64_t e = base_el + static_cast<int64_t>(q * kPThreads + threadIdx.x) * PER;
+    if (e >= T.numel) continue;
+    float y[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) y[k] = __fmul_rn(clip_elem<EB>(v[q], k), c);
+    if (aligned16 && e + PER <= T.numel) {
+      uint4 o;
+      if constexpr (EB == 2) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+          w[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        o = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        o = make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                       __float_as_uint(y[3]));
+      }
+      __stcs(reinterpret_cast<uint4*>(static_cast<uint8_t*>(T.g) + e * EB), o);
+    } else {
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        if (e + k >= T.numel) break;
+        if constexpr (EB == 2) static_cast<__nv_bfloat16*>(T.g)[e + k] = __float2bfloat16_rn(y[k]);
+        else static_cast<float*>(T.g)[e + k] = y[k];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPThreads, 4) clip_norm_kernel(const __grid_constant__ ClipBucketParams p) {
   __shared__ double red[kPThreads / 32];
   const int tid = threadIdx.x;
   for (int64_t it = p.item_begin + blockIdx.x; it < p.item_end; it += gridDim.x) {
     const ClipTensor& T = p.t[clip_tensor_of(p, it)];
-    const int64_t base = (it - T.item0) * kClipChunk;
-    const bool aligned16 = (reinterpret_cast<uintptr_t>(T.g) & 15) == 0;
-    // All four rounds' loads first, so 4 x 8 elements per thread are in flight.
-    float x[4][8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
-      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
-      if (valid > 0) load8_any(T.g, T.bf16 != 0, e, aligned16 && valid == 8, valid, x[j]);
-      else
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[j][k] = 0.0f;
-    }
-    double ss = 0.0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ss = fma(static_cast<double>(x[j][k]), static_cast<double>(x[j][k]), ss);
+    double ss = T.bf16 ? clip_sumsq<2>(T, it) : clip_sumsq<4>(T, it);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
@@ -1466,34 +1557,15 @@ __global__ void __launch_bounds__(256) clip_finalize_kernel(const __grid_constan
   }
 }
 
-__global__ void __launch_bounds__(kPThreads) clip_scale_kernel(const __grid_constant__ ClipBucketParams p) {
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kPThreads, 4) clip_scale_kernel(const __grid_constant__ ClipBucketParams p) {
   const int64_t n = p.item_end - p.item_begin;
   for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
     const int64_t it = p.item_end - 1 - r;
     const ClipTensor& T = p.t[clip_tensor_of(p, it)];
     const float c = p.coef[T.seg];
     if (c == 1.0f) continue;          // the identity: nothing to write
-    const int64_t base = (it - T.item0) * kClipChunk;
-    const bool aligned16 = (reinterpret_cast<uintptr_t>(T.g) & 15) == 0;
-    float x[4][8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
-      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
-      if (valid > 0) load8_any(T.g, T.bf16 != 0, e, aligned16 && valid == 8, valid, x[j]);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t e = base + (static_cast<int64_t>(j) * kPThreads + tid) * 8;
-      const int valid = e < T.numel ? static_cast<int>(T.numel - e < 8 ? T.numel - e : 8) : 0;
-      if (valid <= 0) continue;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) x[j][k] = __fmul_rn(x[j][k], c);
-      const bool vec = aligned16 && valid == 8;
-      if (T.bf16) store8_x<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(T.g) + e, vec, valid, x[j]);
-      else store8_f32(reinterpret_cast<float*>(T.g) + e, vec, valid, x[j]);
-    }
+    if (T.bf16) clip_scale_item<2>(T, it, c);
+    else clip_scale_item<4>(T, it, c);
   }
 }
 

@@ -285,8 +285,8 @@ def test_clip_buckets_argument_checks(lib):
     D = (dm.DmuonGradDesc * 3)(dm.DmuonGradDesc(10000, dm.DMUON_BF16, 0),
                                dm.DmuonGradDesc(5, dm.DMUON_F32, 2),
                                dm.DmuonGradDesc(8192, dm.DMUON_BF16, 1))
-    # 10000 -> 2 items, 5 -> 1, 8192 -> 1: four fp64 partials (256 bytes) and
-    # three coefficients (256 bytes)
+    # 32 KB work items: 10000 bf16 -> 1, 5 fp32 -> 1, 8192 bf16 -> 1: three fp64
+    # partials (256 bytes) and three coefficients (256 bytes)
     assert lib.dmuon_clip_workspace_bytes(D, 3, 3) == 512
     assert lib.dmuon_clip_workspace_bytes(D, 3, 2) == 0          # segment 2 out of range
     G = (ctypes.c_void_p * 3)(0x10000, 0x20000, 0x30000)
