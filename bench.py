@@ -34,14 +34,13 @@ METRIC = "Muon-step ms & NS TFLOP/s (Llama-8B shapes), % of B200 dense BF16 peak
 UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage per full
-# Llama-8B launch: the one-layer ncu capture (--workload llama8b_layer) scaled by 32 identical
-# layers; valid only for the kernel source it was measured on.
-# ncu capture of the GEMM stage on one Llama-8B layer (1.254 GB of DRAM traffic for
-# 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so
-# its traffic is this ratio times the useful FLOPs of that launch.
-PROFILED_TRAFFIC = {"kernels_sha256_prefix": "2f4971a39e1b5031", "workload": "llama8b",
-                    "gemm_bytes_per_useful_flop": 1.2537e9 / 1.735e12}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage: the ncu
+# capture of one Llama-8B layer (528.7 MB read + 408.2 MB written for 1.735e12 useful FLOPs);
+# a launch of the full workload covers several layers, so its traffic is this ratio times the
+# useful FLOPs of that launch.  Valid only for the stage kernel's source it was measured on
+# (ns_stage.cuh and ptx.cuh).
+PROFILED_TRAFFIC = {"kernel_sha256_prefix": "ce732d4630551214", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 0.9370e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -69,14 +68,16 @@ def parse_args():
 
 
 def profiled_traffic(workload: str):
-    """The profiled DRAM bytes per useful GEMM FLOP, or None when the kernels changed since."""
+    """The profiled DRAM bytes per useful GEMM FLOP, or None when the stage kernel's source
+    changed since."""
     import hashlib
-    path = os.path.join(HERE, "newton_schulz_09_b200", "csrc", "kernels.cuh")
+    csrc = os.path.join(HERE, "newton_schulz_09_b200", "csrc")
     try:
-        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
+        data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("ns_stage.cuh", "ptx.cuh"))
     except OSError:
         return None
-    if sha.startswith(PROFILED_TRAFFIC["kernels_sha256_prefix"]) and workload == PROFILED_TRAFFIC["workload"]:
+    sha = hashlib.sha256(data).hexdigest()
+    if sha.startswith(PROFILED_TRAFFIC["kernel_sha256_prefix"]) and workload == PROFILED_TRAFFIC["workload"]:
         return PROFILED_TRAFFIC["gemm_bytes_per_useful_flop"]
     return None
 
