@@ -433,12 +433,22 @@ def measure_config(name, dm, dev, peaks, steps, cpu):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
     tf = fl / (ms * 1e-3) / 1e12
+    # per-stage device time, from a few more steps with each launch bracketed
+    # by events (kept out of the timed steps above)
+    dm.dmuon_stage_times(reset=True)
+    dm.dmuon_stage_timing(True)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    dm.dmuon_stage_timing(False)
+    stages = {k: v[0] / 3 for k, v in dm.dmuon_stage_times(reset=True).items() if v[1]}
     out = {"workload": name, "matrices": len(wl.specs), "ns_steps": wl.ns_steps,
            "dtype": "f32 (tf32 operands)" if wl.dtype == torch.float32 else "bf16",
            "useful_flops_per_step": fl, "ms_per_step": ms, "tflops": tf,
            "pct_of_bf16_peak": {"measured_sustained": tf / peaks["bf16_tflops_sustained"],
                                 "measured_burst": tf / peaks["bf16_tflops"],
-                                "nominal_2250": tf / NOMINAL_BF16_TFLOPS}}
+                                "nominal_2250": tf / NOMINAL_BF16_TFLOPS},
+           "stage_ms_per_step": stages}
     sweep = None
     if name == "square4096":
         sweep = []

@@ -254,7 +254,6 @@ Layout make_layout(const std::vector<MatIn>& in, int steps, bool quintic = false
 struct GroupPlan {
   int dtype;
   bool ranks = false;     // some matrix averages several ranks' gradients
-  bool g_f32 = false;     // some gradient is fp32 (the prologue stages 32 KB of gradient)
   int nmat;
   int first;              // first MatDesc index of the group
   int64_t ptiles;
@@ -570,7 +569,6 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       d.vec4 = vec4_of(x);
       d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
       if (d.world > 1) gp.ranks = true;
-      if (x.gdt == DMUON_F32) gp.g_f32 = true;
       d.Gr = nullptr;   // set once the plan's device memory exists
       d.ptiles_c = static_cast<int>(ml.ptiles_c);
       A.pp.push_back(A.pp.back() + ml.ptiles);
@@ -867,7 +865,6 @@ ElemParams elem_params(const Plan& P, const GroupPlan& g, const StepOpts& o) {
   ep.wd = o.wd;
   ep.clip = o.max_norm > 0.0f ? P.clip : nullptr;
   ep.gpartials = g.gpartials;
-  ep.stage_g = g.g_f32 ? kProStageG : kProStageG16;
   return ep;
 }
 
@@ -890,9 +887,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-    const int smem = g.g_f32 ? kProSmemBytes : kProSmemBytes16;
-    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, smem, st>>>(ep);
-    else prologue_kernel<E, false><<<pgrid, kPThreads, smem, st>>>(ep);
+    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    else prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
@@ -1840,7 +1836,7 @@ int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc desc
   launch_all(false);
   {
     LaunchScope ls(st, DMUON_KERNEL_CLIP);
-    clip_finalize_kernel<<<nseg, 256, 0, st>>>(*fp);
+    clip_finalize_kernel<<<nseg, kClipFinThreads, 0, st>>>(*fp);
   }
   launch_all(true);
   cudaError_t e = cudaGetLastError();
@@ -2072,9 +2068,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   ep.wd = 0.0f;
   ep.clip = nullptr;
   ep.gpartials = nullptr;
-  ep.stage_g = kProStageG16;
   const int pgrid = static_cast<int>(std::min<int64_t>(ml.ptiles, static_cast<int64_t>(di.sms) * 8));
-  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, kProSmemBytes16, st>>>(ep);
+  prologue_kernel<__nv_bfloat16><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
   finalize_kernel<<<1, 32, 0, st>>>(ep);
   g_launches += 2;
   if (steps == 0) {

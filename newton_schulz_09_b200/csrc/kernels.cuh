@@ -122,8 +122,6 @@ struct ElemParams {
   float lr, wd;                 // apply_kernel only
   const float* clip;            // gradient scale (global-norm clipping) or nullptr
   double* gpartials;            // grad_norm_kernel: one partial sum of g^2 per item
-  int stage_g;                  // prologue: bytes of staged gradient before the staged buffer
-                                // (kProStageG16 when every gradient is bf16, else kProStageG)
 };
 
 // ------------------------------------------------------------------ helpers
@@ -227,11 +225,7 @@ constexpr int kTR = 64, kTC = 128;     // transposed item: 64 parameter rows x 1
 // fp32 transpose tile once every thread has read its staged inputs.
 constexpr int kProStageG = kFlatChunk * 4;
 constexpr int kProSmemBytes = kFlatChunk * 8;
-// With bf16 gradients only: 16 KB of gradient + 32 KB of buffer, so that four
-// blocks fit an SM (with the 64-register bound of the kernel).
-constexpr int kProStageG16 = kFlatChunk * 2;
-constexpr int kProSmemBytes16 = kFlatChunk * 6;
-static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes16, "transpose tile must fit the staging area");
+static_assert(kTR * (kTC + 1) * 4 <= kProSmemBytes, "transpose tile must fit the staging area");
 
 // Stage 8 consecutive input elements (one thread's segment) into shared
 // memory with 16-byte asynchronous copies: the gradient at sg (2 or 4 bytes
@@ -421,7 +415,7 @@ __device__ __forceinline__ float prologue_flat(const ElemParams& p, const MatDes
   E* X = reinterpret_cast<E*>(md.X[0]);
   E* Xo = reinterpret_cast<E*>(md.Xop[0]);
   const int gb = md.g_bf16 ? 2 : 4;
-  float* sbuf = reinterpret_cast<float*>(stage + p.stage_g);
+  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
   // Four rounds of 8 consecutive elements per thread.  The whole, aligned
   // segments of all four rounds are staged into shared memory first, so
   // 4 x (8 g + 8 buf) elements per thread are in flight at once; each thread
@@ -490,7 +484,7 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   const bool has_buf = md.buf != nullptr;
   const int64_t c = c0 + tx * 8;
   const int gb = md.g_bf16 ? 2 : 4;
-  float* sbuf = reinterpret_cast<float*>(stage + p.stage_g);
+  float* sbuf = reinterpret_cast<float*>(stage + kProStageG);
   // Stage this thread's four row segments (whole, aligned ones) first.
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -563,12 +557,9 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
   return ss;
 }
 
-// Four resident blocks per SM (64 registers, 48 KB of staging with bf16
-// gradients); the instantiation that averages several ranks' gradients needs
-// more registers and runs with fewer blocks.
 template <typename E, bool kRanks = false>
-__global__ void __launch_bounds__(kPThreads, kRanks ? 2 : 4) prologue_kernel(const __grid_constant__ ElemParams p) {
-  extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes16 or kProSmemBytes
+__global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
+  extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
   // A block's items only move forward through the matrices: one search,
@@ -996,18 +987,28 @@ __global__ void __launch_bounds__(kPThreads, 4) clip_norm_kernel(const __grid_co
   }
 }
 
-__global__ void __launch_bounds__(256) clip_finalize_kernel(const __grid_constant__ ClipFinalizeParams p) {
-  __shared__ double red[8];
+// One block of 1024 threads per segment; each thread keeps four running sums
+// (four loads in flight) over a fixed stride, so the order is fixed.
+constexpr int kClipFinThreads = 1024;
+__global__ void __launch_bounds__(kClipFinThreads) clip_finalize_kernel(const __grid_constant__ ClipFinalizeParams p) {
+  __shared__ double red[kClipFinThreads / 32];
   const int s = blockIdx.x;
-  double acc = 0.0;
-  for (int64_t i = p.seg_item0[s] + threadIdx.x; i < p.seg_item0[s + 1]; i += blockDim.x) acc += p.partials[i];
+  const int64_t b = p.seg_item0[s], e = p.seg_item0[s + 1];
+  double a4[4] = {0.0, 0.0, 0.0, 0.0};
+  int64_t i = b + threadIdx.x;
+  for (; i + 3 * kClipFinThreads < e; i += 4 * kClipFinThreads) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a4[u] += p.partials[i + u * kClipFinThreads];
+  }
+  for (int u = 0; i < e; i += kClipFinThreads, ++u) a4[u] += p.partials[i];
+  double acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {
     double tot = 0.0;
-    for (int w = 0; w < 8; ++w) tot += red[w];
+    for (int w = 0; w < kClipFinThreads / 32; ++w) tot += red[w];
     const double nrm = sqrt(tot);
     const double c = static_cast<double>(p.max_norm[s]) / (nrm + 1e-6);
     const float cf = static_cast<float>(c < 1.0 ? c : 1.0);   // a NaN norm gives 1
