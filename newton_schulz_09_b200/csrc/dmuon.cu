@@ -434,13 +434,13 @@ int classify_pointer(const void* p) {
   return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) ? DMUON_OK : DMUON_ERR_INVALID_ARG;
 }
 
-int check_device_ptr(int dev, const void* p, int i, const char* what) {
+int check_device_ptr(int dev, const void* p, int i, const char* what, const char* kind = "matrix") {
   if (p == nullptr) return DMUON_OK;
   std::unordered_set<const void*>& seen = g_checked[dev];
   if (seen.count(p)) return DMUON_OK;
   if (classify_pointer(p) != DMUON_OK)
-    return fail(DMUON_ERR_INVALID_ARG, "matrix %d: %s is not device memory (host memory cannot be "
-                "passed to the kernels)", i, what);
+    return fail(DMUON_ERR_INVALID_ARG, "%s %d: %s is not device memory (host memory cannot be "
+                "passed to the kernels)", kind, i, what);
   if (seen.size() >= 65536) seen.clear();
   seen.insert(p);
   return DMUON_OK;
@@ -1122,6 +1122,8 @@ int run(const std::vector<MatIn>& in, void* ws, size_t ws_bytes, bool own_ws, co
       return fail(DMUON_ERR_NO_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed",
                   ws_bytes, need);
     if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    r = check_device_ptr(dev, ws, 0, "the workspace", "argument");
+    if (r != DMUON_OK) return r;
   }
   // Every group's plan before any kernel of the call is enqueued (a new
   // plan's upload writes library memory only).  Groups with the same shapes
@@ -1294,6 +1296,8 @@ int run_host(const std::vector<MatIn>& in, const std::vector<const void*>& hg,
       return fail(DMUON_ERR_NO_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed",
                   ws_bytes, need);
     if (!aligned(ws, 256)) return fail(DMUON_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    r = check_device_ptr(dev, ws, 0, "the workspace", "argument");
+    if (r != DMUON_OK) return r;
   }
   // Every group's plan before any copy is enqueued (a new plan's upload
   // writes library memory only).  The cache holds more plans than
@@ -1683,6 +1687,14 @@ int dmuon_adamw_step_batched(void* const params[], const void* const grads[], fl
   int dev = 0;
   int r = current_device(&dev);
   if (r != DMUON_OK) return r;
+  for (size_t k = 0; k < ts.size() && r == DMUON_OK; ++k) {
+    const int i = static_cast<int>(k);
+    r = check_device_ptr(dev, ts[k].p, i, "the parameter", "tensor");
+    if (r == DMUON_OK) r = check_device_ptr(dev, ts[k].g, i, "the gradient", "tensor");
+    if (r == DMUON_OK) r = check_device_ptr(dev, ts[k].m, i, "exp_avg", "tensor");
+    if (r == DMUON_OK) r = check_device_ptr(dev, ts[k].v, i, "exp_avg_sq", "tensor");
+  }
+  if (r != DMUON_OK) return r;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const double bc1 = 1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step));
   const double bc2 = 1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step));
@@ -1794,6 +1806,12 @@ int dmuon_clip_grad_norm_buckets(void* const grads[], const dmuon_grad_desc desc
   std::lock_guard<std::mutex> lk(g_api_mu);
   int dev = 0;
   r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  for (size_t k = 0; k < ts.size() && r == DMUON_OK; ++k)
+    r = check_device_ptr(dev, ts[k].g, idx[k], "the gradient", "tensor");
+  if (r == DMUON_OK) r = check_device_ptr(dev, norms_out, 0, "norms_out", "output");
+  if (r == DMUON_OK) r = check_device_ptr(dev, coefs_out, 0, "coefs_out", "output");
+  if (r == DMUON_OK) r = check_device_ptr(dev, workspace, 0, "the workspace", "argument");
   if (r != DMUON_OK) return r;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void* ws = workspace;
@@ -1992,6 +2010,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   std::lock_guard<std::mutex> lk(g_api_mu);
   int dev = 0;
   r = current_device(&dev);
+  if (r != DMUON_OK) return r;
+  r = check_device_ptr(dev, X, 0, "X");
   if (r != DMUON_OK) return r;
   uint8_t* base = nullptr;
   r = static_scratch_address(dev, &base);

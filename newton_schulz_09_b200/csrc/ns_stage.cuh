@@ -406,6 +406,9 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 #pragma unroll
     for (int s = 0; s < kStages; ++s) { issued[s] = false; issued_phase[s] = 0; }
     int fenced = -1;     // matrix whose tensor maps this thread has acquired
+    // SYRK: the iterate is read by both operand streams of every tile and, for
+    // a 4096-row matrix, by two waves of CTAs; keep it in L2 between them.
+    const uint64_t keep = l2_evict_last();
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
       const TileInfo ti = decode_tile<kMode, BK>(p, t);
       const MatDesc& md = p.mats[ti.mi];
@@ -455,6 +458,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 #pragma unroll
             for (int h = 0; h < EB; ++h)
               tma_load_2d(a_dst + h * (BK * 128), mapAt, &full[stage], ti.tm * kBM + h * (128 / EB), kb * BK);
+          } else if (kMode == kSyrk) {
+            tma_load_2d_hint(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM, keep);
           } else {
             tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
           }
@@ -463,10 +468,13 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
           } else if (kMode != kGemm && nb == 2) {
             // Both 128-row halves of the B operand in one 256-row load.
-            tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
+            if (kMode == kSyrk) tma_load_2d_hint(b_dst, mapBw, &full[stage], kb * BK, b_row0, keep);
+            else tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
           } else {
             for (int j = 0; j < nb; ++j) {
-              if (kMode != kGemm)
+              if (kMode == kSyrk)
+                tma_load_2d_hint(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128, keep);
+              else if (kMode != kGemm)
                 tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
               else
                 tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);

@@ -156,6 +156,20 @@ def test_host_memory_is_refused_before_anything_is_enqueued(cuda_lib):
     S = (dm.DmuonShape * 1)(dm.DmuonShape(128, 256, dm.DMUON_BF16, dm.DMUON_BF16))
     r = lib.dmuon_muon_step_batched(P, G, B, S, 1, 0.02, 0.95, 1, 0.0, 5, None)
     assert r == -1 and "not device memory" in dm.dmuon_last_error()
+    # the clip and AdamW entry points check their tensors too
+    D = (dm.DmuonGradDesc * 1)(dm.DmuonGradDesc(hg.numel(), dm.DMUON_BF16, 0))
+    M = (ctypes.c_float * 1)(1.0)
+    r = lib.dmuon_clip_grad_norm_buckets(G, D, 1, M, 1, None, None, None, 0, None)
+    assert r == -1 and "not device memory" in dm.dmuon_last_error()
+    m = torch.zeros(hg.numel(), dtype=torch.float32, device=DEV)
+    v = torch.zeros(hg.numel(), dtype=torch.float32, device=DEV)
+    TD = (dm.DmuonTensorDesc * 1)(dm.DmuonTensorDesc(hg.numel(), dm.DMUON_BF16, dm.DMUON_BF16))
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    r = lib.dmuon_adamw_step_batched(ctypes.cast(P, pp), ctypes.cast(G, pp),
+                                     ctypes.cast((ctypes.c_void_p * 1)(m.data_ptr()), pp),
+                                     ctypes.cast((ctypes.c_void_p * 1)(v.data_ptr()), pp),
+                                     TD, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, None)
+    assert r == -1 and "not device memory" in dm.dmuon_last_error()
     assert dm.dmuon_launch_count() == n0
     torch.cuda.synchronize()
     assert not p.any() and not b.any()
