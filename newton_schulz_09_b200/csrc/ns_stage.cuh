@@ -406,9 +406,6 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 #pragma unroll
     for (int s = 0; s < kStages; ++s) { issued[s] = false; issued_phase[s] = 0; }
     int fenced = -1;     // matrix whose tensor maps this thread has acquired
-    // SYRK: the iterate is read by both operand streams of every tile and, for
-    // a 4096-row matrix, by two waves of CTAs; keep it in L2 between them.
-    const uint64_t keep = l2_evict_last();
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
       const TileInfo ti = decode_tile<kMode, BK>(p, t);
       const MatDesc& md = p.mats[ti.mi];
@@ -435,7 +432,13 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         nb = (left + BK - 1) / BK;
         if (nb > NBOX_B) nb = NBOX_B;
       }
-      const uint32_t bytes = kAStageBytes + static_cast<uint32_t>(nb) * BOX_B_BYTES;
+      // Diagonal tiles of the SYRK / SQUARE: on the full one (I = 2J) the A
+      // operand's 128 rows are the first half of the B operand's 256, on the
+      // half tile (I = 2J+1) the B rows are the A rows.  One load serves both.
+      const bool a_in_b = (kMode != kGemm) && !ti.half && ti.tm == 2 * ti.tn;
+      const bool b_is_a = (kMode != kGemm) && ti.half;
+      const uint32_t bytes = (a_in_b ? 0u : static_cast<uint32_t>(kAStageBytes)) +
+                             (b_is_a ? 0u : static_cast<uint32_t>(nb) * BOX_B_BYTES);
       if (lane == 0 && ti.mi != fenced) {
         // The maps were written by a kernel (plan upload): order that write
         // before TMA reads them.
@@ -458,23 +461,20 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
 #pragma unroll
             for (int h = 0; h < EB; ++h)
               tma_load_2d(a_dst + h * (BK * 128), mapAt, &full[stage], ti.tm * kBM + h * (128 / EB), kb * BK);
-          } else if (kMode == kSyrk) {
-            tma_load_2d_hint(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM, keep);
-          } else {
+          } else if (!a_in_b) {
             tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
           }
           if (kMode == kGemm && md.b3d) {
             // The four 64-column blocks of the tile in one load, same smem layout.
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
+          } else if (b_is_a) {
+            // half tile: its B rows are its A rows, already loaded
           } else if (kMode != kGemm && nb == 2) {
             // Both 128-row halves of the B operand in one 256-row load.
-            if (kMode == kSyrk) tma_load_2d_hint(b_dst, mapBw, &full[stage], kb * BK, b_row0, keep);
-            else tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
+            tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
           } else {
             for (int j = 0; j < nb; ++j) {
-              if (kMode == kSyrk)
-                tma_load_2d_hint(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128, keep);
-              else if (kMode != kGemm)
+              if (kMode != kGemm)
                 tma_load_2d(b_dst + j * kAStageBytes, mapB, &full[stage], kb * BK, b_row0 + j * 128);
               else
                 tma_load_2d(b_dst + j * BOX_B_BYTES, mapB, &full[stage], ti.tn * kBN + j * BK, kb * BK);
@@ -507,13 +507,17 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
       const uint32_t idesc = (kMode != kGemm && ti.half) ? IDESC_HALF : IDESC;
       const int kb_t = (kMode == kGemm && p.a_upper) ? ti.tm * (kBM / BK) : 0;
+      const bool a_in_b = (kMode != kGemm) && !ti.half && ti.tm == 2 * ti.tn;   // as the producer
+      const bool b_is_a = (kMode != kGemm) && ti.half;
       for (int kb = 0; kb < ti.nkb; ++kb) {
         w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_base = smem_u32(sa + stage * kAStageBytes);
-          const uint32_t b_base = smem_u32(sb + stage * kBStageBytes);
+          const uint32_t a_own = smem_u32(sa + stage * kAStageBytes);
+          const uint32_t b_own = smem_u32(sb + stage * kBStageBytes);
+          const uint32_t a_base = a_in_b ? b_own : a_own;
+          const uint32_t b_base = b_is_a ? a_own : b_own;
           const bool at = kb < kb_t;      // A k-block transposed (MN-major)
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
