@@ -377,6 +377,12 @@ int device_setup(int dev) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kNsSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
   }
+  const void* ks2[] = {reinterpret_cast<const void*>(&syrk256_kernel<__nv_bfloat16>),
+                       reinterpret_cast<const void*>(&syrk256_kernel<float>)};
+  for (const void* k : ks2) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kS2SmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+  }
   const void* pk[] = {reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16, false>),
                       reinterpret_cast<const void*>(&prologue_kernel<float, false>),
                       reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16, true>),
@@ -446,12 +452,17 @@ int check_device_ptr(int dev, const void* p, int i, const char* what, const char
   return DMUON_OK;
 }
 
-// SYRK tiles of an m x m Gram: column bands of 256 with row bands 0..2J+1.
-// SYRK tiles of an m x m Gram: column bands of 256 with row bands 0..2J+1
-// of 128.
+// 128 x 256 tiles of an m x m Gram (the quintic plans' SYRK, whose A is
+// mirrored, and the SQUARE stage): column bands of 256 with row bands
+// 0..2J+1 of 128.
 int64_t syrk_tiles_of(int64_t m) {
   const int64_t nJ = cdiv(m, kBN), nI = cdiv(m, kBM);
   return (nJ - 1) * nJ + nI;
+}
+// 256 x 256 upper tiles of an m x m Gram (syrk256_kernel: the cubic plans).
+int64_t syrk256_tiles_of(int64_t m) {
+  const int64_t nJ = cdiv(m, kBN);
+  return nJ * (nJ + 1) / 2;
 }
 int64_t gemm_tiles_of(int64_t m, int64_t n) { return cdiv(m, kBM) * cdiv(n, kBN); }
 
@@ -622,7 +633,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     A.gp.push_back(0);
     A.qp.push_back(0);
     for (int k = 0; k < gp.nmat; ++k) {
-      st += syrk_tiles_of(descs[first + so[k]].m);
+      st += quintic ? syrk_tiles_of(descs[first + so[k]].m) : syrk256_tiles_of(descs[first + so[k]].m);
       gt += gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
       qt += syrk_tiles_of(descs[first + go[k]].m);   // SQUARE contracts over m: the GEMM's order
       A.sp.push_back(static_cast<int>(st));
@@ -922,7 +933,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     np.ntiles = g.syrk_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_SYRK);
-      launch_ns_stage<kSyrk, E>(np, d, st);
+      if (P.quintic) launch_ns_stage<kSyrk, E>(np, d, st);   // mirrored A for the SQUARE stage
+      else syrk256_kernel<E><<<std::min(np.ntiles, d.sms), kNsThreads, kS2SmemBytes, st>>>(np);
     }
     if (P.quintic) {
       NsParams sq = np;
@@ -2041,7 +2053,7 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   d.g_bf16 = 1;
   d.vec4 = (n % 4 == 0) && aligned(X, 16);
   d.ptiles_c = static_cast<int>(ml.ptiles_c);
-  const int syrk_tiles = static_cast<int>(syrk_tiles_of(ml.m));
+  const int syrk_tiles = static_cast<int>(syrk256_tiles_of(ml.m));
   const int gemm_tiles = static_cast<int>(gemm_tiles_of(ml.m, ml.n));
   sp.order[0] = 0;
   sp.syrk_prefix[1] = syrk_tiles;
@@ -2117,7 +2129,7 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
       np.last = s == steps - 1;
       np.tile_prefix = dsp->syrk_prefix;
       np.ntiles = syrk_tiles;
-      launch_ns_stage<kSyrk, __nv_bfloat16>(np, di, st);
+      syrk256_kernel<__nv_bfloat16><<<std::min(np.ntiles, di.sms), kNsThreads, kS2SmemBytes, st>>>(np);
       np.tile_prefix = dsp->gemm_prefix;
       np.ntiles = gemm_tiles;
       launch_ns_stage<kGemm, __nv_bfloat16>(np, di, st);
