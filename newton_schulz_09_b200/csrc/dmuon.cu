@@ -258,6 +258,7 @@ struct GroupPlan {
   int first;              // first MatDesc index of the group
   int64_t ptiles;
   int syrk_tiles, gemm_tiles, square_tiles;
+  bool syrk256 = true;    // SYRK by syrk256_kernel (256 x 256 tiles), else ns_stage_kernel<kSyrk>
   const int* syrk_order; const int* syrk_prefix;
   const int* gemm_order; const int* gemm_prefix;
   const int* square_prefix;   // SQUARE tiles along gemm_order (quintic plans)
@@ -459,10 +460,23 @@ int64_t syrk_tiles_of(int64_t m) {
   const int64_t nJ = cdiv(m, kBN), nI = cdiv(m, kBM);
   return (nJ - 1) * nJ + nI;
 }
-// 256 x 256 upper tiles of an m x m Gram (syrk256_kernel: the cubic plans).
+// 256 x 256 upper tiles of an m x m Gram (syrk256_kernel).
 int64_t syrk256_tiles_of(int64_t m) {
   const int64_t nJ = cdiv(m, kBN);
   return nJ * (nJ + 1) / 2;
+}
+
+// Which SYRK kernel a group runs.  A 256 x 256 tile does twice the work of a
+// 128 x 256 tile in about 1.75 times its time (fewer operand bytes per FLOP),
+// but a group with few tiles has fewer CTAs working: compare the waves of
+// tiles over the SMs, each weighted by its tile time.  Small groups (the
+// TinyMLP, one 256 x 512 matrix) keep the 128 x 256 tiles; a 4096 x 4096
+// matrix (136 large tiles in one wave against 272 small ones in two) and the
+// Llama-8B groups take the large ones.
+bool use_syrk256(int64_t tiles128, int64_t tiles256, int sms) {
+  const double w128 = static_cast<double>(cdiv(tiles128, sms));
+  const double w256 = static_cast<double>(cdiv(tiles256, sms));
+  return 1.75 * w256 < w128;
 }
 int64_t gemm_tiles_of(int64_t m, int64_t n) { return cdiv(m, kBM) * cdiv(n, kBN); }
 
@@ -628,12 +642,19 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
       return x.m != y.m ? x.m > y.m : x.n > y.n;
     });
+    int64_t t128 = 0, t256 = 0;
+    for (int k = 0; k < gp.nmat; ++k) {
+      t128 += syrk_tiles_of(descs[first + k].m);
+      t256 += syrk256_tiles_of(descs[first + k].m);
+    }
+    gp.syrk256 = use_syrk256(t128, t256, g_dev[dev].sms);
     int64_t st = 0, gt = 0, qt = 0;
     A.sp.push_back(0);
     A.gp.push_back(0);
     A.qp.push_back(0);
     for (int k = 0; k < gp.nmat; ++k) {
-      st += quintic ? syrk_tiles_of(descs[first + so[k]].m) : syrk256_tiles_of(descs[first + so[k]].m);
+      const int64_t mk = descs[first + so[k]].m;
+      st += gp.syrk256 ? syrk256_tiles_of(mk) : syrk_tiles_of(mk);
       gt += gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
       qt += syrk_tiles_of(descs[first + go[k]].m);   // SQUARE contracts over m: the GEMM's order
       A.sp.push_back(static_cast<int>(st));
@@ -933,8 +954,8 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     np.ntiles = g.syrk_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_SYRK);
-      if (P.quintic) launch_ns_stage<kSyrk, E>(np, d, st);   // mirrored A for the SQUARE stage
-      else syrk256_kernel<E><<<std::min(np.ntiles, d.sms), kNsThreads, kS2SmemBytes, st>>>(np);
+      if (g.syrk256) syrk256_kernel<E><<<std::min(np.ntiles, d.sms), kNsThreads, kS2SmemBytes, st>>>(np);
+      else launch_ns_stage<kSyrk, E>(np, d, st);
     }
     if (P.quintic) {
       NsParams sq = np;
@@ -2053,7 +2074,8 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
   d.g_bf16 = 1;
   d.vec4 = (n % 4 == 0) && aligned(X, 16);
   d.ptiles_c = static_cast<int>(ml.ptiles_c);
-  const int syrk_tiles = static_cast<int>(syrk256_tiles_of(ml.m));
+  const bool big_syrk = use_syrk256(syrk_tiles_of(ml.m), syrk256_tiles_of(ml.m), g_dev[dev].sms);
+  const int syrk_tiles = static_cast<int>(big_syrk ? syrk256_tiles_of(ml.m) : syrk_tiles_of(ml.m));
   const int gemm_tiles = static_cast<int>(gemm_tiles_of(ml.m, ml.n));
   sp.order[0] = 0;
   sp.syrk_prefix[1] = syrk_tiles;
@@ -2129,7 +2151,10 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
       np.last = s == steps - 1;
       np.tile_prefix = dsp->syrk_prefix;
       np.ntiles = syrk_tiles;
-      syrk256_kernel<__nv_bfloat16><<<std::min(np.ntiles, di.sms), kNsThreads, kS2SmemBytes, st>>>(np);
+      if (big_syrk)
+        syrk256_kernel<__nv_bfloat16><<<std::min(np.ntiles, di.sms), kNsThreads, kS2SmemBytes, st>>>(np);
+      else
+        launch_ns_stage<kSyrk, __nv_bfloat16>(np, di, st);
       np.tile_prefix = dsp->gemm_prefix;
       np.ntiles = gemm_tiles;
       launch_ns_stage<kGemm, __nv_bfloat16>(np, di, st);

@@ -209,6 +209,7 @@ __device__ __forceinline__ int find_slot64(const int64_t* prefix, int n, int64_t
 
 }  // namespace dmuon
 #include "ns_stage.cuh"   // the Newton-Schulz stage kernel (depends on the types above)
+#include "syrk256.cuh"    // the SYRK stage (256 x 256 tiles)
 namespace dmuon {
 
 // ======================================================================

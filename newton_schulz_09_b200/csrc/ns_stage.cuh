@@ -1,8 +1,9 @@
-// Newton-Schulz stage kernel of the batched Muon update on sm_100a: one
+// Newton-Schulz stage kernels of the batched Muon update on sm_100a: one
 // persistent, warp-specialised tcgen05/TMEM/TMA launch per stage for every
-// matrix of a group (SYRK A = X X^T over upper tiles, the quintic SQUARE
-// P = b A + c A A, and the GEMM X' = c (a X + (A or P) X) with the fused
-// combine or weight update), with its tile decoding and epilogue.
+// matrix of a group.  ns_stage_kernel runs the GEMM X' = c (a X + (A or P) X)
+// with the fused combine or weight update, and the quintic SQUARE
+// P = b A + c A A, and the SYRK with 128 x 256 tiles for groups too small to
+// fill the SMs with the 256 x 256 tiles of syrk256_kernel (syrk256.cuh).
 //
 // Sources: DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销",
 // section "Muon 核心：Newton-Schulz 迭代" (the cubic step and the transpose
@@ -567,226 +568,5 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   }
 }
 
-// ======================================================================
-// SYRK with 256 x 256 tiles per CTA (the cubic step, where A is stored as its
-// upper triangle only).  Each k-block brings 256 rows of X for the A operand
-// and 256 for the B operand (64 KB) and feeds two 128 x 256 UMMA halves that
-// share the B operand: a third fewer operand bytes per FLOP than 128 x 256
-// tiles.  The two fp32 accumulators take all 512 TMEM columns, so a tile's
-// epilogue is not overlapped with the next tile's MMAs; with K = n in the
-// thousands that costs a few percent of the stage.  Diagonal tiles (I = J)
-// load one box for both operands, and their second half is 128 x 128 (the
-// block's lower-left quarter is below the diagonal).
-// Same warp roles as ns_stage_kernel; three 64 KB pipeline stages.
-// ======================================================================
-constexpr int kS2Stages = 3;
-constexpr int kS2OpBytes = kBN * 128;              // 256 rows x 128 bytes of K
-constexpr int kS2SmemBytes = kS2Stages * 2 * kS2OpBytes + 1024 /*align*/ + 256;
-static_assert(kS2SmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
-
-// Upper-triangle 256 x 256 tiles of one matrix, column-band major: band J
-// holds I = 0 .. J and starts at J (J + 1) / 2.
-__device__ __forceinline__ void syrk256_tile_coords(int local, int& I, int& J) {
-  int j = static_cast<int>((sqrtf(8.0f * static_cast<float>(local) + 1.0f) - 1.0f) * 0.5f);
-  while ((j + 1) * (j + 2) / 2 <= local) ++j;
-  while (j * (j + 1) / 2 > local) --j;
-  J = j;
-  I = local - j * (j + 1) / 2;
-}
-
-struct Tile256 {
-  int mi, I, J, nkb;
-  bool diag;
-};
-
-template <int BK>
-__device__ __forceinline__ Tile256 decode_tile256(const NsParams& p, int t) {
-  Tile256 ti;
-  const int slot = find_slot(p.tile_prefix, p.nmat, t);
-  ti.mi = __ldg(p.order + slot);
-  syrk256_tile_coords(t - __ldg(p.tile_prefix + slot), ti.I, ti.J);
-  ti.nkb = (p.mats[ti.mi].n + BK - 1) / BK;
-  ti.diag = ti.I == ti.J;
-  return ti;
-}
-
-template <typename E>
-__global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_constant__ NsParams p) {
-  constexpr int EB = static_cast<int>(sizeof(E));
-  constexpr int BK = 128 / EB;
-  constexpr int MMA_K = 32 / EB;
-  constexpr int KSTEPS = BK / MMA_K;
-  constexpr uint32_t FMT = (EB == 2) ? 1u : 2u;
-  constexpr uint32_t IDESC = make_idesc(FMT, 0u, 0u, kBM, kBN);
-  constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  // stage s: A operand rows at s * 64 KB, B operand rows 32 KB after them
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kS2Stages * 2 * kS2OpBytes);
-  uint64_t* empty = full + kS2Stages;
-  uint64_t* tfull = empty + kS2Stages;
-  uint64_t* tempty = tfull + 1;
-  uint64_t* drain = tempty + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kS2Stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 4 * 32);
-    mbar_init(drain, 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
-
-  bool ok = true;
-  if (warp == 0) {
-    // ------------------------------------------------ TMA producer
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_phase[kS2Stages];
-    bool issued[kS2Stages];
-#pragma unroll
-    for (int s = 0; s < kS2Stages; ++s) { issued[s] = false; issued_phase[s] = 0; }
-    int fenced = -1;
-    for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
-      const CUtensorMap* map = &p.maps[ti.mi].xkw[p.cur];     // 256-row K-major boxes of X
-      if (lane == 0 && ti.mi != fenced) {
-        tensormap_acquire_gpu(map);
-        fenced = ti.mi;
-      }
-      const uint32_t bytes = ti.diag ? kS2OpBytes : 2 * kS2OpBytes;
-      for (int kb = 0; kb < ti.nkb; ++kb) {
-        bool w = mbar_wait(&empty[stage], phase ^ 1u, p.err, p.wait_limit_ns);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          uint8_t* a_dst = smem + stage * 2 * kS2OpBytes;
-          if (!ti.diag) tma_load_2d(a_dst, map, &full[stage], kb * BK, ti.I * kBN);
-          tma_load_2d(a_dst + kS2OpBytes, map, &full[stage], kb * BK, ti.J * kBN);
-        }
-        __syncwarp();
-        issued[stage] = true;
-        issued_phase[stage] = phase;
-        if (++stage == kS2Stages) { stage = 0; phase ^= 1u; }
-      }
-    }
-    if (!ok && lane == 0) {
-      for (int s = 0; s < kS2Stages; ++s)
-        if (issued[s]) mbar_wait(&full[s], issued_phase[s], nullptr, p.wait_limit_ns, 1024);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ UMMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int lt = 0;
-    for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
-      bool w = mbar_wait(tempty, (static_cast<uint32_t>(lt) & 1u) ^ 1u, p.err, p.wait_limit_ns);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
-      for (int kb = 0; kb < ti.nkb; ++kb) {
-        w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t own = smem_u32(smem + stage * 2 * kS2OpBytes);
-          const uint32_t b_base = own + kS2OpBytes;
-          const uint32_t a_base = ti.diag ? b_base : own;
-#pragma unroll
-          for (int k = 0; k < KSTEPS; ++k) {
-            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t ad = sw128_desc(a_base + h * (kS2OpBytes / 2) + k * 32, 16, 1024);
-              const bool quarter = ti.diag && h == 1;   // 128 x 128 over the B rows 128 .. 255
-              const uint64_t bd = sw128_desc(b_base + (quarter ? kS2OpBytes / 2 : 0) + k * 32, 16, 1024);
-              const uint32_t d = tmem_base + static_cast<uint32_t>(h * kBN);
-              if (EB == 2) umma_f16(d, ad, bd, quarter ? IDESC_HALF : IDESC, acc);
-              else umma_tf32(d, ad, bd, quarter ? IDESC_HALF : IDESC, acc);
-            }
-          }
-          umma_commit(&empty[stage]);
-        }
-        __syncwarp();
-        if (++stage == kS2Stages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) break;
-      if (lane == 0) umma_commit(tfull);
-      __syncwarp();
-    }
-    if (!ok && lane == 0) {
-      umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, p.wait_limit_ns, 1024);
-    }
-  } else {
-    // ------------------------------------------------ epilogue (4 warps)
-    const int q4 = warp & 3;
-    const int row_in_tile = q4 * 32 + lane;
-    int lt = 0;
-    for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
-      const MatDesc& md = p.mats[ti.mi];
-      const float s = *md.scale;
-      bool w = mbar_wait(tfull, static_cast<uint32_t>(lt) & 1u, p.err, p.wait_limit_ns);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
-      const float alpha = p.first ? s * s : 1.0f;
-      E* A = reinterpret_cast<E*>(md.A);
-      const int64_t lda = md.lda;
-      const int m = md.m;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const bool quarter = ti.diag && h == 1;
-        const int R = ti.I * kBN + h * kBM + row_in_tile;
-        const int col0 = ti.J * kBN + (quarter ? kBN / 2 : 0);
-        const int nch = quarter ? kBN / 64 : kBN / 32;
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(h * kBN);
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_ld_wait();
-          const int C0 = col0 + c * 32;
-          if (R < m && C0 < m) {
-            float y[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = op_round<E>(alpha * __uint_as_float(v[j]));
-            E* arow = A + static_cast<int64_t>(R) * lda;
-            if (C0 + 32 <= m) {
-              store32<E>(arow + C0, y);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (C0 + j < m) arow[C0 + j] = from_f<E>(y[j]);
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(tempty);
-    }
-  }
-
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
-  }
-}
 
 }  // namespace dmuon
