@@ -1632,8 +1632,8 @@ size_t dmuon_ns_workspace_bytes(int64_t m, int64_t n, int dtype) {
 const char* dmuon_last_error(void) { return t_last_error.c_str(); }
 
 const char* dmuon_backend_string(void) {
-  return "cubic Newton-Schulz · tcgen05 UMMA 128x256 SYRK (upper tiles) + GEMM (fused combine/update) "
-         "· TMA 128B-swizzle · TMEM double buffer · sm_100a";
+  return "cubic Newton-Schulz · tcgen05 UMMA SYRK (upper 256x256 tiles, two halves sharing B) + GEMM "
+         "128x256 (fused combine/update, transposed lower A) · TMA 128B-swizzle · TMEM · sm_100a";
 }
 
 int dmuon_device_status(int clear) {
