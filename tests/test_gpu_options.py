@@ -171,3 +171,25 @@ def test_quintic_caller_workspace_size(cuda_lib):
     with pytest.raises(dm.DmuonError):
         dm.dmuon_muon_step_batched_opts(params, grads, bufs, ns_coefficients=QUINTIC[0],
                                         workspace=ws[:cubic])
+
+
+@pytest.mark.slow
+def test_quintic_on_the_large_tile_syrk(cuda_lib):
+    """A 4096 x 4096 matrix runs its SYRK with 256 x 256 tiles (136 tiles in one
+    wave against 272 small ones in two); in the quintic step that kernel also
+    writes the mirrored lower triangle, which the SQUARE stage reads.  Against
+    the oracle's quintic step."""
+    dm = cuda_lib
+    s = (4096, 4096)
+    p = torch.zeros(s, dtype=torch.bfloat16, device=DEV)
+    g = _rand(s, torch.bfloat16, 90, 1e-3)
+    b = torch.zeros(s, dtype=torch.float32, device=DEV)
+    dm.dmuon_muon_step_batched_opts([p], [g], [b], lr=0.05, nesterov=True, ns_steps=3,
+                                    ns_coefficients=QUINTIC[0])
+    torch.cuda.synchronize()
+    assert dm.dmuon_device_status() == 0
+    buf_ref, X, W_ref = oracle.muon_step(np.zeros(s, np.float32), host(g), np.zeros(s, np.float32), lr=0.05,
+                                         momentum=0.95, nesterov=True, weight_decay=0.0, ns_steps=3,
+                                         ns_coeffs=QUINTIC[0])
+    assert np.array_equal(host(b).view(np.uint32), buf_ref.view(np.uint32))
+    check_rel(host(p), W_ref, TOL_BF16, "quintic 4096^2 (256 x 256 SYRK tiles)")
