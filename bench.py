@@ -449,6 +449,8 @@ def measure_config(name, dm, dev, peaks, steps, cpu):
                                 "measured_burst": tf / peaks["bf16_tflops"],
                                 "nominal_2250": tf / NOMINAL_BF16_TFLOPS},
            "stage_ms_per_step": stages}
+    if name == "mixed1024":
+        out["small_matrices"] = measure_small_class(dm, dev, wl, t, peaks, steps)
     sweep = None
     if name == "square4096":
         sweep = []
@@ -466,6 +468,47 @@ def measure_config(name, dm, dev, peaks, steps, cpu):
     del t
     torch.cuda.empty_cache()
     return out
+
+
+def measure_small_class(dm, dev, wl, t, peaks, steps, max_side=256):
+    """The mixed workload's narrow matrices (short side <= max_side) as a call of
+    their own.  Their Newton-Schulz work is too small to bound them by the tensor
+    cores, so they are reported against HBM: 16 bytes of unavoidable traffic per
+    element (gradient 2, momentum read and write 8, X0 2, weight read and write
+    4; the iterates of matrices this small stay in L2)."""
+    import torch
+    idx = [i for i, s in enumerate(wl.specs) if min(s.rows, s.cols) <= max_side]
+    if not idx:
+        return None
+    ps, gs, bs = [t.params[i] for i in idx], [t.grads[i] for i in idx], [t.bufs[i] for i in idx]
+
+    def step():
+        dm.dmuon_muon_step_batched(ps, gs, bs, lr=wl.lr, momentum=wl.momentum, nesterov=wl.nesterov,
+                                   weight_decay=wl.weight_decay, ns_steps=wl.ns_steps)
+
+    for _ in range(3):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    elems = sum(wl.specs[i].rows * wl.specs[i].cols for i in idx)
+    fl = wl.ns_steps * sum(3.0 * min(wl.specs[i].rows, wl.specs[i].cols) ** 2 *
+                           max(wl.specs[i].rows, wl.specs[i].cols) for i in idx)
+    hbm = 16.0 * elems
+    gbs = hbm / (ms * 1e-3) / 1e9
+    return {"max_short_side": max_side, "matrices": len(idx), "elements": elems,
+            "ms_per_step": ms, "useful_flops_per_step": fl, "tflops": fl / (ms * 1e-3) / 1e12,
+            "bound": "hbm", "hbm_bytes_per_step": hbm, "achieved_gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "note": "one call of these matrices alone; launch and pipeline-fill latency, not HBM "
+                    "bandwidth, sets most of the time"}
 
 
 def oracle_config_time(wl, host, prior, sub, sweep, G=None):
