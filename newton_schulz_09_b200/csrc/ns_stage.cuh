@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         fenced = ti.mi;
       }
       for (int kb = 0; kb < ti.nkb; ++kb) {
-        bool w = mbar_wait(&empty[stage], phase ^ 1u, p.err, p.wait_limit_ns);
+        bool w = mbar_wait_spin(&empty[stage], phase ^ 1u, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], bytes);
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const TileInfo ti = decode_tile<kMode, BK>(p, t);
       const int b = lt & 1;
       const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
-      bool w = mbar_wait(&tempty[b], tph ^ 1u, p.err, p.wait_limit_ns);
+      bool w = mbar_wait_spin(&tempty[b], tph ^ 1u, p.err, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const bool a_in_b = (kMode != kGemm) && !ti.half && ti.tm == 2 * ti.tn;   // as the producer
       const bool b_is_a = (kMode != kGemm) && ti.half;
       for (int kb = 0; kb < ti.nkb; ++kb) {
-        w = mbar_wait(&full[stage], phase, p.err, p.wait_limit_ns);
+        w = mbar_wait_spin(&full[stage], phase, p.err, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {

@@ -74,6 +74,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   }
 }
 
+// Non-blocking probe of phase `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait for the producer and UMMA warps, whose waits are short and on
+// the critical path: the warp keeps polling instead of sleeping in try_wait,
+// so it resumes as soon as the phase completes.  Same bounds as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, int* err,
+                                               uint64_t limit_ns, uint32_t min_polls = 256) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 15u) == 0u) {
+      if (err != nullptr && *reinterpret_cast<volatile int*>(err) != 0) return false;
+      if (it >= min_polls && global_timer_ns() - t0 > limit_ns) {
+        if (err != nullptr) atomicCAS(err, 0, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------------- TMA
 // 2-D tiled bulk-tensor load global -> shared, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
