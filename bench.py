@@ -37,8 +37,8 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage: the ncu
 # capture of one Llama-8B layer (529.2 MB read + 407.2 MB written for 1.735e12 useful FLOPs);
 # a launch of the full workload covers several layers, so its traffic is this ratio times the
-# useful FLOPs of that launch.  Valid only for the stage kernel's source it was measured on
-# (ns_stage.cuh and ptx.cuh).
+# useful FLOPs of that launch.  Valid only for the stage kernels' source it was measured on
+# (ns_stage.cuh, gemm_pair.cuh and ptx.cuh).
 PROFILED_TRAFFIC = {"kernel_sha256_prefix": "a96e166e9347b1ad", "workload": "llama8b",
                     "gemm_bytes_per_useful_flop": 0.9365e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -73,7 +73,8 @@ def profiled_traffic(workload: str):
     import hashlib
     csrc = os.path.join(HERE, "newton_schulz_09_b200", "csrc")
     try:
-        data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("ns_stage.cuh", "ptx.cuh"))
+        data = b"".join(open(os.path.join(csrc, f), "rb").read()
+                        for f in ("ns_stage.cuh", "gemm_pair.cuh", "ptx.cuh"))
     except OSError:
         return None
     sha = hashlib.sha256(data).hexdigest()
@@ -654,8 +655,12 @@ def run_ours(args):
     gemm_launches_step = gemm_n / args.steps if gemm_n else None
     fl_per_launch = gemm_fl_step / gemm_launches_step if gemm_n else None
     bpf = profiled_traffic(wl.name)
+    plan = dm.dmuon_debug_last_plan()
+    pair = bool(plan) and all(g["gemm_pair"] for g in plan)
     roofline = {
-        "kernel": "ns_stage_kernel<GEMM, bf16>", "bound": "tensor",
+        "kernel": "gemm_pair_kernel (256 x 256 tiles on CTA pairs, bf16)" if pair
+                  else "ns_stage_kernel<GEMM, bf16>",
+        "bound": "tensor",
         "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
         "frac": (gemm_tf / peak) if gemm_tf else None,
         "traffic": (bpf * fl_per_launch) if (bpf and fl_per_launch) else None,

@@ -351,6 +351,17 @@ void dmuon_release_cache(void);
  * before builds none, whatever its tensor addresses). */
 int64_t dmuon_plan_builds(void);
 
+/* Test hook (host only, launches nothing): the stage kernels of the launch
+ * plan used most recently (by the last call, or the plan it built).  Writes
+ * one word per dtype group (at most max_groups; kernels may be NULL) and
+ * returns the plan's number of groups, 0 when no plan exists.  Each word
+ * ORs DMUON_PLAN_SYRK256 (the SYRK runs on 256 x 256 tiles, else 128 x 256)
+ * and DMUON_PLAN_GEMM_PAIR (the GEMM runs 256 x 256 tiles on two-CTA
+ * clusters, else 128 x 256 tiles on single CTAs). */
+#define DMUON_PLAN_SYRK256 1
+#define DMUON_PLAN_GEMM_PAIR 2
+int dmuon_debug_last_plan(int* kernels, int max_groups);
+
 /* Test hook (host only, launches nothing): the device-memory check the entry
  * points apply to every tensor address.  DMUON_OK for device or managed
  * memory, DMUON_ERR_INVALID_ARG for host memory (page-locked or not) and

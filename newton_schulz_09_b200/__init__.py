@@ -22,7 +22,7 @@ __all__ = [
     "dmuon_last_error", "dmuon_backend_string", "dmuon_device_status", "dmuon_release_cache",
     "dmuon_debug_fail_allocations", "dmuon_debug_wait_timeout", "dmuon_stage_timing",
     "dmuon_stage_times", "dmuon_launch_count", "KERNEL_KINDS", "dmuon_ns_orthogonalize_noalloc",
-    "dmuon_plan_builds", "dmuon_debug_check_pointer",
+    "dmuon_plan_builds", "dmuon_debug_check_pointer", "dmuon_debug_last_plan",
     "dmuon_muon_step_batched_opts", "DmuonStepOptions", "DMUON_LR_PLAIN", "DMUON_LR_SQRT_MAX",
     "dmuon_adamw_step_batched", "DmuonTensorDesc", "dmuon_muon_step_batched_host",
     "dmuon_muon_step_batched_reduce", "dmuon_clip_grad_norm_buckets", "dmuon_clip_workspace_bytes",
@@ -137,6 +137,7 @@ def load_library() -> ctypes.CDLL:
         "dmuon_workspace_bytes_opts": (sz, [sp, i32, ctypes.POINTER(DmuonStepOptions)]),
         "dmuon_plan_builds": (ctypes.c_int64, []),
         "dmuon_debug_check_pointer": (i32, [vp]),
+        "dmuon_debug_last_plan": (i32, [ctypes.POINTER(i32), i32]),
         "dmuon_clip_grad_norm_buckets": (i32, [pp, ctypes.POINTER(DmuonGradDesc), i32,
                                                ctypes.POINTER(ctypes.c_float), i32, vp, vp, vp, sz, vp]),
     }
@@ -482,6 +483,16 @@ def dmuon_launch_count() -> int:
 def dmuon_plan_builds() -> int:
     """Launch plans built so far (shapes seen before build none)."""
     return int(load_library().dmuon_plan_builds())
+
+
+def dmuon_debug_last_plan() -> list:
+    """Stage kernels of the most recently used launch plan, one dict per
+    dtype group: {"syrk256": bool, "gemm_pair": bool} (launches nothing)."""
+    lib = load_library()
+    n = int(lib.dmuon_debug_last_plan(None, 0))
+    words = (ctypes.c_int32 * max(n, 1))()
+    lib.dmuon_debug_last_plan(words, n)
+    return [{"syrk256": bool(words[i] & 1), "gemm_pair": bool(words[i] & 2)} for i in range(n)]
 
 
 def dmuon_debug_check_pointer(address: int) -> int:

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdmuon.so")
 
 SOURCES = ["dmuon.cu"]
-DEPS = ["dmuon.cu", "kernels.cuh", "ns_stage.cuh", "syrk256.cuh", "ptx.cuh"]
+DEPS = ["dmuon.cu", "kernels.cuh", "ns_stage.cuh", "syrk256.cuh", "gemm_pair.cuh", "ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -110,12 +110,13 @@ bool encode_2d(CUtensorMap* map, int dtype, void* base, uint64_t inner, uint64_t
 // box is the 64 x 256 MN-major operand tile that four 2-D boxes would bring,
 // in the same shared-memory layout (four 8 KB blocks); in the last column
 // tile, blocks past the last column are out of bounds and arrive as zeros.
-bool encode_mn3d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t pitch_elems) {
+bool encode_mn3d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t pitch_elems,
+                 uint32_t blocks = 4) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || cols % 64 != 0) return false;
   cuuint64_t dims[3] = {64, rows, cols / 64};
   cuuint64_t strides[2] = {pitch_elems * 2, 128};
-  cuuint32_t box[3] = {64, 64, 4};
+  cuuint32_t box[3] = {64, 64, blocks};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -259,6 +260,7 @@ struct GroupPlan {
   int64_t ptiles;
   int syrk_tiles, gemm_tiles, square_tiles;
   bool syrk256 = true;    // SYRK by syrk256_kernel (256 x 256 tiles), else ns_stage_kernel<kSyrk>
+  bool gemm_pair = false; // GEMM by gemm_pair_kernel (256 x 256 tiles on CTA pairs)
   const int* syrk_order; const int* syrk_prefix;
   const int* gemm_order; const int* gemm_prefix;
   const int* square_prefix;   // SQUARE tiles along gemm_order (quintic plans)
@@ -304,6 +306,7 @@ struct Plan {
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
+  int pair_clusters = 0;   // co-resident two-CTA clusters of gemm_pair_kernel (0: not used)
   int* err = nullptr;
   cudaMemPool_t pool = nullptr;
 };
@@ -383,6 +386,33 @@ int device_setup(int dev) {
   for (const void* k : ks2) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kS2SmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+  }
+  {
+    const void* k = reinterpret_cast<const void*>(&gemm_pair_kernel);
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kG2SmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(d.sms / 2), 1, 1);
+    cfg.blockDim = dim3(kNsThreads, 1, 1);
+    cfg.dynamicSmemBytes = kG2SmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    // Without a usable answer the pair GEMM is not used.
+    if (cudaOccupancyMaxActiveClusters(&nc, k, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      nc = 0;
+    }
+    d.pair_clusters = std::min(nc, d.sms / 2);
+    if (log_enabled())
+      std::fprintf(stderr, "dmuon: device %d: %d SMs, %d co-resident CTA pairs for the pair GEMM\n", dev,
+                   d.sms, nc);
   }
   const void* pk[] = {reinterpret_cast<const void*>(&prologue_kernel<__nv_bfloat16, false>),
                       reinterpret_cast<const void*>(&prologue_kernel<float, false>),
@@ -479,6 +509,8 @@ bool use_syrk256(int64_t tiles128, int64_t tiles256, int sms) {
   return 1.75 * w256 < w128;
 }
 int64_t gemm_tiles_of(int64_t m, int64_t n) { return cdiv(m, kBM) * cdiv(n, kBN); }
+// 256 x 256 tiles of the pair GEMM (gemm_pair_kernel).
+int64_t gemm_pair_tiles_of(int64_t m, int64_t n) { return cdiv(m, 2 * kBM) * cdiv(n, kBN); }
 
 // Builds (or finds) the plan for these matrices and this workspace.
 // 16-byte vector access of a matrix's parameter, gradient and buffer rows.
@@ -569,6 +601,21 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     gp.ptiles = g.ptiles;
     GroupArrays& A = ga[gi];
     A.pp.push_back(0);
+    {
+      // The SYRK kernel, then the GEMM kernel: CTA pairs for bf16 cubic
+      // groups on 256 x 256 SYRK tiles whose matrices have m % 256 == 0 and
+      // n % 64 == 0 (whole pair tiles, 3-D X operand loads).
+      int64_t t128 = 0, t256 = 0;
+      bool pair_ok = dt == DMUON_BF16 && !quintic && g_dev[dev].pair_clusters > 0;
+      for (int k = 0; k < gp.nmat; ++k) {
+        const MatLayout& ml = L.mats[g.idx[k]];
+        t128 += syrk_tiles_of(ml.m);
+        t256 += syrk256_tiles_of(ml.m);
+        pair_ok = pair_ok && ml.m % (2 * kBM) == 0 && ml.n % 64 == 0;
+      }
+      gp.syrk256 = use_syrk256(t128, t256, g_dev[dev].sms);
+      gp.gemm_pair = gp.syrk256 && pair_ok;
+    }
     for (int k = 0; k < gp.nmat; ++k) {
       const int i = g.idx[k];
       const MatIn& x = in[i];
@@ -607,7 +654,10 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
           if (d.Xop[b] && !encode_mn3d(&mm.xmn[b], d.Xop[b], ml.n, ml.m, ml.ldx)) d.b3d = 0;
         for (int b = 0; b < 2; ++b) {
           void* xb = d.Xop[b];
-          if (!xb) { mm.xk[b] = mm.xk[0]; mm.xkw[b] = mm.xkw[0]; mm.xmn[b] = mm.xmn[0]; continue; }
+          if (!xb) {
+            mm.xk[b] = mm.xk[0]; mm.xkw[b] = mm.xkw[0]; mm.xmn[b] = mm.xmn[0]; mm.xmn2[b] = mm.xmn2[0];
+            continue;
+          }
           okm &= encode_2d(&mm.xk[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBM);
           okm &= encode_2d(&mm.xkw[b], dt, xb, ml.n, ml.m, ml.ldx, BK, kBN);
           // MN-major 32-bit operands need 32-byte swizzle units.
@@ -615,6 +665,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
             okm &= encode_2d(&mm.xmn[b], dt, xb, ml.n, ml.m, ml.ldx, BK, BK,
                              dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                              : CU_TENSOR_MAP_SWIZZLE_128B);
+          if (gp.gemm_pair) okm &= d.b3d && encode_mn3d(&mm.xmn2[b], xb, ml.n, ml.m, ml.ldx, 2);
         }
         const CUtensorMapSwizzle mn_sw =
             dt == DMUON_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
@@ -642,12 +693,6 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
       return x.m != y.m ? x.m > y.m : x.n > y.n;
     });
-    int64_t t128 = 0, t256 = 0;
-    for (int k = 0; k < gp.nmat; ++k) {
-      t128 += syrk_tiles_of(descs[first + k].m);
-      t256 += syrk256_tiles_of(descs[first + k].m);
-    }
-    gp.syrk256 = use_syrk256(t128, t256, g_dev[dev].sms);
     int64_t st = 0, gt = 0, qt = 0;
     A.sp.push_back(0);
     A.gp.push_back(0);
@@ -655,7 +700,8 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     for (int k = 0; k < gp.nmat; ++k) {
       const int64_t mk = descs[first + so[k]].m;
       st += gp.syrk256 ? syrk256_tiles_of(mk) : syrk_tiles_of(mk);
-      gt += gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
+      gt += gp.gemm_pair ? gemm_pair_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n)
+                         : gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
       qt += syrk_tiles_of(descs[first + go[k]].m);   // SQUARE contracts over m: the GEMM's order
       A.sp.push_back(static_cast<int>(st));
       A.gp.push_back(static_cast<int>(gt));
@@ -940,6 +986,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   np.quintic = P.quintic ? 1 : 0;
   np.mirror = P.quintic ? 1 : 0;     // the SQUARE stage reads all of A
   np.a_upper = 1;                    // the GEMM reads A (or P) from its upper triangle
+  np.diag_full = g.gemm_pair ? 1 : 0;  // the pair GEMM reads whole diagonal 256-blocks
   np.ca = o.ca;
   np.cb = P.quintic ? 1.0f : o.cb;   // quintic: X <- a X + P X with P = b A + c A A
   np.cc = 0.0f;
@@ -973,7 +1020,10 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     np.ntiles = g.gemm_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_GEMM);
-      launch_ns_stage<kGemm, E>(np, d, st);
+      if (g.gemm_pair)
+        gemm_pair_kernel<<<2 * std::min(np.ntiles, d.pair_clusters), kNsThreads, kG2SmemBytes, st>>>(np);
+      else
+        launch_ns_stage<kGemm, E>(np, d, st);
     }
   }
 }
@@ -1669,6 +1719,17 @@ int64_t dmuon_plan_builds(void) {
   return g_plan_builds;
 }
 
+int dmuon_debug_last_plan(int* kernels, int max_groups) {
+  std::lock_guard<std::mutex> lk(g_api_mu);
+  if (g_plans.empty()) return 0;
+  const Plan& P = *g_plans.front();
+  const int n = static_cast<int>(P.groups.size());
+  for (int i = 0; i < n && i < max_groups; ++i)
+    if (kernels)
+      kernels[i] = (P.groups[i].syrk256 ? DMUON_PLAN_SYRK256 : 0) | (P.groups[i].gemm_pair ? DMUON_PLAN_GEMM_PAIR : 0);
+  return n;
+}
+
 int dmuon_debug_check_pointer(const void* p) {
   t_last_error.clear();
   if (p == nullptr) return fail(DMUON_ERR_INVALID_ARG, "NULL pointer");
@@ -2143,6 +2204,7 @@ extern "C" int dmuon_ns_orthogonalize_noalloc(void* X, int64_t m, int64_t n, int
     np.quintic = 0;
     np.mirror = 0;
     np.a_upper = 1;
+    np.diag_full = 0;
     np.err = di.err;
     np.wait_limit_ns = kWaitLimitNs;
     for (int s = 0; s < steps; ++s) {

@@ -88,6 +88,8 @@ struct alignas(64) MatMaps {
   CUtensorMap p;       // P as K-major operand (the GEMM's A operand in quintic mode)
   CUtensorMap amn;     // A as MN-major operand, box (128 B of M) x (BK rows of K): the GEMM
   CUtensorMap pmn;     // reads A's (or P's) lower k-blocks transposed from the upper triangle
+  CUtensorMap xmn2[2]; // with b3d: the 3-D view of xmn with a box of 2 blocks (128 columns),
+                       // one CTA's half of the B operand of a pair GEMM tile
 };
 
 struct NsParams {
@@ -107,6 +109,9 @@ struct NsParams {
   int mirror;              // SYRK / SQUARE: also write the lower triangle (A^T of the upper)
   int a_upper;             // GEMM: A (or P) holds its upper triangle and the diagonal 128-blocks
                            // only; the k-blocks left of the diagonal block are read transposed
+  int diag_full;           // SYRK with 256 x 256 tiles: also store the lower-left 128 x 128
+                           // quarter of each diagonal 256-block (the pair GEMM reads the whole
+                           // diagonal 256-block K-major)
   int* err;                // device error word
   uint64_t wait_limit_ns;
 };
@@ -210,6 +215,7 @@ __device__ __forceinline__ int find_slot64(const int64_t* prefix, int n, int64_t
 }  // namespace dmuon
 #include "ns_stage.cuh"   // the Newton-Schulz stage kernel (depends on the types above)
 #include "syrk256.cuh"    // the SYRK stage (256 x 256 tiles)
+#include "gemm_pair.cuh"  // the GEMM stage on CTA pairs (256 x 256 tiles)
 namespace dmuon {
 
 // ======================================================================

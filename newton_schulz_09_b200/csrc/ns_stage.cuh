@@ -30,9 +30,10 @@ struct TileInfo {
   int half;   // SYRK: 128 x 128 tile over columns tn * 256 + 128 ..
 };
 
-// Tile t of a launch (128 x 256 tiles).
-template <int kMode, int BK>
-__device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
+// Tile t of a launch (128 x 256 tiles).  kPair: the GEMM's tiles are
+// 256 x 256 pairs, and CTA `rank` of the pair takes rows 128 rank .. of it.
+template <int kMode, int BK, bool kPair = false>
+__device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t, int rank = 0) {
   TileInfo ti;
   const int slot = find_slot(p.tile_prefix, p.nmat, t);
   ti.mi = __ldg(p.order + slot);
@@ -43,6 +44,11 @@ __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
     syrk_tile_coords(local, ti.tm, ti.tn);
     ti.nkb = ((kMode == kSyrk ? md.n : md.m) + BK - 1) / BK;
     ti.half = (ti.tm == 2 * ti.tn + 1) ? 1 : 0;
+  } else if (kPair) {
+    const int nI = (md.m + 2 * kBM - 1) / (2 * kBM);
+    ti.tn = local / nI;
+    ti.tm = 2 * (local - ti.tn * nI) + rank;
+    ti.nkb = (md.m + BK - 1) / BK;
   } else {
     const int nI = (md.m + kBM - 1) / kBM;
     ti.tn = local / nI;
@@ -58,10 +64,18 @@ __device__ __forceinline__ TileInfo decode_tile(const NsParams& p, int t) {
 // The accumulator buffer is released by `release(b)` once fully read.
 // Returns false when a bounded wait gave up.
 // ======================================================================
-template <int kMode, typename E, typename Release>
+// The epilogue's waits: sleeping in try_wait on one CTA, polling in the pair
+// kernel (whose accumulators arrive by a commit from the other SM).
+template <bool kPair>
+__device__ __forceinline__ bool epi_wait(uint64_t* bar, uint32_t parity, const NsParams& p) {
+  return kPair ? mbar_wait_spin(bar, parity, p.err, p.wait_limit_ns)
+               : mbar_wait(bar, parity, p.err, p.wait_limit_ns);
+}
+
+template <int kMode, typename E, bool kPair = false, typename Release>
 __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_base, uint8_t* epi,
                                              uint64_t* tfull, uint64_t* xfull, int warp, int lane,
-                                             int t0, int tstride, Release release) {
+                                             int t0, int tstride, Release release, int rank = 0) {
   constexpr int EB = static_cast<int>(sizeof(E));
   constexpr int BK = 128 / EB;
   const int q4 = warp & 3;                 // TMEM lane quarter of this warp
@@ -85,7 +99,7 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
     };
     auto load_next = [&]() {
       if (ld_t >= p.ntiles) return;
-      const TileInfo ti = decode_tile<kMode, BK>(p, ld_t);
+      const TileInfo ti = decode_tile<kMode, BK, kPair>(p, ld_t, rank);
       if (ti.mi != fenced) {
         tensormap_acquire_gpu(&p.maps[ti.mi].xk[p.cur]);
         tensormap_acquire_gpu(&p.maps[ti.mi].xk[p.cur ^ 1]);
@@ -104,19 +118,19 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
     uint32_t g = 0;
     int lt = 0;
     for (int t = t0; t < p.ntiles && ok; t += tstride, ++lt) {
-      const TileInfo ti = decode_tile<kMode, BK>(p, t);
+      const TileInfo ti = decode_tile<kMode, BK, kPair>(p, t, rank);
       const MatDesc& md = p.mats[ti.mi];
       const int b = lt & 1;
       const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
       const float cs = p.first ? *md.scale : 1.0f;
       const int nq = quarters_of(ti);
-      bool w = mbar_wait(&tfull[b], tph, p.err, p.wait_limit_ns);
+      bool w = epi_wait<kPair>(&tfull[b], tph, p);
       if (!named_bar_and(1, 128, w)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(b * kBN);
       for (int qq = 0; qq < nq; ++qq, ++g) {
         const int slot = static_cast<int>(g & 1u);
-        w = mbar_wait(&xfull[slot], (g >> 1) & 1u, p.err, p.wait_limit_ns);
+        w = epi_wait<kPair>(&xfull[slot], (g >> 1) & 1u, p);
         if (!named_bar_and(1, 128, w)) { ok = false; break; }
         uint32_t v0[32], v1[32];
         tmem_ld32(taddr + qq * 64, v0);
@@ -164,12 +178,12 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
 
   int lt = 0;
   for (int t = t0; t < p.ntiles && ok; t += tstride, ++lt) {
-    const TileInfo ti = decode_tile<kMode, BK>(p, t);
+    const TileInfo ti = decode_tile<kMode, BK, kPair>(p, t, rank);
     const MatDesc& md = p.mats[ti.mi];
     const int b = lt & 1;
     const uint32_t tph = (static_cast<uint32_t>(lt) >> 1) & 1u;
     const float s = *md.scale;
-    bool w = mbar_wait(&tfull[b], tph, p.err, p.wait_limit_ns);
+    bool w = epi_wait<kPair>(&tfull[b], tph, p);
     if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
     tc_fence_after();
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) + static_cast<uint32_t>(b * kBN);

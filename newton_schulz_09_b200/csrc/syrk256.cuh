@@ -10,8 +10,8 @@
 namespace dmuon {
 // ======================================================================
 // SYRK with 256 x 256 tiles per CTA.  A is stored as its upper triangle and
-// diagonal 128-blocks, or in full (mirrored) when the quintic SQUARE stage
-// reads it.  Each k-block brings 256 rows of X for the A operand
+// diagonal 128-blocks (with diag_full: diagonal 256-blocks, for the pair
+// GEMM), or in full (mirrored) when the quintic SQUARE stage reads it.  Each k-block brings 256 rows of X for the A operand
 // and 256 for the B operand (64 KB) and feeds two 128 x 256 UMMA halves that
 // share the B operand: a third fewer operand bytes per FLOP than 128 x 256
 // tiles.  The two fp32 accumulators take all 512 TMEM columns, so a tile's
@@ -217,6 +217,14 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                   if (C0 + j < m) arow[C0 + j] = from_f<E>(y[j]);
+              }
+              if (p.diag_full && ti.diag && h == 0 && c >= nch / 2) {
+                // the diagonal block's upper-right quarter, mirrored into its
+                // lower-left one (a warp's lanes are consecutive R: each j
+                // stores one contiguous run)
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (C0 + j < m) A[static_cast<int64_t>(C0 + j) * lda + R] = from_f<E>(y[j]);
               }
             } else {
               // the whole symmetric A (the quintic SQUARE stage reads all of

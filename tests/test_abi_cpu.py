@@ -332,3 +332,9 @@ def test_options_struct_sizes_and_quintic_workspace(lib):
     assert lib.dmuon_workspace_bytes_opts(S2, 2, ctypes.byref(o)) == cubic + 2 * 256 * 256 * 2
     o.ns_steps = 0
     assert lib.dmuon_workspace_bytes_opts(S2, 2, ctypes.byref(o)) == lib.dmuon_workspace_bytes(S2, 2, 0)
+
+
+def test_last_plan_query_without_plans(lib):
+    # host only: no plan exists in a process that made no device call
+    assert lib.dmuon_debug_last_plan(None, 0) == 0
+    assert dm.dmuon_debug_last_plan() == []
