@@ -602,11 +602,11 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     GroupArrays& A = ga[gi];
     A.pp.push_back(0);
     {
-      // The SYRK kernel, then the GEMM kernel: CTA pairs for bf16 cubic
-      // groups on 256 x 256 SYRK tiles whose matrices have m % 256 == 0 and
-      // n % 64 == 0 (whole pair tiles, 3-D X operand loads).
+      // The SYRK kernel, then the GEMM kernel: CTA pairs for bf16 groups on
+      // 256 x 256 SYRK tiles whose matrices have m % 256 == 0 and n % 64 == 0
+      // (whole pair tiles, 3-D X operand loads).
       int64_t t128 = 0, t256 = 0;
-      bool pair_ok = dt == DMUON_BF16 && !quintic && g_dev[dev].pair_clusters > 0;
+      bool pair_ok = dt == DMUON_BF16 && g_dev[dev].pair_clusters > 0;
       for (int k = 0; k < gp.nmat; ++k) {
         const MatLayout& ml = L.mats[g.idx[k]];
         t128 += syrk_tiles_of(ml.m);
@@ -1009,6 +1009,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
       sq.cb = o.cb;
       sq.cc = o.cc;
       sq.mirror = 0;
+      sq.diag_full = g.gemm_pair ? 1 : 0;   // the pair GEMM reads P's whole diagonal 256-blocks
       sq.order = g.gemm_order;
       sq.tile_prefix = g.square_prefix;
       sq.ntiles = g.square_tiles;

@@ -109,9 +109,9 @@ struct NsParams {
   int mirror;              // SYRK / SQUARE: also write the lower triangle (A^T of the upper)
   int a_upper;             // GEMM: A (or P) holds its upper triangle and the diagonal 128-blocks
                            // only; the k-blocks left of the diagonal block are read transposed
-  int diag_full;           // SYRK with 256 x 256 tiles: also store the lower-left 128 x 128
-                           // quarter of each diagonal 256-block (the pair GEMM reads the whole
-                           // diagonal 256-block K-major)
+  int diag_full;           // SYRK with 256 x 256 tiles, SQUARE: also store the lower-left
+                           // 128 x 128 quarter of each diagonal 256-block (the pair GEMM reads
+                           // the whole diagonal 256-block K-major)
   int* err;                // device error word
   uint64_t wait_limit_ns;
 };

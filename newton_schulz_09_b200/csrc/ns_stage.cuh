@@ -235,6 +235,13 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
               for (int j = 0; j < 32; ++j)
                 if (C0 + j < m) arow[C0 + j] = from_f<E>(y[j]);
             }
+            if (p.diag_full && !ti.half && ti.tm == 2 * ti.tn && C0 >= col0 + kBN / 2) {
+              // the diagonal 256-block's upper-right quarter, mirrored into its
+              // lower-left one (lanes are consecutive R: contiguous runs)
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (C0 + j < m) A[static_cast<int64_t>(C0 + j) * lda + R] = from_f<E>(y[j]);
+            }
             continue;
           }
           if (C0 >= R && C0 + 32 <= m) {

@@ -5,8 +5,8 @@ plan chose it, then compares the update with the oracle's Muon step on the
 same inputs.  Cases: one square matrix (first, middle and last GEMM steps),
 a batch with transposed (tall) parameters, column counts that end inside a
 pair tile's second half (n % 256 == 64 and 192), Nesterov off with weight
-decay on real weights, and one Newton-Schulz step (the first GEMM is the
-last)."""
+decay on real weights, one Newton-Schulz step (the first GEMM is the
+last), and the quintic coefficients."""
 import numpy as np
 import pytest
 import torch
@@ -25,22 +25,27 @@ def _rand(shape, dtype, seed, std=1.0):
     return (torch.randn(shape, generator=g, device=DEV) * std).to(dtype)
 
 
-def _run(dm, shapes, *, seed, ns_steps, zero_w=True, nesterov=True, wd=0.0, lr=0.05):
+def _run(dm, shapes, *, seed, ns_steps, zero_w=True, nesterov=True, wd=0.0, lr=0.05, coeffs=None):
     params = [torch.zeros(s, dtype=torch.bfloat16, device=DEV) if zero_w
               else _rand(s, torch.bfloat16, seed + 100 + i, 0.02) for i, s in enumerate(shapes)]
     w0 = [host(p) for p in params]
     grads = [_rand(s, torch.bfloat16, seed + i, 1e-3) for i, s in enumerate(shapes)]
     bufs = [_rand(s, torch.float32, seed + 50 + i, 1e-3) for i, s in enumerate(shapes)]
     b0 = [host(b) for b in bufs]
-    dm.dmuon_muon_step_batched(params, grads, bufs, lr=lr, momentum=0.95, nesterov=nesterov,
-                               weight_decay=wd, ns_steps=ns_steps)
+    if coeffs is None:
+        dm.dmuon_muon_step_batched(params, grads, bufs, lr=lr, momentum=0.95, nesterov=nesterov,
+                                   weight_decay=wd, ns_steps=ns_steps)
+    else:
+        dm.dmuon_muon_step_batched_opts(params, grads, bufs, lr=lr, momentum=0.95, nesterov=nesterov,
+                                        weight_decay=wd, ns_steps=ns_steps, ns_coefficients=coeffs)
     torch.cuda.synchronize()
     assert dm.dmuon_device_status() == 0
     plan = dm.dmuon_debug_last_plan()
     assert plan and all(g["gemm_pair"] and g["syrk256"] for g in plan), plan
     for i, s in enumerate(shapes):
         buf_ref, X_ref, W_ref = oracle.muon_step(w0[i], host(grads[i]), b0[i], lr=lr, momentum=0.95,
-                                                 nesterov=nesterov, weight_decay=wd, ns_steps=ns_steps)
+                                                 nesterov=nesterov, weight_decay=wd, ns_steps=ns_steps,
+                                                 ns_coeffs=coeffs or (1.5, -0.5))
         assert np.array_equal(host(bufs[i]).view(np.uint32), buf_ref.view(np.uint32))
         if zero_w and wd == 0.0:
             check_rel(host(params[i]), W_ref, TOL_BF16, f"pair GEMM {s} k={ns_steps}")
@@ -76,3 +81,10 @@ def test_weight_decay_without_nesterov(cuda_lib):
 def test_one_step(cuda_lib):
     shapes = [(768, 3072)] * 14
     _run(cuda_lib, shapes, seed=340, ns_steps=1)
+
+
+def test_quintic_coefficients(cuda_lib):
+    # P = b A + c A A from the SQUARE stage, whose diagonal 256-blocks are
+    # stored whole for the pair GEMM
+    shapes = [(1024, 4096)] * 4 + [(4096, 1024)] * 2 + [(1024, 2048)] * 2
+    _run(cuda_lib, shapes, seed=350, ns_steps=3, coeffs=(3.4445, -4.7750, 2.0315))
