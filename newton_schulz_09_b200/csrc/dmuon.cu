@@ -603,15 +603,15 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
     A.pp.push_back(0);
     {
       // The SYRK kernel, then the GEMM kernel: CTA pairs for bf16 groups on
-      // 256 x 256 SYRK tiles whose matrices have m % 256 == 0 and n % 64 == 0
-      // (whole pair tiles, 3-D X operand loads).
+      // 256 x 256 SYRK tiles whose matrices have n % 64 == 0 (3-D X operand
+      // loads).  Any m: rows past m load as zeros and are not stored.
       int64_t t128 = 0, t256 = 0;
       bool pair_ok = dt == DMUON_BF16 && g_dev[dev].pair_clusters > 0;
       for (int k = 0; k < gp.nmat; ++k) {
         const MatLayout& ml = L.mats[g.idx[k]];
         t128 += syrk_tiles_of(ml.m);
         t256 += syrk256_tiles_of(ml.m);
-        pair_ok = pair_ok && ml.m % (2 * kBM) == 0 && ml.n % 64 == 0;
+        pair_ok = pair_ok && ml.n % 64 == 0;
       }
       gp.syrk256 = use_syrk256(t128, t256, g_dev[dev].sms);
       gp.gemm_pair = gp.syrk256 && pair_ok;

@@ -158,8 +158,11 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (leader) {
-          tma_store_2d(&p.maps[ti.mi].xk[p.cur ^ 1], epi + slot * kEpiSlotBytes,
-                       ti.tn * kBN + 64 * qq, ti.tm * kBM);
+          // (the odd CTA of a pair tile that ends inside the matrix's last
+          // 128 rows holds no rows of it: nothing to store)
+          if (ti.tm * kBM < md.m)
+            tma_store_2d(&p.maps[ti.mi].xk[p.cur ^ 1], epi + slot * kEpiSlotBytes,
+                         ti.tn * kBN + 64 * qq, ti.tm * kBM);
           bulk_commit_group();
           bulk_wait_group_read0();               // slot read out: it may be refilled
           slot_busy[slot] = false;

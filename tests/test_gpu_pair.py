@@ -88,3 +88,11 @@ def test_quintic_coefficients(cuda_lib):
     # stored whole for the pair GEMM
     shapes = [(1024, 4096)] * 4 + [(4096, 1024)] * 2 + [(1024, 2048)] * 2
     _run(cuda_lib, shapes, seed=350, ns_steps=3, coeffs=(3.4445, -4.7750, 2.0315))
+
+
+@pytest.mark.parametrize("shapes", [
+    [(384, 1536)] * 36 + [(1536, 384)] * 4,      # m % 256 == 128: the last pair's odd CTA holds no rows
+    [(1000, 3008)] * 8 + [(3008, 1000)] * 2,     # ragged m: the last pair's odd CTA holds 104 rows
+], ids=["m%256=128", "m=1000"])
+def test_rows_ending_inside_a_pair_tile(cuda_lib, shapes):
+    _run(cuda_lib, shapes, seed=360, ns_steps=2)
