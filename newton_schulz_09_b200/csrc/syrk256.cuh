@@ -23,7 +23,9 @@ namespace dmuon {
 // ======================================================================
 constexpr int kS2Stages = 3;
 constexpr int kS2OpBytes = kBN * 128;              // 256 rows x 128 bytes of K
-constexpr int kS2SmemBytes = kS2Stages * 2 * kS2OpBytes + 1024 /*align*/ + 256;
+// + two 16 KB slots (128 rows x 64 bf16 columns) through which the epilogue
+// stages its stores for TMA
+constexpr int kS2SmemBytes = kS2Stages * 2 * kS2OpBytes + kEpiSlots * kEpiSlotBytes + 1024 /*align*/ + 256;
 static_assert(kS2SmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
 
 // Upper-triangle 256 x 256 tiles of one matrix, column-band major: band J
@@ -66,7 +68,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   // stage s: A operand rows at s * 64 KB, B operand rows 32 KB after them
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kS2Stages * 2 * kS2OpBytes);
+  uint8_t* epi = smem + kS2Stages * 2 * kS2OpBytes;    // bf16 store slots
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiSlots * kEpiSlotBytes);
   uint64_t* empty = full + kS2Stages;
   uint64_t* tfull = empty + kS2Stages;
   uint64_t* tempty = tfull + 1;
@@ -179,6 +182,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
     // ------------------------------------------------ epilogue (4 warps)
     const int q4 = warp & 3;
     const int row_in_tile = q4 * 32 + lane;
+    int fenced_a = -1;        // matrix whose A map the store leader has acquired
+    uint32_t gq = 0;          // store quarters so far (slot ring position)
     int lt = 0;
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
       const Tile256 ti = decode_tile256<BK>(p, t);
@@ -191,6 +196,76 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
       E* A = reinterpret_cast<E*>(md.A);
       const int64_t lda = md.lda;
       const int m = md.m;
+      if (EB == 2 && !p.mirror) {
+        // Upper triangle and diagonal 128-blocks through shared memory: each
+        // 128 x 64 quarter goes TMEM -> registers -> a 128B-swizzled slot ->
+        // one TMA store into A (clipped at m).  Two slots alternate; a slot
+        // is rewritten only after the store two quarters back has read it.
+        // The accumulators are released after the tile's last TMEM load.
+        const bool leader = (warp == 2 && lane == 0);
+        if (leader && ti.mi != fenced_a) {
+          tensormap_acquire_gpu(&p.maps[ti.mi].a);
+          fenced_a = ti.mi;
+        }
+        const int nq0 = kBN / 64;
+        const int nq = nq0 + (ti.diag ? kBN / 128 : kBN / 64);
+#pragma unroll 1
+        for (int qi = 0; qi < nq; ++qi, ++gq) {
+          const int h = qi < nq0 ? 0 : 1;
+          const int q = qi - h * nq0;
+          const bool quarter = ti.diag && h == 1;
+          const int R0 = ti.I * kBN + h * kBM;
+          const int C0 = ti.J * kBN + (quarter ? kBN / 2 : 0) + q * 64;
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) +
+                                 static_cast<uint32_t>(h * kBN + q * 64);
+          uint32_t v0[32], v1[32];
+          tmem_ld32(taddr, v0);
+          tmem_ld32(taddr + 32, v1);
+          tmem_ld_wait();
+          if (qi == nq - 1) {
+            tc_fence_before();
+            mbar_arrive(tempty);            // every TMEM load of the tile has landed
+          }
+          const int slot = static_cast<int>(gq & 1u);
+          uint8_t* rowp = epi + slot * kEpiSlotBytes + row_in_tile * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int col = c * 8 + 2 * j;
+              const float a0 = alpha * __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
+              const float a1 = alpha * __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
+              __nv_bfloat162 yv = __floats2bfloat162_rn(a0, a1);
+              wv[j] = *reinterpret_cast<uint32_t*>(&yv);
+            }
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (row_in_tile & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+          if (p.diag_full && ti.diag && h == 0 && q >= nq0 / 2) {
+            // the diagonal block's upper-right quarter, mirrored into its
+            // lower-left one (a warp's lanes are consecutive R: each column
+            // is one contiguous run)
+            const int R = R0 + row_in_tile;
+            if (R < m) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j) {
+                const float a = alpha * __uint_as_float(j < 32 ? v0[j] : v1[j - 32]);
+                if (C0 + j < m) A[static_cast<int64_t>(C0 + j) * lda + R] = __float2bfloat16_rn(a);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (leader) {
+            if (R0 < m && C0 < m)
+              tma_store_2d(&p.maps[ti.mi].a, epi + slot * kEpiSlotBytes, C0, R0);
+            bulk_commit_group();
+            bulk_wait_group_read1();     // the other slot's store has read it
+          }
+          named_bar_sync(1, 128);        // ... before anyone writes that slot
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         const bool quarter = ti.diag && h == 1;
@@ -248,6 +323,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(tempty);
     }
+    if (warp == 2 && lane == 0) bulk_wait_group0();   // the TMA stores have completed
   }
 
   __syncthreads();
