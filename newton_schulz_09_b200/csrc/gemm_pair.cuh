@@ -1,6 +1,7 @@
 // GEMM stage of the batched Muon update on CTA pairs (sm_100a): X' = c (a X +
-// A X) over 256 x 256 output tiles, each computed by a two-CTA cluster with
-// pair UMMAs (tcgen05 cta_group::2), for every matrix of a bf16 group.
+// b A X) (quintic: c (a X + P X)) over 256 x 256 output tiles, each computed
+// by a two-CTA cluster with pair UMMAs (tcgen05 cta_group::2), for every
+// matrix of a bf16 group.
 //
 // Source: DMuon blog post "DMuon：让矩阵正交化优化器达到接近 AdamW 的分布式训练开销",
 // section "Muon 核心：Newton-Schulz 迭代" (the cubic step X <- a X + b A X).
@@ -26,9 +27,10 @@ namespace dmuon {
 // buffer on the even CTA's `tempty`.  Producer, UMMA and epilogue waits poll
 // (their signals come from the other SM).
 //
-// A is read as the SYRK stored it: upper triangle plus full diagonal
-// 256-blocks.  The k-blocks left of the pair's diagonal block come
-// transposed (MN-major) from the upper triangle, as in ns_stage_kernel.
+// A (or P) is read as the SYRK (or the quintic SQUARE stage) stored it:
+// upper triangle plus full diagonal 256-blocks.  The k-blocks left of the
+// pair's diagonal block come transposed (MN-major) from the upper triangle,
+// as in ns_stage_kernel.
 // ======================================================================
 constexpr int kG2Stages = 6;
 constexpr int kG2ABytes = kBM * 128;            // 128 rows (or 128 M columns) x 128 bytes of K
