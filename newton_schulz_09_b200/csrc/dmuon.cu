@@ -255,6 +255,7 @@ Layout make_layout(const std::vector<MatIn>& in, int steps, bool quintic = false
 struct GroupPlan {
   int dtype;
   bool ranks = false;     // some matrix averages several ranks' gradients
+  bool g_bf16 = true;     // every gradient of the group is bf16
   int nmat;
   int first;              // first MatDesc index of the group
   int64_t ptiles;
@@ -422,6 +423,12 @@ int device_setup(int dev) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kProSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prologue smem)");
   }
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&prologue_tma_kernel<true>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, PtCfg<true>::kSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pipelined prologue smem)");
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&prologue_tma_kernel<false>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, PtCfg<false>::kSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pipelined prologue smem)");
   if (!encode_fn()) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cudaMemPoolProps props;
   std::memset(&props, 0, sizeof(props));
@@ -641,6 +648,7 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       d.vec4 = vec4_of(x);
       d.world = x.gr.size() > 1 ? static_cast<int>(x.gr.size()) : 1;
       if (d.world > 1) gp.ranks = true;
+      if (!d.g_bf16) gp.g_bf16 = false;
       d.Gr = nullptr;   // set once the plan's device memory exists
       d.ptiles_c = static_cast<int>(ml.ptiles_c);
       A.pp.push_back(A.pp.back() + ml.ptiles);
@@ -961,12 +969,24 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
                   cudaStream_t st) {
   const float lr = o.lr, wd = o.wd;
   const int steps = o.steps;
-  const ElemParams ep = elem_params<E>(P, g, o);
+  ElemParams ep = elem_params<E>(P, g, o);
+  ep.err = d.err;
+  ep.wait_limit_ns = kWaitLimitNs;
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-    if (g.ranks) prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
-    else prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    if (g.ranks) {
+      prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    } else if (sizeof(E) == 2) {
+      // bf16 iterates: the pipelined prologue, two blocks per SM when every
+      // gradient is bf16 (48 KB stages), else one (64 KB stages).
+      const int per_sm = g.g_bf16 ? PtCfg<true>::kBlocksPerSm : PtCfg<false>::kBlocksPerSm;
+      const int tgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * per_sm));
+      if (g.g_bf16) prologue_tma_kernel<true><<<tgrid, kPtThreads, PtCfg<true>::kSmem, st>>>(ep);
+      else prologue_tma_kernel<false><<<tgrid, kPtThreads, PtCfg<false>::kSmem, st>>>(ep);
+    } else {
+      prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+    }
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);

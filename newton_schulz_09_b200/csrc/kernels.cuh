@@ -127,6 +127,8 @@ struct ElemParams {
   float lr, wd;                 // apply_kernel only
   const float* clip;            // gradient scale (global-norm clipping) or nullptr
   double* gpartials;            // grad_norm_kernel: one partial sum of g^2 per item
+  int* err;                     // prologue_tma_kernel: device error word and bound of its waits
+  uint64_t wait_limit_ns;
 };
 
 // ------------------------------------------------------------------ helpers
@@ -390,17 +392,18 @@ __device__ __forceinline__ void store8_x(E* dst, bool vec, int valid, const floa
   }
 }
 
-// Momentum / Nesterov on 8 values; returns M, updates b in place.  With
+// Momentum / Nesterov on N values; returns M, updates b in place.  With
 // gradient clipping the gradient enters as fl32(g * c).
-__device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, float (&g)[8],
-                                          float (&b)[8], float (&M)[8]) {
+template <int N>
+__device__ __forceinline__ void momentum_n(const ElemParams& p, bool has_buf, float (&g)[N],
+                                           float (&b)[N], float (&M)[N]) {
   if (p.clip != nullptr) {
     const float c = *p.clip;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(g[e], c);
+    for (int e = 0; e < N; ++e) g[e] = __fmul_rn(g[e], c);
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
+  for (int e = 0; e < N; ++e) {
     if (has_buf) {
       // buf <- fl(fl(mu * buf) + g): two roundings, never fused.
       b[e] = __fadd_rn(__fmul_rn(p.mu, b[e]), g[e]);
@@ -409,6 +412,10 @@ __device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, flo
       M[e] = g[e];
     }
   }
+}
+__device__ __forceinline__ void momentum8(const ElemParams& p, bool has_buf, float (&g)[8],
+                                          float (&b)[8], float (&M)[8]) {
+  momentum_n<8>(p, has_buf, g, b, M);
 }
 
 template <typename E, bool kRanks>
@@ -590,6 +597,286 @@ __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_consta
       p.partials[t] = acc;
     }
     __syncthreads();
+  }
+}
+
+// ======================================================================
+// Pipelined prologue for bf16 iterates and one gradient buffer per matrix.
+// The same work items as prologue_kernel.  A producer warp streams each
+// item's gradient and momentum into a ring of shared-memory stages with bulk
+// asynchronous copies (two for a flat item, two per parameter row of a
+// transposed item) while eight consumer warps work on an earlier stage, so
+// the loads stay in flight across items instead of being issued and awaited
+// one item at a time.  A transposed item is mapped so that each consumer
+// thread owns 8 parameter rows x 4 columns: its four X row segments (8
+// consecutive parameter rows of one column, 16 bytes) are stored straight to
+// global memory, without a shared-memory transpose.  Items that are not
+// whole and 16-byte aligned (a matrix's ragged edge) are read from global
+// memory directly by the consumers.
+// ======================================================================
+constexpr int kPtConsumers = 256;                 // 8 consumer warps
+constexpr int kPtThreads = kPtConsumers + 32;     // + 1 producer warp
+template <bool kGBf16> struct PtCfg {
+  static constexpr int kGBytes = kFlatChunk * (kGBf16 ? 2 : 4);   // an item's gradient
+  static constexpr int kBBytes = kFlatChunk * 4;                   // an item's momentum
+  static constexpr int kStageBytes = kGBytes + kBBytes;
+  static constexpr int kStages = kGBf16 ? 2 : 3;                   // 2 blocks / SM for bf16 gradients
+  static constexpr int kBlocksPerSm = kGBf16 ? 2 : 1;
+  static constexpr int kSmem = kStages * kStageBytes;
+};
+static_assert(kTR * kTC == kFlatChunk, "a transposed item fills one stage like a flat item");
+static_assert(PtCfg<false>::kSmem <= 232448 - 1024, "prologue stages exceed shared memory");
+static_assert(2 * (PtCfg<true>::kSmem + 1024 + 256) <= 233472, "two bf16 prologue blocks must fit an SM");
+
+// Whether an item's inputs come through the staged ring: whole items of
+// matrices whose rows start on 16-byte boundaries.
+__device__ __forceinline__ bool pt_whole(const MatDesc& md, int64_t item) {
+  if (!md.vec4) return false;
+  if (!md.T) return (item + 1) * kFlatChunk <= md.rows * md.cols;
+  const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+  return (md.cols % 8 == 0) && (tr + 1) * kTR <= md.rows && (tc + 1) * kTC <= md.cols;
+}
+
+// Flat item: thread `ct` handles the same 4 x 8 elements as prologue_flat,
+// with the same arithmetic and summation order.
+__device__ __forceinline__ float pt_flat(const ElemParams& p, const MatDesc& md, int64_t item, bool whole,
+                                         const uint8_t* sg, const float* sb, int ct) {
+  const int64_t numel = md.rows * md.cols;
+  const int64_t e_begin = item * kFlatChunk;
+  const bool has_buf = md.buf != nullptr;
+  const bool flat_x = (md.ldx == md.cols);
+  const int gb = md.g_bf16 ? 2 : 4;
+  __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(md.X[0]);
+  float ss = 0.0f;
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    const int le = (j * kPtConsumers + ct) * 8;
+    const int64_t e = e_begin + le;
+    if (e >= numel) break;
+    const int valid = static_cast<int>(numel - e < 8 ? numel - e : 8);
+    const bool vec = md.vec4 && valid == 8;
+    float g[8], b[8], M[8];
+    if (whole) {
+      unstage8<false>(md, has_buf, sg + le * gb, sb + le, g, b);
+    } else {
+      load8_in<false>(md, e, vec, valid, g);
+      if (has_buf) load8_f32(md.buf + e, vec, valid, b);
+    }
+    momentum8(p, has_buf, g, b, M);
+    if (has_buf) store8_f32(md.buf + e, vec, valid, b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= valid) M[k] = 0.0f;
+      ss = fmaf(M[k], M[k], ss);
+    }
+    if (flat_x) {
+      store8_x<__nv_bfloat16>(X + e, valid == 8, valid, M);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < valid) {
+          const int64_t r = (e + k) / md.cols, c = (e + k) - r * md.cols;
+          X[r * md.ldx + c] = __float2bfloat16_rn(M[k]);
+        }
+      }
+    }
+  }
+  return ss;
+}
+
+// Transposed item (64 parameter rows x 128 columns): thread `ct` owns rows
+// rb*8 .. rb*8+7 and columns cg*4 .. cg*4+3 of the item.  Within a warp the
+// 8 column groups x 4 row blocks read 128 contiguous bytes of momentum per
+// staged row (no bank conflicts) and write 64-byte runs of 4 X rows.
+__device__ __forceinline__ float pt_transposed(const ElemParams& p, const MatDesc& md, int64_t item, bool whole,
+                                               const uint8_t* sg, const float* sb, int ct) {
+  const int w = ct >> 5, l = ct & 31;
+  const int rb = (l >> 3) + 4 * (w & 1);     // 0..7
+  const int cg = (l & 7) + 8 * (w >> 1);     // 0..31
+  const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+  const int64_t r0 = tr * kTR, c0 = tc * kTC;
+  const int64_t rows = md.rows, cols = md.cols;
+  const bool has_buf = md.buf != nullptr;
+  const int lc = cg * 4;
+  const int64_t c = c0 + lc;
+  float Mv[8][4];
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int lr = rb * 8 + j;
+    const int64_t r = r0 + lr;
+    float g[4], b[4];
+    int valid = 4;
+    if (whole) {
+      if (md.g_bf16) {
+        const uint2 u = *reinterpret_cast<const uint2*>(sg + (lr * kTC + lc) * 2);
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        g[0] = f0.x; g[1] = f0.y; g[2] = f1.x; g[3] = f1.y;
+      } else {
+        const float4 v = *reinterpret_cast<const float4*>(sg + (lr * kTC + lc) * 4);
+        g[0] = v.x; g[1] = v.y; g[2] = v.z; g[3] = v.w;
+      }
+      if (has_buf) {
+        const float4 v = *reinterpret_cast<const float4*>(sb + lr * kTC + lc);
+        b[0] = v.x; b[1] = v.y; b[2] = v.z; b[3] = v.w;
+      }
+    } else {
+      valid = (r < rows && c < cols) ? static_cast<int>(cols - c < 4 ? cols - c : 4) : 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const bool in = k < valid;
+        const int64_t idx = r * cols + c + k;
+        g[k] = !in ? 0.0f
+               : md.g_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(md.G)[idx])
+                           : reinterpret_cast<const float*>(md.G)[idx];
+        b[k] = (in && has_buf) ? md.buf[idx] : 0.0f;
+      }
+    }
+    momentum_n<4>(p, has_buf, g, b, Mv[j]);
+    if (has_buf) {
+      float* dst = md.buf + r * cols + c;
+      if (whole) {
+        *reinterpret_cast<float4*>(dst) = make_float4(b[0], b[1], b[2], b[3]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k < valid) dst[k] = b[k];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k >= valid) Mv[j][k] = 0.0f;
+      ss = fmaf(Mv[j][k], Mv[j][k], ss);
+    }
+  }
+  // X row = parameter column, X columns = parameter rows.
+  __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(md.X[0]);
+  const int64_t xc = r0 + rb * 8;
+  const bool vec_x = whole && (md.ldx % 8 == 0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t xr = c + q;
+    if (vec_x) {
+      uint32_t u[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(Mv[2 * h][q], Mv[2 * h + 1][q]);
+        u[h] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      *reinterpret_cast<uint4*>(X + xr * md.ldx + xc) = make_uint4(u[0], u[1], u[2], u[3]);
+    } else if (xr < cols && xc < rows) {
+      const int valid = (rows - xc >= 8) ? 8 : static_cast<int>(rows - xc);
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < valid) X[xr * md.ldx + xc + h] = __float2bfloat16_rn(Mv[h][q]);
+    }
+  }
+  return ss;
+}
+
+template <bool kGBf16>
+__global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_constant__ ElemParams p) {
+  using Cfg = PtCfg<kGBf16>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ __align__(128) uint8_t pt_smem[];   // Cfg::kSmem
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ float red[2][kPtConsumers / 32];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kPtConsumers / 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  int mi = blockIdx.x < p.ntiles ? find_slot64(p.ptile_prefix, p.nmat, blockIdx.x) : 0;
+  if (warp == kPtConsumers / 32) {
+    // ---------------------------------------------------------- producer
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+      while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
+      const MatDesc& md = p.mats[mi];
+      const int64_t item = t - __ldg(p.ptile_prefix + mi);
+      const int s = static_cast<int>(it % S);
+      if (it >= S && !mbar_wait(&empty_bar[s], ((it / S) & 1u) ^ 1u, p.err, p.wait_limit_ns)) {
+        ok = false;
+        break;
+      }
+      uint8_t* sg = pt_smem + s * Cfg::kStageBytes;
+      float* sb = reinterpret_cast<float*>(sg + Cfg::kGBytes);
+      const bool has_buf = md.buf != nullptr;
+      const uint32_t gb = md.g_bf16 ? 2u : 4u;
+      if (!pt_whole(md, item)) {
+        if (lane == 0) mbar_arrive(&full_bar[s]);
+        continue;
+      }
+      if (!md.T) {
+        if (lane == 0) {
+          const int64_t e = item * kFlatChunk;
+          mbar_arrive_expect_tx(&full_bar[s], kFlatChunk * (gb + (has_buf ? 4u : 0u)));
+          bulk_load(sg, static_cast<const uint8_t*>(md.G) + e * gb, kFlatChunk * gb, &full_bar[s]);
+          if (has_buf) bulk_load(sb, md.buf + e, kFlatChunk * 4, &full_bar[s]);
+        }
+      } else {
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], kFlatChunk * (gb + (has_buf ? 4u : 0u)));
+        __syncwarp();
+        const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+#pragma unroll
+        for (int h = 0; h < kTR / 32; ++h) {
+          const int lr = lane + 32 * h;
+          const int64_t idx = (tr * kTR + lr) * md.cols + tc * kTC;
+          bulk_load(sg + lr * kTC * gb, static_cast<const uint8_t*>(md.G) + idx * gb, kTC * gb, &full_bar[s]);
+          if (has_buf) bulk_load(sb + lr * kTC, md.buf + idx, kTC * 4, &full_bar[s]);
+        }
+      }
+    }
+    // Before leaving after a failed wait, let the copies already issued land
+    // (bounded): the phase of each stage's last use, if any.
+    if (!ok) {
+      for (int s = 0; s < S; ++s) {
+        if (it > static_cast<uint32_t>(s)) {
+          const uint32_t last = it - 1 - ((it - 1 - s) % S);   // last iteration that used stage s
+          mbar_wait(&full_bar[s], (last / S) & 1u, nullptr, p.wait_limit_ns);
+        }
+      }
+    }
+    return;
+  }
+  // ------------------------------------------------------------ consumers
+  uint32_t it = 0;
+  for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
+    while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
+    const MatDesc& md = p.mats[mi];
+    const int64_t item = t - __ldg(p.ptile_prefix + mi);
+    const int s = static_cast<int>(it % S);
+    // The consumers leave together, at the same item, if a wait gives up.
+    const bool ok = mbar_wait(&full_bar[s], (it / S) & 1u, p.err, p.wait_limit_ns);
+    if (!named_bar_and(2, kPtConsumers, ok)) break;
+    const uint8_t* sg = pt_smem + s * Cfg::kStageBytes;
+    const float* sb = reinterpret_cast<const float*>(sg + Cfg::kGBytes);
+    const bool whole = pt_whole(md, item);
+    float ss = md.T ? pt_transposed(p, md, item, whole, sg, sb, tid) : pt_flat(p, md, item, whole, sg, sb, tid);
+    // This warp has read its staged values: release the stage.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    // Fixed-order reduction of the item's sum of squares (red is double
+    // buffered, so one barrier per item suffices).
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) red[it & 1u][warp] = ss;
+    named_bar_sync(1, kPtConsumers);
+    if (tid == 0) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kPtConsumers / 32; ++w) acc += red[it & 1u][w];
+      p.partials[t] = acc;
+    }
   }
 }
 
