@@ -686,6 +686,22 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
           okm &= encode_2d(&mm.p, dt, d.P, ml.m, ml.m, ml.lda, BK, kBM);
           okm &= encode_2d(&mm.pmn, dt, d.P, ml.m, ml.m, ml.lda, BK, BK, mn_sw);
         }
+        // Transposed bf16 matrices with 16-byte aligned rows: the prologue
+        // loads each 64 x 128 item of G and buf with one 2-D tensor load.
+        // The maps hold the caller's addresses (a placeholder in the
+        // workspace while they are not 16-byte aligned); patch_kernel keeps
+        // them current.
+        d.tmaps = 0;
+        if (d.T && dt == DMUON_BF16 && d.world <= 1 && x.cols % 8 == 0) {
+          const bool ga = aligned(x.G, 16), ba = x.buf == nullptr || aligned(x.buf, 16);
+          void* gbase = ga ? const_cast<void*>(x.G) : static_cast<void*>(wsb);
+          void* bbase = (x.buf && ba) ? static_cast<void*>(x.buf) : static_cast<void*>(wsb);
+          bool okt = encode_2d(&mm.gt, x.gdt, gbase, x.cols, x.rows, x.cols, kTC, kTR,
+                               CU_TENSOR_MAP_SWIZZLE_NONE);
+          if (x.buf) okt = okt && encode_2d(&mm.bt, DMUON_F32, bbase, x.cols, x.rows, x.cols, kTC, kTR,
+                                            CU_TENSOR_MAP_SWIZZLE_NONE);
+          d.tmaps = okt ? 1 : 0;
+        }
         if (!okm) return fail(DMUON_ERR_CUDA, "cuTensorMapEncodeTiled failed for matrix %d", i);
       }
     }
@@ -851,6 +867,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
     if (!pp) {
       pp.reset(new PatchParams());
       pp->mats = const_cast<MatDesc*>(P.d_mats);
+      pp->maps = const_cast<MatMaps*>(P.d_maps);
       pp->n = 0;
     }
     PatchEntry& en = pp->e[pp->n++];
@@ -951,6 +968,9 @@ ElemParams elem_params(const Plan& P, const GroupPlan& g, const StepOpts& o) {
   ep.wd = o.wd;
   ep.clip = o.max_norm > 0.0f ? P.clip : nullptr;
   ep.gpartials = g.gpartials;
+  ep.err = nullptr;
+  ep.wait_limit_ns = 0;
+  ep.maps = P.d_maps + g.first;
   return ep;
 }
 

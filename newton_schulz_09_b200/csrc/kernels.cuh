@@ -76,6 +76,7 @@ struct MatDesc {
   int b3d;             // xmn maps are 3-D (bf16, n % 64 == 0): one load brings a whole B operand
   int world;           // > 1: the gradient is the mean of `world` buffers Gr[0..world)
   const void* const* Gr;  // device array of the ranks' gradient buffers (rank order), or nullptr
+  int tmaps;           // the gt / bt tensor maps bring a transposed prologue item's G and buf
 };
 
 struct alignas(64) MatMaps {
@@ -90,6 +91,8 @@ struct alignas(64) MatMaps {
   CUtensorMap pmn;     // reads A's (or P's) lower k-blocks transposed from the upper triangle
   CUtensorMap xmn2[2]; // with b3d: the 3-D view of xmn with a box of 2 blocks (128 columns),
                        // one CTA's half of the B operand of a pair GEMM tile
+  CUtensorMap gt;      // with tmaps: G (rows x cols) and buf, box kTC columns x kTR rows, no
+  CUtensorMap bt;      // swizzle; their addresses follow the caller's through patch_kernel
 };
 
 struct NsParams {
@@ -129,6 +132,7 @@ struct ElemParams {
   double* gpartials;            // grad_norm_kernel: one partial sum of g^2 per item
   int* err;                     // prologue_tma_kernel: device error word and bound of its waits
   uint64_t wait_limit_ns;
+  const MatMaps* maps;          // prologue_tma_kernel: the matrices' gt / bt maps
 };
 
 // ------------------------------------------------------------------ helpers
@@ -622,7 +626,7 @@ template <bool kGBf16> struct PtCfg {
   static constexpr int kStageBytes = kGBytes + kBBytes;
   static constexpr int kStages = kGBf16 ? 2 : 3;                   // 2 blocks / SM for bf16 gradients
   static constexpr int kBlocksPerSm = kGBf16 ? 2 : 1;
-  static constexpr int kSmem = kStages * kStageBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 128 /*align*/;
 };
 static_assert(kTR * kTC == kFlatChunk, "a transposed item fills one stage like a flat item");
 static_assert(PtCfg<false>::kSmem <= 232448 - 1024, "prologue stages exceed shared memory");
@@ -684,15 +688,18 @@ __device__ __forceinline__ float pt_flat(const ElemParams& p, const MatDesc& md,
   return ss;
 }
 
-// Transposed item (64 parameter rows x 128 columns): thread `ct` owns rows
+// Transposed item (kTR parameter rows x kTC columns): thread `ct` owns rows
 // rb*8 .. rb*8+7 and columns cg*4 .. cg*4+3 of the item.  Within a warp the
 // 8 column groups x 4 row blocks read 128 contiguous bytes of momentum per
-// staged row (no bank conflicts) and write 64-byte runs of 4 X rows.
+// staged row (no bank conflicts) and write 64-byte runs of 8 X rows.
+constexpr int kPtRB = kTR / 8, kPtCG = kTC / 4;   // row blocks and column groups of an item
+static_assert(kPtRB * kPtCG == kPtConsumers && kPtRB % 4 == 0 && kPtCG % 8 == 0,
+              "transposed item mapping: 4 row blocks x 8 column groups per warp");
 __device__ __forceinline__ float pt_transposed(const ElemParams& p, const MatDesc& md, int64_t item, bool whole,
                                                const uint8_t* sg, const float* sb, int ct) {
   const int w = ct >> 5, l = ct & 31;
-  const int rb = (l >> 3) + 4 * (w & 1);     // 0..7
-  const int cg = (l & 7) + 8 * (w >> 1);     // 0..31
+  const int rb = (l >> 3) + 4 * (w % (kPtRB / 4));
+  const int cg = (l & 7) + 8 * (w / (kPtRB / 4));
   const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
   const int64_t r0 = tr * kTR, c0 = tc * kTC;
   const int64_t rows = md.rows, cols = md.cols;
@@ -779,7 +786,9 @@ template <bool kGBf16>
 __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_constant__ ElemParams p) {
   using Cfg = PtCfg<kGBf16>;
   constexpr int S = Cfg::kStages;
-  extern __shared__ __align__(128) uint8_t pt_smem[];   // Cfg::kSmem
+  extern __shared__ __align__(128) uint8_t pt_raw[];    // Cfg::kSmem
+  uint8_t* pt_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pt_raw) + 127) &
+                                                ~static_cast<uintptr_t>(127));
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ float red[2][kPtConsumers / 32];
@@ -799,6 +808,7 @@ __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_c
     // ---------------------------------------------------------- producer
     uint32_t it = 0;
     bool ok = true;
+    int fenced = -1;                 // matrix whose tensor maps lane 0 has acquired
     for (int64_t t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++it) {
       while (t >= __ldg(p.ptile_prefix + mi + 1)) ++mi;
       const MatDesc& md = p.mats[mi];
@@ -823,7 +833,23 @@ __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_c
           bulk_load(sg, static_cast<const uint8_t*>(md.G) + e * gb, kFlatChunk * gb, &full_bar[s]);
           if (has_buf) bulk_load(sb, md.buf + e, kFlatChunk * 4, &full_bar[s]);
         }
+      } else if (md.tmaps) {
+        // One 2-D tensor load each for the item's gradient and momentum.
+        if (lane == 0) {
+          const MatMaps& mp = p.maps[mi];
+          if (mi != fenced) {
+            tensormap_acquire_gpu(&mp.gt);
+            if (has_buf) tensormap_acquire_gpu(&mp.bt);
+            fenced = mi;
+          }
+          const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
+          const int32_t x = static_cast<int32_t>(tc * kTC), y = static_cast<int32_t>(tr * kTR);
+          mbar_arrive_expect_tx(&full_bar[s], kFlatChunk * (gb + (has_buf ? 4u : 0u)));
+          tma_load_2d(sg, &mp.gt, &full_bar[s], x, y);
+          if (has_buf) tma_load_2d(sb, &mp.bt, &full_bar[s], x, y);
+        }
       } else {
+        // One bulk copy per parameter row of the item.
         if (lane == 0) mbar_arrive_expect_tx(&full_bar[s], kFlatChunk * (gb + (has_buf ? 4u : 0u)));
         __syncwarp();
         const int64_t tr = item / md.ptiles_c, tc = item - tr * md.ptiles_c;
@@ -1354,6 +1380,7 @@ struct PatchEntry {
 constexpr int kPatchMax = 480;        // entries per launch (about 15 KB of parameters)
 struct PatchParams {
   MatDesc* mats;
+  MatMaps* maps;
   int n;
   PatchEntry e[kPatchMax];
 };
@@ -1364,7 +1391,15 @@ __global__ void __launch_bounds__(256) patch_kernel(const __grid_constant__ Patc
     d.G = p.e[i].G;
     d.buf = p.e[i].buf;
     d.vec4 = p.e[i].vec4;
+    // The prologue's G / buf tensor maps take the new addresses (used only
+    // when the rows are 16-byte aligned, i.e. with vec4).
+    if (d.tmaps && p.e[i].vec4) {
+      MatMaps& mm = p.maps[p.e[i].index];
+      tensormap_replace_address(&mm.gt, p.e[i].G);
+      if (p.e[i].buf) tensormap_replace_address(&mm.bt, p.e[i].buf);
+    }
   }
+  tensormap_release_gpu();
 }
 
 // Test kernel: waits on a barrier that nothing arrives at; the bounded wait

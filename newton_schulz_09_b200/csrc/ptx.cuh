@@ -199,6 +199,15 @@ __device__ __forceinline__ void tensormap_acquire_gpu(const CUtensorMap* map) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
 }
 
+// Sets the global address of a tensor map held in global memory (the other
+// fields stay); readers acquire it as above.
+__device__ __forceinline__ void tensormap_replace_address(CUtensorMap* map, const void* addr) {
+  asm volatile("tensormap.replace.tile.global_address.global.b1024.b64 [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "l"(reinterpret_cast<uint64_t>(addr))
+               : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
