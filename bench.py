@@ -35,13 +35,12 @@ UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage: the ncu
-# capture of one Llama-8B layer's GEMM on CTA pairs (580.1 MB read + 414.6 MB written for
+# capture of one Llama-8B layer's GEMM on CTA pairs (574.3 MB read + 411.7 MB written for
 # 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so its traffic is
 # this ratio times the useful FLOPs of that launch.  Valid only for the stage kernels' source it
-# was measured on (ns_stage.cuh, gemm_pair.cuh and ptx.cuh; the capture's copy differed from
-# this one only in the header comment of gemm_pair.cuh).
-PROFILED_TRAFFIC = {"kernel_sha256_prefix": "79358ba06cfdd8e9", "workload": "llama8b",
-                    "gemm_bytes_per_useful_flop": 0.9947e9 / 1.735e12}
+# was measured on (ns_stage.cuh, gemm_pair.cuh and ptx.cuh).
+PROFILED_TRAFFIC = {"kernel_sha256_prefix": "9b968d2fc5d72c98", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 0.9860e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -671,6 +670,16 @@ def run_ours(args):
         "syrk": {"achieved": syrk_tf, "frac": (syrk_tf / peak) if syrk_tf else None},
         "stage_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
     }
+    # The prologue against the HBM roofline: per element it reads the gradient
+    # and the fp32 momentum and writes the momentum and the iterate X.
+    pro_ms, pro_n = stages["prologue"]
+    if pro_n:
+        eb = torch.tensor([], dtype=wl.dtype).element_size()
+        pro_bytes = wl.numel * (eb + 4 + 4 + eb)
+        pro_gbs = pro_bytes / (pro_ms / args.steps * 1e-3) / 1e9
+        roofline["prologue"] = {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": pro_gbs / peaks["hbm_gbs"], "bytes_per_element": eb + 4 + 4 + eb,
+                                "peak_source": f"{peak_src} hbm_gbs"}
 
     # ---- AdamW of the model's non-orthogonalised parameters (HBM-bound leg)
     adamw = None
