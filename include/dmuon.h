@@ -39,8 +39,9 @@
  *     shapes, types, options and scratch address of a call, not on the tensor
  *     addresses: a call with new shapes builds one on the host and uploads it
  *     with small kernels on `stream`; later calls with the same shapes reuse
- *     it, and new tensor addresses are written into it by one small kernel
- *     per group, in stream order.  Library memory (plans, the per-stream
+ *     it, and new tensor addresses are written into it (descriptors and the
+ *     tensor maps through which the bf16 prologue reads gradients and momentum
+ *     buffers) by one small kernel per group, in stream order.  Library memory (plans, the per-stream
  *     scratch arena) comes from a library memory pool in stream order
  *     (cudaMallocFromPoolAsync / cudaFreeAsync); a plan evicted from the cache
  *     (more than 64) is freed after the latest work that used it.  The first
