@@ -681,6 +681,12 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
           okm &= encode_2d(&mm.a, dt, d.A, ml.m, ml.m, ml.lda, BK, kBM);
           okm &= encode_2d(&mm.amn, dt, d.A, ml.m, ml.m, ml.lda, BK, BK, mn_sw);
         }
+        // A as a 3-D MN-major view: one load per transposed operand of the
+        // quintic SQUARE stage.
+        d.a3d = 0;
+        if (d.P && dt == DMUON_BF16 && ml.m % 64 == 0)
+          d.a3d = (encode_mn3d(&mm.amn3[0], d.A, ml.m, ml.m, ml.lda, 4) &&
+                   encode_mn3d(&mm.amn3[1], d.A, ml.m, ml.m, ml.lda, 2)) ? 1 : 0;
         if (d.P) {
           okm &= encode_2d(&mm.aw, dt, d.A, ml.m, ml.m, ml.lda, BK, kBN);
           okm &= encode_2d(&mm.p, dt, d.P, ml.m, ml.m, ml.lda, BK, kBM);
@@ -1024,7 +1030,10 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   np.lr = lr;
   np.wd = wd;
   np.quintic = P.quintic ? 1 : 0;
-  np.mirror = P.quintic ? 1 : 0;     // the SQUARE stage reads all of A
+  // The quintic SQUARE stage reads all of A: mirrored by the SYRK, or, on pair
+  // groups (whose A holds whole diagonal 256-blocks), read from the upper
+  // triangle with the lower k-blocks transposed.
+  np.mirror = (P.quintic && !g.gemm_pair) ? 1 : 0;
   np.a_upper = 1;                    // the GEMM reads A (or P) from its upper triangle
   np.diag_full = g.gemm_pair ? 1 : 0;  // the pair GEMM reads whole diagonal 256-blocks
   np.ca = o.ca;
@@ -1049,6 +1058,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
       sq.cb = o.cb;
       sq.cc = o.cc;
       sq.mirror = 0;
+      sq.a_upper = g.gemm_pair ? 1 : 0;
       sq.diag_full = g.gemm_pair ? 1 : 0;   // the pair GEMM reads P's whole diagonal 256-blocks
       sq.order = g.gemm_order;
       sq.tile_prefix = g.square_prefix;

@@ -7,8 +7,8 @@
 //                       s = 1 / (||M||_F + 1e-7).
 //   ns_stage_kernel     one Newton-Schulz stage for every matrix of a group
 //                       in one persistent launch:
-//                         SYRK  A = s^2 X X^T  (upper tiles; mirrored only when
-//                               the quintic SQUARE stage reads A)
+//                         SYRK  A = s^2 X X^T  (upper tiles; mirrored only for
+//                               quintic groups that do not run on CTA pairs)
 //                         SQUARE P = b A + c A A  (quintic coefficients only)
 //                         GEMM  X' = c (1.5 X - 0.5 A X), or on the last step
 //                               the weight update / output write.   [tensor]
@@ -77,6 +77,7 @@ struct MatDesc {
   int world;           // > 1: the gradient is the mean of `world` buffers Gr[0..world)
   const void* const* Gr;  // device array of the ranks' gradient buffers (rank order), or nullptr
   int tmaps;           // the gt / bt tensor maps bring a transposed prologue item's G and buf
+  int a3d;             // amn3 exists (bf16, m % 64 == 0): one load per transposed SQUARE operand
 };
 
 struct alignas(64) MatMaps {
@@ -91,6 +92,9 @@ struct alignas(64) MatMaps {
   CUtensorMap pmn;     // reads A's (or P's) lower k-blocks transposed from the upper triangle
   CUtensorMap xmn2[2]; // with b3d: the 3-D view of xmn with a box of 2 blocks (128 columns),
                        // one CTA's half of the B operand of a pair GEMM tile
+  CUtensorMap amn3[2]; // with a3d: A as a 3-D MN-major view {64 columns, rows, column blocks}
+                       // (as xmn), boxes of 4 and 2 blocks: a 256- or 128-row transposed
+                       // operand of the SQUARE stage
   CUtensorMap gt;      // with tmaps: G (rows x cols) and buf, box kTC columns x kTR rows, no
   CUtensorMap bt;      // swizzle; their addresses follow the caller's through patch_kernel
 };
@@ -111,7 +115,9 @@ struct NsParams {
   int quintic;             // GEMM reads P instead of A
   int mirror;              // SYRK / SQUARE: also write the lower triangle (A^T of the upper)
   int a_upper;             // GEMM: A (or P) holds its upper triangle and the diagonal 128-blocks
-                           // only; the k-blocks left of the diagonal block are read transposed
+                           // only; the k-blocks left of the diagonal block are read transposed.
+                           // SQUARE: A holds its upper triangle and whole diagonal 256-blocks;
+                           // both operands read their k-blocks left of that block transposed
   int diag_full;           // SYRK with 256 x 256 tiles, SQUARE: also store the lower-left
                            // 128 x 128 quarter of each diagonal 256-block (the pair GEMM reads
                            // the whole diagonal 256-block K-major)

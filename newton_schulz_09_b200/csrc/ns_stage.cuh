@@ -379,6 +379,10 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   constexpr uint32_t IDESC = make_idesc(FMT, 0u, kMode == kGemm ? 1u : 0u, kBM, kBN);
   constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);   // SYRK / SQUARE half tiles
   constexpr uint32_t IDESC_AT = make_idesc(FMT, 1u, 1u, kBM, kBN);         // GEMM, A k-block MN-major
+  // SQUARE from an upper-only A: k-blocks with both operands MN-major, or only B
+  constexpr uint32_t IDESC_TT_HALF = make_idesc(FMT, 1u, 1u, kBM, kBN / 2);
+  constexpr uint32_t IDESC_KT = make_idesc(FMT, 0u, 1u, kBM, kBN);
+  constexpr uint32_t IDESC_KT_HALF = make_idesc(FMT, 0u, 1u, kBM, kBN / 2);
   constexpr int NBOX_B = (kMode == kGemm) ? kBN / BK : 2;
   constexpr uint32_t BOX_B_BYTES = (kMode == kGemm) ? BK * 128 : kAStageBytes;
 
@@ -442,10 +446,16 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       const CUtensorMap* mapB = (kMode == kSyrk) ? &mp.xk[p.cur]
                               : (kMode == kSquare) ? &mp.a : &mp.xmn[p.cur];
       const CUtensorMap* mapBw = (kMode == kSyrk) ? &mp.xkw[p.cur] : &mp.aw;
-      const CUtensorMap* mapAt = p.quintic ? &mp.pmn : &mp.amn;
-      // GEMM with an upper-only A: k-blocks left of the row block's diagonal
-      // block come from the upper triangle, A[k rows][M columns], MN-major.
-      const int kb_t = (kMode == kGemm && p.a_upper) ? ti.tm * (kBM / BK) : 0;
+      const CUtensorMap* mapAt = (kMode == kGemm && p.quintic) ? &mp.pmn : &mp.amn;
+      // k-blocks read from the upper triangle, A[k rows][M columns], MN-major:
+      // the GEMM's A operand left of the row block's diagonal 128-block; with
+      // a_upper in the SQUARE stage (A holds its upper triangle and whole
+      // diagonal 256-blocks), the A operand left of its row block's diagonal
+      // 256-block and the B operand left of the tile's column band.
+      const int kb_t = !p.a_upper ? 0
+                     : (kMode == kGemm) ? ti.tm * (kBM / BK)
+                     : (kMode == kSquare) ? (ti.tm >> 1) * (2 * kBM / BK) : 0;
+      const int kb_bt = (kMode == kSquare && p.a_upper) ? ti.tn * (kBN / BK) : 0;
       int nb = 0;
       const int b_row0 = ti.tn * kBN + (ti.half ? kBN / 2 : 0);   // SYRK / SQUARE B operand rows
       if (kMode == kSyrk || kMode == kSquare) {
@@ -470,7 +480,13 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
         tensormap_acquire_gpu(mapA);
         tensormap_acquire_gpu(mapB);
         if (kMode != kGemm) tensormap_acquire_gpu(mapBw);
-        if (kMode == kGemm && p.a_upper) tensormap_acquire_gpu(mapAt);
+        if ((kMode == kGemm || kMode == kSquare) && p.a_upper) {
+          tensormap_acquire_gpu(mapAt);
+          if (kMode == kSquare && md.a3d) {
+            tensormap_acquire_gpu(&mp.amn3[0]);
+            tensormap_acquire_gpu(&mp.amn3[1]);
+          }
+        }
         fenced = ti.mi;
       }
       for (int kb = 0; kb < ti.nkb; ++kb) {
@@ -480,12 +496,18 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* a_dst = sa + stage * kAStageBytes;
           uint8_t* b_dst = sb + stage * kBStageBytes;
-          if (kMode == kGemm && kb < kb_t) {
+          if (kb < kb_t && !a_in_b) {
             // 128 M columns in 128-byte chunks (2 for bf16, 4 for fp32), each
-            // BK rows of K: the MN-major layout of the B operand.
+            // BK rows of K: the MN-major layout of the B operand.  The SQUARE
+            // stage loads both 64-column blocks at once through A's 3-D view
+            // (for the GEMM's A operand one load measured slower than two).
+            if (kMode == kSquare && EB == 2 && md.a3d) {
+              tma_load_3d(a_dst, &mp.amn3[1], &full[stage], 0, kb * BK, ti.tm * (kBM / 64));
+            } else {
 #pragma unroll
-            for (int h = 0; h < EB; ++h)
-              tma_load_2d(a_dst + h * (BK * 128), mapAt, &full[stage], ti.tm * kBM + h * (128 / EB), kb * BK);
+              for (int h = 0; h < EB; ++h)
+                tma_load_2d(a_dst + h * (BK * 128), mapAt, &full[stage], ti.tm * kBM + h * (128 / EB), kb * BK);
+            }
           } else if (!a_in_b) {
             tma_load_2d(a_dst, mapA, &full[stage], kb * BK, ti.tm * kBM);
           }
@@ -494,6 +516,16 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
             tma_load_3d(b_dst, mapB, &full[stage], 0, kb * BK, ti.tn * (kBN / 64));
           } else if (b_is_a) {
             // half tile: its B rows are its A rows, already loaded
+          } else if (kMode == kSquare && kb < kb_bt) {
+            // the B operand's rows as columns of the upper triangle, in
+            // 128-byte chunks of BK rows of K (MN-major, as the GEMM's X):
+            // one 3-D load of nb x 2 column blocks, else one 2-D box per chunk
+            if (EB == 2 && md.a3d) {
+              tma_load_3d(b_dst, &mp.amn3[nb == 2 ? 0 : 1], &full[stage], 0, kb * BK, b_row0 / 64);
+            } else {
+              for (int j = 0; j < nb * EB; ++j)
+                tma_load_2d(b_dst + j * (BK * 128), mapAt, &full[stage], b_row0 + j * (128 / EB), kb * BK);
+            }
           } else if (kMode != kGemm && nb == 2) {
             // Both 128-row halves of the B operand in one 256-row load.
             tma_load_2d(b_dst, mapBw, &full[stage], kb * BK, b_row0);
@@ -531,7 +563,10 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
       const uint32_t idesc = (kMode != kGemm && ti.half) ? IDESC_HALF : IDESC;
-      const int kb_t = (kMode == kGemm && p.a_upper) ? ti.tm * (kBM / BK) : 0;
+      const int kb_t = !p.a_upper ? 0                                            // as the producer
+                     : (kMode == kGemm) ? ti.tm * (kBM / BK)
+                     : (kMode == kSquare) ? (ti.tm >> 1) * (2 * kBM / BK) : 0;
+      const int kb_bt = (kMode == kSquare && p.a_upper) ? ti.tn * (kBN / BK) : 0;
       const bool a_in_b = (kMode != kGemm) && !ti.half && ti.tm == 2 * ti.tn;   // as the producer
       const bool b_is_a = (kMode != kGemm) && ti.half;
       for (int kb = 0; kb < ti.nkb; ++kb) {
@@ -544,6 +579,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
           const uint32_t a_base = a_in_b ? b_own : a_own;
           const uint32_t b_base = b_is_a ? a_own : b_own;
           const bool at = kb < kb_t;      // A k-block transposed (MN-major)
+          const bool bt = kMode == kGemm || kb < kb_bt;   // B operand MN-major
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
             const uint64_t ad =
@@ -553,12 +589,14 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
             // MN-major B: 16-bit operands use the 16-byte-unit swizzle (8-line
             // K groups); 32-bit operands must use 32-byte units (4-line groups).
             const uint64_t bd =
-                (kMode != kGemm)
-                    ? sw128_desc(b_base + k * 32, 16, 1024)
+                !bt ? sw128_desc(b_base + k * 32, 16, 1024)
                     : sw128_desc(b_base + k * MMA_K * 128, BK * 128, EB == 2 ? 1024 : 512,
                                  EB == 2 ? kSwizzle128B : kSwizzle128B32);
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-            const uint32_t id = at ? IDESC_AT : idesc;
+            const uint32_t id = (kMode == kSquare)
+                                    ? (at ? (ti.half ? IDESC_TT_HALF : IDESC_AT)
+                                          : bt ? (ti.half ? IDESC_KT_HALF : IDESC_KT) : idesc)
+                                    : (at ? IDESC_AT : idesc);
             if (EB == 2) umma_f16(d_tmem, ad, bd, id, acc);
             else umma_tf32(d_tmem, ad, bd, id, acc);
           }

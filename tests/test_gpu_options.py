@@ -176,9 +176,10 @@ def test_quintic_caller_workspace_size(cuda_lib):
 @pytest.mark.slow
 def test_quintic_on_the_large_tile_syrk(cuda_lib):
     """A 4096 x 4096 matrix runs its SYRK with 256 x 256 tiles (136 tiles in one
-    wave against 272 small ones in two); in the quintic step that kernel also
-    writes the mirrored lower triangle, which the SQUARE stage reads.  Against
-    the oracle's quintic step."""
+    wave against 272 small ones in two) and its GEMM on CTA pairs; in the
+    quintic step the SQUARE stage reads A's upper triangle, the k-blocks left
+    of each operand's diagonal 256-block transposed.  Against the oracle's
+    quintic step."""
     dm = cuda_lib
     s = (4096, 4096)
     p = torch.zeros(s, dtype=torch.bfloat16, device=DEV)

@@ -84,8 +84,9 @@ def test_one_step(cuda_lib):
 
 
 def test_quintic_coefficients(cuda_lib):
-    # P = b A + c A A from the SQUARE stage, whose diagonal 256-blocks are
-    # stored whole for the pair GEMM
+    # P = b A + c A A from the SQUARE stage, which reads A's upper triangle
+    # (lower k-blocks transposed) and stores P's diagonal 256-blocks whole for
+    # the pair GEMM
     shapes = [(1024, 4096)] * 4 + [(4096, 1024)] * 2 + [(1024, 2048)] * 2
     _run(cuda_lib, shapes, seed=350, ns_steps=3, coeffs=(3.4445, -4.7750, 2.0315))
 
@@ -96,3 +97,13 @@ def test_quintic_coefficients(cuda_lib):
 ], ids=["m%256=128", "m=1000"])
 def test_rows_ending_inside_a_pair_tile(cuda_lib, shapes):
     _run(cuda_lib, shapes, seed=360, ns_steps=2)
+
+
+@pytest.mark.parametrize("shapes", [
+    [(384, 1536)] * 36 + [(1536, 384)] * 4,
+    [(1000, 3008)] * 8 + [(3008, 1000)] * 2,
+], ids=["m%256=128", "m=1000"])
+def test_quintic_rows_ending_inside_a_pair_tile(cuda_lib, shapes):
+    # the SQUARE stage reads A's k-blocks left of each operand's diagonal
+    # 256-block transposed, with the last column band partly past m
+    _run(cuda_lib, shapes, seed=370, ns_steps=2, coeffs=(3.4445, -4.7750, 2.0315))
