@@ -844,6 +844,29 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
   return DMUON_OK;
 }
 
+// Launches `kernel` on `st` with programmatic stream serialization: its CTAs
+// may be scheduled while the previous kernel in the stream is still running.
+// Every library kernel begins with griddep_wait(), so none touches memory
+// before that kernel has completed; what overlaps is the launch and CTA
+// dispatch.  Errors surface as for a <<<>>> launch (cudaGetLastError).
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  std::memset(&attr, 0, sizeof(attr));
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Before a plan's kernels run on `st`: order after the plan's latest use on
 // another stream, then write the caller's addresses where they differ from
 // the ones the descriptors hold.
@@ -863,7 +886,7 @@ int prepare_plan(Plan& P, const std::vector<MatIn>& in, cudaStream_t st) {
   auto flush = [&]() {
     if (!pp || pp->n == 0) return;
     ++g_launches;
-    patch_kernel<<<1, 256, 0, st>>>(*pp);
+    launch_pdl(patch_kernel, 1, 256, 0, st, *pp);
     pp->n = 0;
   };
   for (size_t i = 0; i < in.size(); ++i) {
@@ -957,7 +980,7 @@ struct LaunchScope {
 // most one CTA per SM.
 template <int kMode, typename E>
 void launch_ns_stage(const NsParams& np, const DeviceInfo& d, cudaStream_t st) {
-  ns_stage_kernel<kMode, E><<<std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st>>>(np);
+  launch_pdl(ns_stage_kernel<kMode, E>, std::min(np.ntiles, d.sms), kNsThreads, kNsSmemBytes, st, np);
 }
 
 template <typename E>
@@ -986,8 +1009,8 @@ void launch_grad_norm(const Plan& P, const GroupPlan& g, const DeviceInfo& d, co
   const ElemParams ep = elem_params<E>(P, g, o);
   const int pgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * 8));
   LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
-  if (g.ranks) grad_norm_kernel<E, true><<<pgrid, kPThreads, 0, st>>>(ep);
-  else grad_norm_kernel<E, false><<<pgrid, kPThreads, 0, st>>>(ep);
+  if (g.ranks) launch_pdl(grad_norm_kernel<E, true>, pgrid, kPThreads, 0, st, ep);
+  else launch_pdl(grad_norm_kernel<E, false>, pgrid, kPThreads, 0, st, ep);
 }
 
 template <typename E>
@@ -1002,25 +1025,25 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
   {
     LaunchScope ls(st, DMUON_KERNEL_PROLOGUE);
     if (g.ranks) {
-      prologue_kernel<E, true><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+      launch_pdl(prologue_kernel<E, true>, pgrid, kPThreads, kProSmemBytes, st, ep);
     } else if (sizeof(E) == 2) {
       // bf16 iterates: the pipelined prologue, two blocks per SM when every
       // gradient is bf16 (48 KB stages), else one (64 KB stages).
       const int per_sm = g.g_bf16 ? PtCfg<true>::kBlocksPerSm : PtCfg<false>::kBlocksPerSm;
       const int tgrid = static_cast<int>(std::min<int64_t>(g.ptiles, static_cast<int64_t>(d.sms) * per_sm));
-      if (g.g_bf16) prologue_tma_kernel<true><<<tgrid, kPtThreads, PtCfg<true>::kSmem, st>>>(ep);
-      else prologue_tma_kernel<false><<<tgrid, kPtThreads, PtCfg<false>::kSmem, st>>>(ep);
+      if (g.g_bf16) launch_pdl(prologue_tma_kernel<true>, tgrid, kPtThreads, PtCfg<true>::kSmem, st, ep);
+      else launch_pdl(prologue_tma_kernel<false>, tgrid, kPtThreads, PtCfg<false>::kSmem, st, ep);
     } else {
-      prologue_kernel<E, false><<<pgrid, kPThreads, kProSmemBytes, st>>>(ep);
+      launch_pdl(prologue_kernel<E, false>, pgrid, kPThreads, kProSmemBytes, st, ep);
     }
   }
   {
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
-    finalize_kernel<<<g.nmat, 32, 0, st>>>(ep);
+    launch_pdl(finalize_kernel, g.nmat, 32, 0, st, ep);
   }
   if (steps == 0) {
     LaunchScope ls(st, DMUON_KERNEL_APPLY);
-    apply_kernel<E><<<pgrid, kPThreads, 0, st>>>(ep);
+    launch_pdl(apply_kernel<E>, pgrid, kPThreads, 0, st, ep);
     return;
   }
   NsParams np;
@@ -1050,7 +1073,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     np.ntiles = g.syrk_tiles;
     {
       LaunchScope ls(st, DMUON_KERNEL_SYRK);
-      if (g.syrk256) syrk256_kernel<E><<<std::min(np.ntiles, d.sms), kNsThreads, kS2SmemBytes, st>>>(np);
+      if (g.syrk256) launch_pdl(syrk256_kernel<E>, std::min(np.ntiles, d.sms), kNsThreads, kS2SmemBytes, st, np);
       else launch_ns_stage<kSyrk, E>(np, d, st);
     }
     if (P.quintic) {
@@ -1072,7 +1095,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
     {
       LaunchScope ls(st, DMUON_KERNEL_GEMM);
       if (g.gemm_pair)
-        gemm_pair_kernel<<<2 * std::min(np.ntiles, d.pair_clusters), kNsThreads, kG2SmemBytes, st>>>(np);
+        launch_pdl(gemm_pair_kernel, 2 * std::min(np.ntiles, d.pair_clusters), kNsThreads, kG2SmemBytes, st, np);
       else
         launch_ns_stage<kGemm, E>(np, d, st);
     }
@@ -1098,7 +1121,7 @@ int launch_plan(const Plan& P, const StepOpts& o, cudaStream_t st) {
     cp.coef = P.clip;
     cp.norm_out = o.norm_out;
     LaunchScope ls(st, DMUON_KERNEL_FINALIZE);
-    clip_coef_kernel<<<1, 256, 0, st>>>(cp);
+    launch_pdl(clip_coef_kernel, 1, 256, 0, st, cp);
   }
   for (const GroupPlan& g : P.groups) {
     if (g.dtype == DMUON_BF16) launch_group<__nv_bfloat16>(P, g, d, o, st);

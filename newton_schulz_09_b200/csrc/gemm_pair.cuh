@@ -42,6 +42,8 @@ constexpr uint32_t kG2TemptyArrivals = 2 * 4;  // one per epilogue warp of both 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNsThreads, 1)
     gemm_pair_kernel(const __grid_constant__ NsParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   using E = __nv_bfloat16;
   constexpr int BK = 64;          // K elements per stage (one 128-byte row)
   constexpr int MMA_K = 16;       // K per UMMA instruction

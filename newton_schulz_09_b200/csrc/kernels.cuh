@@ -583,6 +583,8 @@ __device__ __forceinline__ float prologue_transposed(const ElemParams& p, const 
 
 template <typename E, bool kRanks = false>
 __global__ void __launch_bounds__(kPThreads) prologue_kernel(const __grid_constant__ ElemParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(128) uint8_t pro_stage[];   // kProSmemBytes
   __shared__ float red[kPThreads / 32];
   const int tid = threadIdx.x;
@@ -790,6 +792,8 @@ __device__ __forceinline__ float pt_transposed(const ElemParams& p, const MatDes
 
 template <bool kGBf16>
 __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_constant__ ElemParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   using Cfg = PtCfg<kGBf16>;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(128) uint8_t pt_raw[];    // Cfg::kSmem
@@ -916,6 +920,8 @@ __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_c
 // prologue work item (the items cover every gradient element exactly once).
 template <typename E, bool kRanks = false>
 __global__ void __launch_bounds__(kPThreads) grad_norm_kernel(const __grid_constant__ ElemParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ double red[kPThreads / 32];
   const int tid = threadIdx.x;
   // A block's items only move forward through the matrices: one search,
@@ -980,6 +986,8 @@ struct ClipParams {
 };
 
 __global__ void clip_coef_kernel(const __grid_constant__ ClipParams cp) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ double red[32];
   double acc = 0.0;
   for (int gi = 0; gi < 2; ++gi)
@@ -1001,6 +1009,8 @@ __global__ void clip_coef_kernel(const __grid_constant__ ClipParams cp) {
 // One warp per matrix: s = 1 / (sqrt(sum of partials) + 1e-7), summed in a
 // fixed order (deterministic).
 __global__ void finalize_kernel(const __grid_constant__ ElemParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int mi = blockIdx.x;
   const int lane = threadIdx.x;
   const int64_t b = p.ptile_prefix[mi], e = p.ptile_prefix[mi + 1];
@@ -1015,6 +1025,8 @@ __global__ void finalize_kernel(const __grid_constant__ ElemParams p) {
 // prologue.
 template <typename E>
 __global__ void __launch_bounds__(kPThreads) apply_kernel(const __grid_constant__ ElemParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   // A block's items only move forward through the matrices: one search,
   // then a cursor.
   int mi = blockIdx.x < p.ntiles ? find_slot64(p.ptile_prefix, p.nmat, blockIdx.x) : 0;
@@ -1105,6 +1117,8 @@ __device__ __forceinline__ void load8_any(const void* base, bool bf16, int64_t i
 }
 
 __global__ void __launch_bounds__(kPThreads) adamw_kernel(const __grid_constant__ AdamParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int64_t it = blockIdx.x; it < p.nitems; it += gridDim.x) {
     int lo = 0, hi = p.count - 1;
     while (lo < hi) {
@@ -1294,6 +1308,8 @@ __device__ __forceinline__ void clip_scale_item(const ClipTensor& T, int64_t it,
 }
 
 __global__ void __launch_bounds__(kPThreads, 4) clip_norm_kernel(const __grid_constant__ ClipBucketParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ double red[kPThreads / 32];
   const int tid = threadIdx.x;
   for (int64_t it = p.item_begin + blockIdx.x; it < p.item_end; it += gridDim.x) {
@@ -1317,6 +1333,8 @@ __global__ void __launch_bounds__(kPThreads, 4) clip_norm_kernel(const __grid_co
 // (four loads in flight) over a fixed stride, so the order is fixed.
 constexpr int kClipFinThreads = 1024;
 __global__ void __launch_bounds__(kClipFinThreads) clip_finalize_kernel(const __grid_constant__ ClipFinalizeParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ double red[kClipFinThreads / 32];
   const int s = blockIdx.x;
   const int64_t b = p.seg_item0[s], e = p.seg_item0[s + 1];
@@ -1345,6 +1363,8 @@ __global__ void __launch_bounds__(kClipFinThreads) clip_finalize_kernel(const __
 }
 
 __global__ void __launch_bounds__(kPThreads, 4) clip_scale_kernel(const __grid_constant__ ClipBucketParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t n = p.item_end - p.item_begin;
   for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
     const int64_t it = p.item_end - 1 - r;
@@ -1372,6 +1392,8 @@ struct UploadParams {
   uint4 w[kUploadWords];
 };
 __global__ void __launch_bounds__(256) upload_kernel(const __grid_constant__ UploadParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = threadIdx.x; i < p.nwords; i += blockDim.x) p.dst[i] = p.w[i];
   tensormap_release_gpu();
 }
@@ -1391,6 +1413,8 @@ struct PatchParams {
   PatchEntry e[kPatchMax];
 };
 __global__ void __launch_bounds__(256) patch_kernel(const __grid_constant__ PatchParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = threadIdx.x; i < p.n; i += blockDim.x) {
     MatDesc& d = p.mats[p.e[i].index];
     d.W = p.e[i].W;

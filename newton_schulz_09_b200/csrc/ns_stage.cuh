@@ -371,6 +371,8 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
 // ======================================================================
 template <int kMode, typename E>
 __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_constant__ NsParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int EB = static_cast<int>(sizeof(E));
   constexpr int BK = 128 / EB;              // K elements per stage (one 128-byte row)
   constexpr int MMA_K = 32 / EB;            // K per UMMA instruction

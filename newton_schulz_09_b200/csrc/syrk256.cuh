@@ -56,6 +56,8 @@ __device__ __forceinline__ Tile256 decode_tile256(const NsParams& p, int t) {
 
 template <typename E>
 __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_constant__ NsParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int EB = static_cast<int>(sizeof(E));
   constexpr int BK = 128 / EB;
   constexpr int MMA_K = 32 / EB;
