@@ -901,8 +901,9 @@ __global__ void __launch_bounds__(kPtThreads) prologue_tma_kernel(const __grid_c
     // This warp has read its staged values: release the stage.
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
-    // Fixed-order reduction of the item's sum of squares (red is double
-    // buffered, so one barrier per item suffices).
+    // Fixed-order reduction of the item's sum of squares over the eight
+    // warps (red alternates between two rows, so the next item's writes never
+    // race thread 0's read of this one).
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (lane == 0) red[it & 1u][warp] = ss;
