@@ -35,12 +35,12 @@ UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage: the ncu
-# capture of one Llama-8B layer's GEMM on CTA pairs (550.0 MB read + 411.5 MB written for
+# capture of one Llama-8B layer's GEMM on CTA pairs (547.5 MB read + 410.5 MB written for
 # 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so its traffic is
 # this ratio times the useful FLOPs of that launch.  Valid only for the stage kernels' source it
 # was measured on (ns_stage.cuh, gemm_pair.cuh and ptx.cuh).
-PROFILED_TRAFFIC = {"kernel_sha256_prefix": "2c9ef7edaa07a704", "workload": "llama8b",
-                    "gemm_bytes_per_useful_flop": 0.9615e9 / 1.735e12}
+PROFILED_TRAFFIC = {"kernel_sha256_prefix": "23cd5b6c8c04e86e", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 0.9580e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -755,7 +755,7 @@ def run_ours(args):
 
     # ---- the same stack with quintic coefficients (one more symmetric product)
     quintic = None
-    if not args.no_quintic and wl.name == "llama8b":
+    if not args.no_quintic and wl.name in ("llama8b", "llama8b_layer"):
         quintic = measure_quintic(dm, t, wl, dev, stream, world, peaks, 3)
 
     status = dm.dmuon_device_status()
