@@ -582,9 +582,26 @@ def pin_quintic_coefficients(o, seed: int = 24) -> None:
     assert _rel(o.newton_schulz(G, 4, (1.875, -0.875, 0.0)), o.newton_schulz(G, 4, (1.875, -0.875))) <= 1e-15
 
 
+def pin_ns_flops(o) -> None:
+    """Useful Newton-Schulz FLOPs as the metric counts them: per step m^2 n for
+    the symmetric product X X^T (half of the dense 2 m^2 n) and 2 m^2 n for
+    (X X^T) X, with m the short side and n the long one; the quintic form adds
+    m^3 for the symmetric square A A (half of the dense 2 m^3).  Hand-counted:
+    * 2 x 3, one step: 4 * 3 + 2 * 4 * 3 = 36; its transpose 3 x 2 too;
+    * five steps: 180; quintic, one step: 36 + 2^3 = 44;
+    * 1024 x 4096, one step: 3 * 2^20 * 2^12 = 12 884 901 888;
+    * 4096 x 4096, five steps: 15 * 2^36 = 1 030 792 151 040."""
+    assert o.ns_flops(2, 3, 1) == 36.0, o.ns_flops(2, 3, 1)
+    assert o.ns_flops(3, 2, 1) == 36.0, o.ns_flops(3, 2, 1)
+    assert o.ns_flops(2, 3, 5) == 180.0
+    assert o.ns_flops(2, 3, 1, quintic=True) == 44.0, o.ns_flops(2, 3, 1, quintic=True)
+    assert o.ns_flops(1024, 4096, 1) == 12884901888.0
+    assert o.ns_flops(4096, 4096, 5) == 1030792151040.0
+
+
 ALL_PINS = (pin_scalar_closed_form, pin_spectral_map, pin_orthogonal_input,
             pin_monotone_error, pin_symmetries, pin_momentum_bitwise,
             pin_nesterov_post_update, pin_update_closed_form, pin_custom_coefficients,
             pin_lr_scale, pin_gradient_clipping, pin_adamw, pin_rank_mean,
             pin_relative_frobenius, pin_orthogonality_error, pin_round_to_bf16,
-            pin_clip_buckets, pin_quintic_coefficients)
+            pin_clip_buckets, pin_quintic_coefficients, pin_ns_flops)

@@ -287,6 +287,26 @@ MUTANTS["quintic_b_c_swapped"] = dict(ns_iteration=_quintic_variant("b_c_swapped
 MUTANTS["quintic_c_ignored"] = dict(ns_iteration=_quintic_variant("c_ignored"))
 
 
+def _ns_flops_variant(kind):
+    def f(rows, cols, steps, quintic=False):
+        m, n = min(rows, cols), max(rows, cols)
+        if kind == "long_side":            # m and n swapped
+            m, n = n, m
+        if kind == "dense_gram":           # X X^T counted as the dense 2 m^2 n
+            per = 4.0 * m * m * n
+        else:
+            per = 3.0 * m * m * n
+        if quintic:
+            per += (2.0 if kind == "dense_square" else 1.0) * float(m) ** 3
+        return float(steps) * per
+    return f
+
+
+MUTANTS["ns_flops_long_side"] = dict(ns_flops=_ns_flops_variant("long_side"))
+MUTANTS["ns_flops_dense_gram"] = dict(ns_flops=_ns_flops_variant("dense_gram"))
+MUTANTS["ns_flops_dense_square"] = dict(ns_flops=_ns_flops_variant("dense_square"))
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(name):
     m = _mutant(**MUTANTS[name])
