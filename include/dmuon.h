@@ -357,10 +357,12 @@ int64_t dmuon_plan_builds(void);
  * one word per dtype group (at most max_groups; kernels may be NULL) and
  * returns the plan's number of groups, 0 when no plan exists.  Each word
  * ORs DMUON_PLAN_SYRK256 (the SYRK runs on 256 x 256 tiles, else 128 x 256)
- * and DMUON_PLAN_GEMM_PAIR (the GEMM runs 256 x 256 tiles on two-CTA
- * clusters, else 128 x 256 tiles on single CTAs). */
+ * DMUON_PLAN_GEMM_PAIR (the GEMM runs 256 x 256 tiles on two-CTA clusters,
+ * else 128 x 256 tiles on single CTAs) and DMUON_PLAN_SQUARE256 (quintic
+ * plans: the SQUARE stage runs on 256 x 256 tiles, else 128 x 256). */
 #define DMUON_PLAN_SYRK256 1
 #define DMUON_PLAN_GEMM_PAIR 2
+#define DMUON_PLAN_SQUARE256 4
 int dmuon_debug_last_plan(int* kernels, int max_groups);
 
 /* Test hook (host only, launches nothing): the device-memory check the entry

@@ -487,12 +487,14 @@ def dmuon_plan_builds() -> int:
 
 def dmuon_debug_last_plan() -> list:
     """Stage kernels of the most recently used launch plan, one dict per
-    dtype group: {"syrk256": bool, "gemm_pair": bool} (launches nothing)."""
+    dtype group: {"syrk256": bool, "gemm_pair": bool, "square256": bool}
+    (launches nothing)."""
     lib = load_library()
     n = int(lib.dmuon_debug_last_plan(None, 0))
     words = (ctypes.c_int32 * max(n, 1))()
     lib.dmuon_debug_last_plan(words, n)
-    return [{"syrk256": bool(words[i] & 1), "gemm_pair": bool(words[i] & 2)} for i in range(n)]
+    return [{"syrk256": bool(words[i] & 1), "gemm_pair": bool(words[i] & 2), "square256": bool(words[i] & 4)}
+            for i in range(n)]
 
 
 def dmuon_debug_check_pointer(address: int) -> int:

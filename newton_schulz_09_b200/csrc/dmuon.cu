@@ -262,6 +262,7 @@ struct GroupPlan {
   int syrk_tiles, gemm_tiles, square_tiles;
   bool syrk256 = true;    // SYRK by syrk256_kernel (256 x 256 tiles), else ns_stage_kernel<kSyrk>
   bool gemm_pair = false; // GEMM by gemm_pair_kernel (256 x 256 tiles on CTA pairs)
+  bool square256 = false; // quintic SQUARE by syrk256_kernel<kSquare> (pair groups whose A has a 3-D view)
   const int* syrk_order; const int* syrk_prefix;
   const int* gemm_order; const int* gemm_prefix;
   const int* square_prefix;   // SQUARE tiles along gemm_order (quintic plans)
@@ -383,7 +384,8 @@ int device_setup(int dev) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
   }
   const void* ks2[] = {reinterpret_cast<const void*>(&syrk256_kernel<__nv_bfloat16>),
-                       reinterpret_cast<const void*>(&syrk256_kernel<float>)};
+                       reinterpret_cast<const void*>(&syrk256_kernel<float>),
+                       reinterpret_cast<const void*>(&syrk256_kernel<__nv_bfloat16, kSquare>)};
   for (const void* k : ks2) {
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kS2SmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
@@ -723,6 +725,8 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       const MatDesc& x = descs[first + a]; const MatDesc& y = descs[first + b];
       return x.m != y.m ? x.m > y.m : x.n > y.n;
     });
+    gp.square256 = gp.gemm_pair;
+    for (int k = 0; k < gp.nmat; ++k) gp.square256 = gp.square256 && descs[first + k].a3d;
     int64_t st = 0, gt = 0, qt = 0;
     A.sp.push_back(0);
     A.gp.push_back(0);
@@ -732,7 +736,9 @@ int get_plan(const std::vector<MatIn>& in, int steps, bool quintic, void* ws, in
       st += gp.syrk256 ? syrk256_tiles_of(mk) : syrk_tiles_of(mk);
       gt += gp.gemm_pair ? gemm_pair_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n)
                          : gemm_tiles_of(descs[first + go[k]].m, descs[first + go[k]].n);
-      qt += syrk_tiles_of(descs[first + go[k]].m);   // SQUARE contracts over m: the GEMM's order
+      // SQUARE contracts over m, in the GEMM's order; on 256 x 256 tiles
+      // (syrk256_kernel) when square256, else on 128 x 256 ones
+      qt += gp.square256 ? syrk256_tiles_of(descs[first + go[k]].m) : syrk_tiles_of(descs[first + go[k]].m);
       A.sp.push_back(static_cast<int>(st));
       A.gp.push_back(static_cast<int>(gt));
       A.qp.push_back(static_cast<int>(qt));
@@ -1087,7 +1093,15 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
       sq.tile_prefix = g.square_prefix;
       sq.ntiles = g.square_tiles;
       LaunchScope ls(st, DMUON_KERNEL_SQUARE);
-      launch_ns_stage<kSquare, E>(sq, d, st);
+      bool big = false;
+      if constexpr (sizeof(E) == 2) {
+        if (g.square256) {
+          // 256 x 256 tiles; A holds its upper triangle and whole diagonal 256-blocks
+          launch_pdl(syrk256_kernel<E, kSquare>, std::min(sq.ntiles, d.sms), kNsThreads, kS2SmemBytes, st, sq);
+          big = true;
+        }
+      }
+      if (!big) launch_ns_stage<kSquare, E>(sq, d, st);
     }
     np.order = g.gemm_order;
     np.tile_prefix = g.gemm_prefix;
@@ -1800,7 +1814,8 @@ int dmuon_debug_last_plan(int* kernels, int max_groups) {
   const int n = static_cast<int>(P.groups.size());
   for (int i = 0; i < n && i < max_groups; ++i)
     if (kernels)
-      kernels[i] = (P.groups[i].syrk256 ? DMUON_PLAN_SYRK256 : 0) | (P.groups[i].gemm_pair ? DMUON_PLAN_GEMM_PAIR : 0);
+      kernels[i] = (P.groups[i].syrk256 ? DMUON_PLAN_SYRK256 : 0) | (P.groups[i].gemm_pair ? DMUON_PLAN_GEMM_PAIR : 0) |
+                   (P.quintic && P.groups[i].square256 ? DMUON_PLAN_SQUARE256 : 0);
   return n;
 }
 

@@ -43,18 +43,24 @@ struct Tile256 {
   bool diag;
 };
 
-template <int BK>
+template <int BK, int kMode = kSyrk>
 __device__ __forceinline__ Tile256 decode_tile256(const NsParams& p, int t) {
   Tile256 ti;
   const int slot = find_slot(p.tile_prefix, p.nmat, t);
   ti.mi = __ldg(p.order + slot);
   syrk256_tile_coords(t - __ldg(p.tile_prefix + slot), ti.I, ti.J);
-  ti.nkb = (p.mats[ti.mi].n + BK - 1) / BK;
+  ti.nkb = ((kMode == kSquare ? p.mats[ti.mi].m : p.mats[ti.mi].n) + BK - 1) / BK;
   ti.diag = ti.I == ti.J;
   return ti;
 }
 
-template <typename E>
+// kMode == kSquare: the quintic SQUARE stage P = cb A + cc A A on the same
+// tiles (bf16 groups on CTA pairs only).  Its operands are rows of A, K = m;
+// A holds its upper triangle and whole diagonal 256-blocks, so an operand's
+// k-blocks left of its own diagonal 256-block come transposed from the upper
+// triangle (one 3-D load through A's MN-major view, MN-major descriptors).
+// The epilogue adds cb A, read back from A's tile, and stores P like A.
+template <typename E, int kMode = kSyrk>
 __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_constant__ NsParams p) {
   griddep_wait();
   griddep_launch_dependents();
@@ -65,6 +71,12 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
   constexpr uint32_t FMT = (EB == 2) ? 1u : 2u;
   constexpr uint32_t IDESC = make_idesc(FMT, 0u, 0u, kBM, kBN);
   constexpr uint32_t IDESC_HALF = make_idesc(FMT, 0u, 0u, kBM, kBN / 2);
+  // SQUARE k-blocks with the B operand, or both operands, MN-major
+  constexpr uint32_t IDESC_KT = make_idesc(FMT, 0u, 1u, kBM, kBN);
+  constexpr uint32_t IDESC_KT_HALF = make_idesc(FMT, 0u, 1u, kBM, kBN / 2);
+  constexpr uint32_t IDESC_TT = make_idesc(FMT, 1u, 1u, kBM, kBN);
+  constexpr uint32_t IDESC_TT_HALF = make_idesc(FMT, 1u, 1u, kBM, kBN / 2);
+  static_assert(kMode == kSyrk || EB == 2, "the SQUARE mode is bf16 only");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -110,10 +122,16 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
     for (int s = 0; s < kS2Stages; ++s) { issued[s] = false; issued_phase[s] = 0; }
     int fenced = -1;
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
-      const CUtensorMap* map = &p.maps[ti.mi].xkw[p.cur];     // 256-row K-major boxes of X
+      const Tile256 ti = decode_tile256<BK, kMode>(p, t);
+      const MatMaps& mp = p.maps[ti.mi];
+      // 256-row K-major boxes of X (SYRK) or A (SQUARE)
+      const CUtensorMap* map = (kMode == kSquare) ? &mp.aw : &mp.xkw[p.cur];
+      // SQUARE: k-blocks left of the A rows' (B rows') diagonal 256-block
+      const int kb_at = (kMode == kSquare) ? ti.I * (kBN / BK) : 0;
+      const int kb_bt = (kMode == kSquare) ? ti.J * (kBN / BK) : 0;
       if (lane == 0 && ti.mi != fenced) {
         tensormap_acquire_gpu(map);
+        if (kMode == kSquare) tensormap_acquire_gpu(&mp.amn3[0]);
         fenced = ti.mi;
       }
       const uint32_t bytes = ti.diag ? kS2OpBytes : 2 * kS2OpBytes;
@@ -123,8 +141,12 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* a_dst = smem + stage * 2 * kS2OpBytes;
-          if (!ti.diag) tma_load_2d(a_dst, map, &full[stage], kb * BK, ti.I * kBN);
-          tma_load_2d(a_dst + kS2OpBytes, map, &full[stage], kb * BK, ti.J * kBN);
+          if (!ti.diag) {
+            if (kb < kb_at) tma_load_3d(a_dst, &mp.amn3[0], &full[stage], 0, kb * BK, ti.I * (kBN / 64));
+            else tma_load_2d(a_dst, map, &full[stage], kb * BK, ti.I * kBN);
+          }
+          if (kb < kb_bt) tma_load_3d(a_dst + kS2OpBytes, &mp.amn3[0], &full[stage], 0, kb * BK, ti.J * (kBN / 64));
+          else tma_load_2d(a_dst + kS2OpBytes, map, &full[stage], kb * BK, ti.J * kBN);
         }
         __syncwarp();
         issued[stage] = true;
@@ -142,7 +164,9 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
     uint32_t phase = 0;
     int lt = 0;
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
+      const Tile256 ti = decode_tile256<BK, kMode>(p, t);
+      const int kb_at = (kMode == kSquare) ? ti.I * (kBN / BK) : 0;   // as the producer
+      const int kb_bt = (kMode == kSquare) ? ti.J * (kBN / BK) : 0;
       bool w = mbar_wait(tempty, (static_cast<uint32_t>(lt) & 1u) ^ 1u, p.err, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
@@ -154,17 +178,26 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
           const uint32_t own = smem_u32(smem + stage * 2 * kS2OpBytes);
           const uint32_t b_base = own + kS2OpBytes;
           const uint32_t a_base = ti.diag ? b_base : own;
+          const bool at = kb < kb_at, bt = kb < kb_bt;    // MN-major operands (SQUARE)
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const uint64_t ad = sw128_desc(a_base + h * (kS2OpBytes / 2) + k * 32, 16, 1024);
+              // a half is 128 rows: 16 KB K-major, or two 8 KB column blocks MN-major
+              const uint32_t a_h = a_base + h * (kS2OpBytes / 2);
+              const uint64_t ad = at ? sw128_desc(a_h + k * MMA_K * 128, BK * 128, 1024, kSwizzle128B)
+                                     : sw128_desc(a_h + k * 32, 16, 1024);
               const bool quarter = ti.diag && h == 1;   // 128 x 128 over the B rows 128 .. 255
-              const uint64_t bd = sw128_desc(b_base + (quarter ? kS2OpBytes / 2 : 0) + k * 32, 16, 1024);
+              const uint32_t b_q = b_base + (quarter ? kS2OpBytes / 2 : 0);
+              const uint64_t bd = bt ? sw128_desc(b_q + k * MMA_K * 128, BK * 128, 1024, kSwizzle128B)
+                                     : sw128_desc(b_q + k * 32, 16, 1024);
+              const uint32_t id = at ? (quarter ? IDESC_TT_HALF : IDESC_TT)
+                                : bt ? (quarter ? IDESC_KT_HALF : IDESC_KT)
+                                     : (quarter ? IDESC_HALF : IDESC);
               const uint32_t d = tmem_base + static_cast<uint32_t>(h * kBN);
-              if (EB == 2) umma_f16(d, ad, bd, quarter ? IDESC_HALF : IDESC, acc);
-              else umma_tf32(d, ad, bd, quarter ? IDESC_HALF : IDESC, acc);
+              if (EB == 2) umma_f16(d, ad, bd, id, acc);
+              else umma_tf32(d, ad, bd, id, acc);
             }
           }
           umma_commit(&empty[stage]);
@@ -188,25 +221,28 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
     uint32_t gq = 0;          // store quarters so far (slot ring position)
     int lt = 0;
     for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++lt) {
-      const Tile256 ti = decode_tile256<BK>(p, t);
+      const Tile256 ti = decode_tile256<BK, kMode>(p, t);
       const MatDesc& md = p.mats[ti.mi];
       const float s = *md.scale;
       bool w = mbar_wait(tfull, static_cast<uint32_t>(lt) & 1u, p.err, p.wait_limit_ns);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      const float alpha = p.first ? s * s : 1.0f;
-      E* A = reinterpret_cast<E*>(md.A);
+      // SYRK: A = alpha X X^T.  SQUARE: P = cc (A A) + cb A.
+      const float alpha = (kMode == kSquare) ? p.cc : (p.first ? s * s : 1.0f);
+      E* A = reinterpret_cast<E*>(kMode == kSquare ? md.P : md.A);    // the stored matrix
+      const E* Asrc = reinterpret_cast<const E*>(md.A);
       const int64_t lda = md.lda;
       const int m = md.m;
-      if (EB == 2 && !p.mirror) {
+      if (EB == 2 && (!p.mirror || kMode == kSquare)) {
         // Upper triangle and diagonal 128-blocks through shared memory: each
         // 128 x 64 quarter goes TMEM -> registers -> a 128B-swizzled slot ->
         // one TMA store into A (clipped at m).  Two slots alternate; a slot
         // is rewritten only after the store two quarters back has read it.
         // The accumulators are released after the tile's last TMEM load.
         const bool leader = (warp == 2 && lane == 0);
+        const CUtensorMap* smap = (kMode == kSquare) ? &p.maps[ti.mi].p : &p.maps[ti.mi].a;
         if (leader && ti.mi != fenced_a) {
-          tensormap_acquire_gpu(&p.maps[ti.mi].a);
+          tensormap_acquire_gpu(smap);
           fenced_a = ti.mi;
         }
         const int nq0 = kBN / 64;
@@ -220,6 +256,36 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
           const int C0 = ti.J * kBN + (quarter ? kBN / 2 : 0) + q * 64;
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16) +
                                  static_cast<uint32_t>(h * kBN + q * 64);
+          // SQUARE: this row's 64 values of A under the quarter (cb A), loaded
+          // before the TMEM reads so that both latencies overlap
+          uint32_t ar[32];
+          if (kMode == kSquare) {
+            const int R = R0 + row_in_tile;
+            const E* arow = Asrc + static_cast<int64_t>(R) * lda + C0;
+            if (R < m && C0 + 64 <= m) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const uint4 u = reinterpret_cast<const uint4*>(arow)[i];
+                ar[4 * i] = u.x; ar[4 * i + 1] = u.y; ar[4 * i + 2] = u.z; ar[4 * i + 3] = u.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const bool in0 = R < m && C0 + 2 * i < m, in1 = R < m && C0 + 2 * i + 1 < m;
+                const __nv_bfloat162 pr = __floats2bfloat162_rn(in0 ? to_f<E>(arow[2 * i]) : 0.0f,
+                                                                in1 ? to_f<E>(arow[2 * i + 1]) : 0.0f);
+                ar[i] = *reinterpret_cast<const uint32_t*>(&pr);
+              }
+            }
+          }
+          // the stored value from an accumulator: alpha acc (SYRK), or
+          // fl(cb A + fl(cc acc)) (SQUARE, as ns_stage_kernel rounds it)
+          auto value = [&](uint32_t acc_bits, int col) -> float {
+            const float y = alpha * __uint_as_float(acc_bits);
+            if (kMode != kSquare) return y;
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ar[col >> 1]));
+            return fmaf(p.cb, (col & 1) ? f.y : f.x, y);
+          };
           uint32_t v0[32], v1[32];
           tmem_ld32(taddr, v0);
           tmem_ld32(taddr + 32, v1);
@@ -236,8 +302,8 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int col = c * 8 + 2 * j;
-              const float a0 = alpha * __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
-              const float a1 = alpha * __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
+              const float a0 = value(col < 32 ? v0[col] : v1[col - 32], col);
+              const float a1 = value(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32], col + 1);
               __nv_bfloat162 yv = __floats2bfloat162_rn(a0, a1);
               wv[j] = *reinterpret_cast<uint32_t*>(&yv);
             }
@@ -251,7 +317,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
             if (R < m) {
 #pragma unroll
               for (int j = 0; j < 64; ++j) {
-                const float a = alpha * __uint_as_float(j < 32 ? v0[j] : v1[j - 32]);
+                const float a = value(j < 32 ? v0[j] : v1[j - 32], j);
                 if (C0 + j < m) A[static_cast<int64_t>(C0 + j) * lda + R] = __float2bfloat16_rn(a);
               }
             }
@@ -260,7 +326,7 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
           named_bar_sync(1, 128);
           if (leader) {
             if (R0 < m && C0 < m)
-              tma_store_2d(&p.maps[ti.mi].a, epi + slot * kEpiSlotBytes, C0, R0);
+              tma_store_2d(smap, epi + slot * kEpiSlotBytes, C0, R0);
             bulk_commit_group();
             bulk_wait_group_read1();     // the other slot's store has read it
           }

@@ -42,6 +42,10 @@ def _run(dm, shapes, *, seed, ns_steps, zero_w=True, nesterov=True, wd=0.0, lr=0
     assert dm.dmuon_device_status() == 0
     plan = dm.dmuon_debug_last_plan()
     assert plan and all(g["gemm_pair"] and g["syrk256"] for g in plan), plan
+    if coeffs is not None and len(coeffs) == 3:
+        # the SQUARE on 256 x 256 tiles wherever A has its 3-D view (m % 64 == 0)
+        want = all(min(s) % 64 == 0 for s in shapes)
+        assert all(g["square256"] == want for g in plan), plan
     for i, s in enumerate(shapes):
         buf_ref, X_ref, W_ref = oracle.muon_step(w0[i], host(grads[i]), b0[i], lr=lr, momentum=0.95,
                                                  nesterov=nesterov, weight_decay=wd, ns_steps=ns_steps,
