@@ -11,7 +11,8 @@ namespace dmuon {
 // ======================================================================
 // SYRK with 256 x 256 tiles per CTA.  A is stored as its upper triangle and
 // diagonal 128-blocks (with diag_full: diagonal 256-blocks, for the pair
-// GEMM), or in full (mirrored) when the quintic SQUARE stage reads it.  Each k-block brings 256 rows of X for the A operand
+// GEMM), or in full (mirrored) when a quintic SQUARE stage on 128 x 256 tiles
+// reads it K-major.  Each k-block brings 256 rows of X for the A operand
 // and 256 for the B operand (64 KB) and feeds two 128 x 256 UMMA halves that
 // share the B operand: a third fewer operand bytes per FLOP than 128 x 256
 // tiles.  The two fp32 accumulators take all 512 TMEM columns, so a tile's
