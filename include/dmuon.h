@@ -119,7 +119,7 @@ size_t dmuon_ns_workspace_bytes(int64_t m, int64_t n, int dtype);
  * dmuon_muon_step_batched -- one Muon update of `count` matrices, with one
  * launch per stage for a whole group of them (the per-parameter loop of the
  * blog's Vanilla Muon, "代码实现" section, done as grouped kernels).  A call
- * of more than 2^29 elements runs as consecutive groups of at most about
+ * of more than 2^28 elements runs as consecutive groups of at most about
  * that many (in the order given, at most 32 groups, one after the other on
  * the stream and sharing one scratch region); the result of each matrix does
  * not depend on the grouping.  With gradient clipping the call is one group.

@@ -1214,9 +1214,11 @@ int gather(void* const params[], const void* const grads[], float* const bufs[],
 // the stream, sharing one scratch region.  Measured on the Llama-8B stack
 // (224 matrices, 7e9 elements): groups of one to four layers run at a higher
 // SM clock under the power cap than one launch per stage over every matrix
-// (413 ms against 440 ms per step), two-layer groups (~2^29 elements) best
-// by about 1 %; the arithmetic of each matrix does not depend on the grouping.
-constexpr int64_t kGroupElems = int64_t(1) << 29;
+// (413 ms against 440 ms per step).  With the current kernels, groups of
+// about one layer (2^28 elements) run 0.5-2 % faster than two-layer groups
+// and 3-4 % faster than four-layer ones, at a higher SM clock; the arithmetic
+// of each matrix does not depend on the grouping.
+constexpr int64_t kGroupElems = int64_t(1) << 28;
 constexpr int kMaxGroups = 32;   // < kMaxPlans: one call never evicts its own plans
 
 // Boundaries of consecutive groups: a matrix joins the current group unless

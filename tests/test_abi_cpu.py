@@ -175,16 +175,16 @@ def _llama_dims():
 
 
 def test_device_call_groups(lib):
-    """Consecutive groups of at most 2^29 elements, each as full as the next
+    """Consecutive groups of at most 2^28 elements, each as full as the next
     matrix allows, at most 32."""
     dims = _llama_dims()
     b = _partition(lib, dims, 0)
     elems = [r * c for r, c in dims]
     for lo, hi in zip(b, b[1:]):
-        assert sum(elems[lo:hi]) <= 2 ** 29 or hi - lo == 1
+        assert sum(elems[lo:hi]) <= 2 ** 28 or hi - lo == 1
         if hi < len(dims):
-            assert sum(elems[lo:hi + 1]) > 2 ** 29
-    assert len(b) - 1 == 14
+            assert sum(elems[lo:hi + 1]) > 2 ** 28
+    assert len(b) - 1 == 32
     assert _partition(lib, [(256, 512), (512, 256)], 0) == [0, 2]
     big = [(16384, 16384)] * 64                       # 1.7e10 elements: the cap of 32 groups
     assert len(_partition(lib, big, 0)) - 1 <= 32

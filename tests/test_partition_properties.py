@@ -1,10 +1,10 @@
 """Properties of the library's two grouping rules over random shape lists
 (host logic, no GPU), read through ``dmuon_debug_partition``:
 
-* device groups (a call above 2^29 elements runs as consecutive groups):
-  at most 32 groups; a call of at most 2^29 elements is one group; a group
+* device groups (a call above 2^28 elements runs as consecutive groups):
+  at most 32 groups; a call of at most 2^28 elements is one group; a group
   is closed only when the next matrix would take it past a target of at
-  least 2^29 elements;
+  least 2^28 elements;
 * host-buffer groups (the ramp of the host-buffer step): at most 32 groups;
   every group but the last holds at least max(64 MiB, total / 128) of
   gradient bytes, so a small call is one group.
@@ -51,11 +51,11 @@ def test_device_groups(dims):
     elems = [r * c for r, c in dims]
     total = sum(elems)
     assert len(b) - 1 <= 32
-    if total <= 2 ** 29:
+    if total <= 2 ** 28:
         assert b == [0, len(dims)]
     for lo, hi in zip(b[:-1], b[1:-1]):
-        # closed only because the next matrix would overflow the target (>= 2^29)
-        assert sum(elems[lo:hi + 1]) > 2 ** 29
+        # closed only because the next matrix would overflow the target (>= 2^28)
+        assert sum(elems[lo:hi + 1]) > 2 ** 28
 
 
 @SETTINGS
