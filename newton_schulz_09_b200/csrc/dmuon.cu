@@ -1406,7 +1406,7 @@ std::vector<int> ramp_bounds(const std::vector<size_t>& bytes) {
   const int n = static_cast<int>(bytes.size());
   size_t total = 0;
   for (size_t b : bytes) total += b;
-  const size_t first = std::max(kChunkTargetBytes, total / 128);
+  const size_t first = kChunkTargetBytes;
   const size_t mid = std::max(size_t(1) << 30, total / (DMUON_MAX_CHUNKS / 2));
   std::vector<int> bnd(1, 0);
   size_t acc = 0, done = 0;

@@ -201,7 +201,7 @@ def test_host_step_groups_ramp(lib):
     assert 8 <= len(sizes) <= 32
     assert sizes[0] <= total / 32 and sizes[-1] <= total / 32
     assert max(sizes) <= (1 << 30) + biggest
-    first = max(64 << 20, total // 128)
+    first = 64 << 20
     for k, sz in enumerate(sizes[:-1]):
         assert sz < first * 1.5 ** k + biggest
     assert _partition(lib, [(256, 512)] * 3, 1) == [0, 3]     # small totals: one group

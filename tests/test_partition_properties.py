@@ -6,7 +6,7 @@
   is closed only when the next matrix would take it past a target of at
   least 2^28 elements;
 * host-buffer groups (the ramp of the host-buffer step): at most 32 groups;
-  every group but the last holds at least max(64 MiB, total / 128) of
+  every group but the last holds at least 64 MiB of
   gradient bytes, so a small call is one group.
 """
 import ctypes
@@ -64,7 +64,7 @@ def test_host_buffer_groups(dims):
     b = partition(dims, 1)
     nbytes = [2 * r * c for r, c in dims]
     total = sum(nbytes)
-    first = max(64 << 20, total // 128)
+    first = 64 << 20
     assert len(b) - 1 <= 32
     for lo, hi in zip(b[:-2], b[1:-1]):
         assert sum(nbytes[lo:hi]) >= first
