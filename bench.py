@@ -35,12 +35,12 @@ UNIT = "TFLOP/s"
 NOMINAL_BF16_TFLOPS = 2250.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the GEMM stage: the ncu
-# capture of one Llama-8B layer's GEMM on CTA pairs (547.5 MB read + 410.5 MB written for
+# capture of one Llama-8B layer's GEMM on CTA pairs (631.8 MB read + 413.2 MB written for
 # 1.735e12 useful FLOPs); a launch of the full workload covers several layers, so its traffic is
 # this ratio times the useful FLOPs of that launch.  Valid only for the stage kernels' source it
 # was measured on (ns_stage.cuh, gemm_pair.cuh and ptx.cuh).
-PROFILED_TRAFFIC = {"kernel_sha256_prefix": "23cd5b6c8c04e86e", "workload": "llama8b",
-                    "gemm_bytes_per_useful_flop": 0.9580e9 / 1.735e12}
+PROFILED_TRAFFIC = {"kernel_sha256_prefix": "eee49fdfaf9de58a", "workload": "llama8b",
+                    "gemm_bytes_per_useful_flop": 1.0450e9 / 1.735e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

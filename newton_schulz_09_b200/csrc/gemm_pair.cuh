@@ -42,8 +42,6 @@ constexpr uint32_t kG2TemptyArrivals = 2 * 4;  // one per epilogue warp of both 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNsThreads, 1)
     gemm_pair_kernel(const __grid_constant__ NsParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
   using E = __nv_bfloat16;
   constexpr int BK = 64;          // K elements per stage (one 128-byte row)
   constexpr int MMA_K = 16;       // K per UMMA instruction
@@ -93,6 +91,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNsThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Barriers and TMEM were set up without touching global memory, while the
+  // previous kernel in the stream may still run (no CTA of another stage
+  // kernel fits beside this one's shared memory, so the TMEM is free); from
+  // here on its results are needed.
+  griddep_wait();
+  griddep_launch_dependents();
 
   bool ok = true;
   if (warp == 0) {

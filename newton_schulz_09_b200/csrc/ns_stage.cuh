@@ -371,8 +371,6 @@ __device__ __forceinline__ bool run_epilogue(const NsParams& p, uint32_t tmem_ba
 // ======================================================================
 template <int kMode, typename E>
 __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_constant__ NsParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
   constexpr int EB = static_cast<int>(sizeof(E));
   constexpr int BK = 128 / EB;              // K elements per stage (one 128-byte row)
   constexpr int MMA_K = 32 / EB;            // K per UMMA instruction
@@ -426,6 +424,12 @@ __global__ void __launch_bounds__(kNsThreads, 1) ns_stage_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Barriers and TMEM were set up without touching global memory, while the
+  // previous kernel in the stream may still run (no CTA of another stage
+  // kernel fits beside this one's shared memory, so the TMEM is free); from
+  // here on its results are needed.
+  griddep_wait();
+  griddep_launch_dependents();
 
   bool ok = true;
   if (warp == 0) {

@@ -19,12 +19,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // ------------------------------------------------ programmatic dependent launch
-// Every kernel of the library starts with these two: wait until the grids it
-// depends on (the previous kernel in the stream) have completed and their
-// memory is visible -- a no-op for a grid launched without programmatic
-// stream serialization -- then let the next grid in the stream be scheduled.
-// The next grid's CTAs thus launch while this one runs, and wait at their own
-// griddep_wait() before touching memory.
+// Every kernel of the library calls these two before it touches global memory
+// (the stage kernels after setting up their barriers and TMEM, the others
+// first thing): wait until the grids it depends on (the previous kernel in
+// the stream) have completed and their memory is visible -- a no-op for a
+// grid launched without programmatic stream serialization -- then let the
+// next grid in the stream be scheduled.  The next grid's CTAs thus launch
+// while this one runs, and wait at their own griddep_wait().
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -63,8 +63,6 @@ __device__ __forceinline__ Tile256 decode_tile256(const NsParams& p, int t) {
 // The epilogue adds cb A, read back from A's tile, and stores P like A.
 template <typename E, int kMode = kSyrk>
 __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_constant__ NsParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
   constexpr int EB = static_cast<int>(sizeof(E));
   constexpr int BK = 128 / EB;
   constexpr int MMA_K = 32 / EB;
@@ -111,6 +109,12 @@ __global__ void __launch_bounds__(kNsThreads, 1) syrk256_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Barriers and TMEM were set up without touching global memory, while the
+  // previous kernel in the stream may still run (no CTA of another stage
+  // kernel fits beside this one's shared memory, so the TMEM is free); from
+  // here on its results are needed.
+  griddep_wait();
+  griddep_launch_dependents();
 
   bool ok = true;
   if (warp == 0) {
