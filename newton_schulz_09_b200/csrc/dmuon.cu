@@ -937,6 +937,7 @@ bool g_timing = false;
 struct Bracket {
   cudaEvent_t a, b;
   int kind;
+  bool own_a;     // a is this bracket's own event (not the previous bracket's b)
 };
 std::vector<Bracket> g_brackets;       // recorded, not yet harvested
 std::vector<cudaEvent_t> g_event_pool;
@@ -960,23 +961,44 @@ const char* const kKindNames[DMUON_KERNEL_KINDS] = {"dmuon prologue", "dmuon fin
                                                     "dmuon gemm",     "dmuon apply",    "dmuon adamw",
                                                     "dmuon clip",     "dmuon square"};
 
+// Inside a TimingChain (one group's launches, back to back on one stream,
+// nothing else enqueued between them) a bracket starts at the previous
+// bracket's end event: one event per launch instead of two.
+bool g_chain_active = false;
+cudaEvent_t g_chain_event = nullptr;
+cudaStream_t g_chain_stream = nullptr;
+struct TimingChain {
+  TimingChain() { g_chain_active = true; g_chain_event = nullptr; }
+  ~TimingChain() { g_chain_active = false; g_chain_event = nullptr; }
+};
+
 struct LaunchScope {
   cudaStream_t st;
   int kind;
   cudaEvent_t a = nullptr;
+  bool own_a = true;
   LaunchScope(cudaStream_t s, int k) : st(s), kind(k) {
     ++g_launches;
     nvtxRangePushA(kKindNames[k]);
     if (g_timing) {
-      a = pool_event();
-      cudaEventRecord(a, st);
+      if (g_chain_active && g_chain_event && g_chain_stream == st) {
+        a = g_chain_event;
+        own_a = false;
+      } else {
+        a = pool_event();
+        cudaEventRecord(a, st);
+      }
     }
   }
   ~LaunchScope() {
     if (a) {
       cudaEvent_t b = pool_event();
       cudaEventRecord(b, st);
-      g_brackets.push_back(Bracket{a, b, kind});
+      g_brackets.push_back(Bracket{a, b, kind, own_a});
+      if (g_chain_active) {
+        g_chain_event = b;
+        g_chain_stream = st;
+      }
     }
     nvtxRangePop();
   }
@@ -1024,6 +1046,7 @@ void launch_group(const Plan& P, const GroupPlan& g, const DeviceInfo& d, const 
                   cudaStream_t st) {
   const float lr = o.lr, wd = o.wd;
   const int steps = o.steps;
+  TimingChain chain;   // the group's launches follow one another on `st`
   ElemParams ep = elem_params<E>(P, g, o);
   ep.err = d.err;
   ep.wait_limit_ns = kWaitLimitNs;
@@ -2064,7 +2087,7 @@ int dmuon_stage_times(double* ms, int64_t* launches, int n, int reset) {
       g_kind_ms[br.kind] += t;
       g_kind_n[br.kind] += 1;
     }
-    g_event_pool.push_back(br.a);
+    if (br.own_a) g_event_pool.push_back(br.a);
     g_event_pool.push_back(br.b);
   }
   g_brackets.clear();
